@@ -1,0 +1,252 @@
+"""Plain fp64 CPU oracle for FlashNorm (RMSNorm followed by a linear layer).
+
+TEST INFRASTRUCTURE ONLY. This module is imported by the tests, by the graft
+smoke check and by the CPU-baseline leg of the benchmark. The library itself
+never imports it, calls it or falls back to it; it shares no code with the
+CUDA kernels (only the seeded input generator feeds both).
+
+Sources. The method is stated in prose in the abstract of "FlashNorm: Fast
+Normalization for Transformers" (arXiv 2407.09577; mlsanity paper page and
+arxivdaily page, section "Abstract"). The pages print no equation, so each
+function below states the plainest reading of that prose:
+
+* RMSNorm (the paper builds on "Root Mean Square Layer Normalization", listed
+  under "Builds on"): RMSNorm(x) = x / sqrt(mean(x^2) + eps) * g, the mean
+  taken over the d features of one row, eps inside the square root.
+* (i) weight folding: the gain g is folded into the next linear layer,
+  W* = diag(g) . W.
+* (ii) deferred normalization: the scalar 1/rms is applied to the output of
+  the matrix multiplication, y = (x . W*) * 1/sqrt(mean(x^2) + eps).
+* GLU feed-forward variant ("feed-forward networks with GLU variants"): the
+  deferred scale is applied to the gate and the up outputs before SiLU,
+  y = silu(z_gate) * z_up, silu(t) = t / (1 + exp(-t)).
+* Redundant-norm removal ("an RMSNorm followed by a linear layer followed by
+  another RMSNorm allows the first RMSNorm to be eliminated"): linear ->
+  RMSNorm replaces RMSNorm -> linear -> RMSNorm by the scale invariance of RMS.
+
+Everything is computed in float64 from inputs given as bf16 bit patterns; the
+only library primitive is numpy's float64 matrix product. No blocking, fusion
+or reordering beyond the formulas above.
+
+Every function here is pinned by the CPU tests (hand-worked golden cases,
+closed forms, invariants, brute force in exact arithmetic, and torch's own
+CPU RMSNorm / SiLU / bf16 conversion on the special cases they cover). None is
+"parity unpinned".
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+
+# ---------------------------------------------------------------------------
+# bf16 encoding (IEEE-754 binary32 truncated to 16 bits: 1 sign, 8 exponent,
+# 7 stored mantissa bits; 8 significant bits with the implicit one).
+# ---------------------------------------------------------------------------
+
+def bf16_to_f64(bits) -> np.ndarray:
+    """Decode bf16 bit patterns exactly to float64."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def f64_to_bf16(v) -> np.ndarray:
+    """Round float64 values to bf16 with round-to-nearest, ties to even.
+
+    Written from the definition: a finite value is rounded to a multiple of
+    its quantum, 2^(e-8) for |v| in [2^(e-1), 2^e) (8 significant bits), with
+    the quantum floored at 2^-133 (bf16 subnormals). np.rint rounds halfway
+    cases to the even integer, which is ties-to-even on the significand.
+    Magnitudes that round to 2^128 or beyond become infinities.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    finite = np.isfinite(v)
+    vf = np.where(finite, v, 0.0)
+    _, e = np.frexp(vf)
+    quantum = np.ldexp(1.0, np.maximum(e - 8, -133))
+    r = np.rint(vf / quantum) * quantum
+    with np.errstate(over="ignore"):
+        r32 = r.astype(np.float32)  # exact: r has at most 8 significant bits
+    bits = (r32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    out[...] = bits
+    nan = np.isnan(v)
+    out[nan] = np.uint16(0x7FC0)
+    posinf = np.isposinf(v)
+    neginf = np.isneginf(v)
+    out[posinf] = np.uint16(0x7F80)
+    out[neginf] = np.uint16(0xFF80)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm and the unfolded, undeferred chain (the plain definition).
+# ---------------------------------------------------------------------------
+
+def inv_rms(x: np.ndarray, eps: float) -> np.ndarray:
+    """Per-row 1 / sqrt(mean_i x_i^2 + eps), mean over the feature axis."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1)
+    return 1.0 / np.sqrt(ms + eps)
+
+
+def rmsnorm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    """RMSNorm(x) = x / sqrt(mean(x^2) + eps) * g, row-wise."""
+    x = np.asarray(x, dtype=np.float64)
+    return x * inv_rms(x, eps)[..., None] * np.asarray(g, dtype=np.float64)
+
+
+def norm_then_project(x, g, W, eps):
+    """The operation FlashNorm reformulates: RMSNorm(x) . W, W of shape [d, N]."""
+    return rmsnorm(x, g, eps) @ np.asarray(W, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# (i) Weight folding and (ii) deferred normalization.
+# ---------------------------------------------------------------------------
+
+def fold(W, g) -> np.ndarray:
+    """W* = diag(g) . W in float64 (row i of W scaled by g_i)."""
+    return np.asarray(g, dtype=np.float64)[:, None] * np.asarray(W, dtype=np.float64)
+
+
+def fold_bf16(w_bits, g_bits) -> np.ndarray:
+    """W* rounded once to bf16: bits of RNE(g_i * W_ij), same [d, N] shape as W."""
+    return f64_to_bf16(fold(bf16_to_f64(w_bits), bf16_to_f64(g_bits)))
+
+
+def deferred(x, Wstar, eps):
+    """(x . W*) scaled per row by 1/sqrt(mean(x^2) + eps): the reformulated form."""
+    x = np.asarray(x, dtype=np.float64)
+    return (x @ np.asarray(Wstar, dtype=np.float64)) * inv_rms(x, eps)[:, None]
+
+
+# ---------------------------------------------------------------------------
+# GLU (SwiGLU) feed-forward variant. W has 2F columns: gate = [0, F), up = [F, 2F).
+# ---------------------------------------------------------------------------
+
+def silu(t):
+    """SiLU(t) = t / (1 + exp(-t))."""
+    t = np.asarray(t, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return t / (1.0 + np.exp(-t))
+
+
+def glu_norm_then_project(x, g, W_gu, eps):
+    """silu(z_gate) * z_up with z = RMSNorm(x) . W (unfolded, undeferred)."""
+    z = norm_then_project(x, g, W_gu, eps)
+    F = z.shape[1] // 2
+    return silu(z[:, :F]) * z[:, F:]
+
+
+def glu_deferred(x, Wstar_gu, eps):
+    """silu(r * (x . W*_gate)) * (r * (x . W*_up)), r = 1/rms(x): scale before SiLU."""
+    x = np.asarray(x, dtype=np.float64)
+    r = inv_rms(x, eps)[:, None]
+    z = x @ np.asarray(Wstar_gu, dtype=np.float64)
+    F = z.shape[1] // 2
+    return silu(r * z[:, :F]) * (r * z[:, F:])
+
+
+# ---------------------------------------------------------------------------
+# Redundant-norm removal: RMSNorm -> linear -> RMSNorm becomes linear -> RMSNorm.
+# The second norm acts per head of width head_dim with a shared gain g2.
+# ---------------------------------------------------------------------------
+
+def _per_head_rmsnorm(v, g2, eps2, head_dim):
+    M, N = v.shape
+    vh = v.reshape(M, N // head_dim, head_dim)
+    return rmsnorm(vh, g2, eps2).reshape(M, N)
+
+
+def postnorm_full(x, g1, W, g2, eps1, eps2, head_dim):
+    """The full chain: per-head RMSNorm(RMSNorm(x; g1) . W; g2). Keeps the first norm."""
+    v = norm_then_project(x, g1, W, eps1)
+    return _per_head_rmsnorm(v, g2, eps2, head_dim)
+
+
+def postnorm_elided(x, Wstar1, g2, eps2, head_dim):
+    """The first norm dropped: per-head RMSNorm(x . W*1; g2), with g1 folded into W*1."""
+    u = np.asarray(x, dtype=np.float64) @ np.asarray(Wstar1, dtype=np.float64)
+    return _per_head_rmsnorm(u, g2, eps2, head_dim)
+
+
+def postnorm_elided_exact_eps(x, Wstar1, g2, eps1, eps2, head_dim):
+    """What the full chain equals when eps1, eps2 > 0, written through u = x . W*1.
+
+    With v = u * r1 and r1 = 1/sqrt(ms_x + eps1), mean(v^2) = r1^2 mean(u^2), so
+    v / sqrt(mean(v^2) + eps2) = u / sqrt(mean(u^2) + eps2 (ms_x + eps1)).
+    The elided form drops the eps2 (ms_x + eps1) correction; it is exact at eps = 0.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    u = x @ np.asarray(Wstar1, dtype=np.float64)
+    M, N = u.shape
+    uh = u.reshape(M, N // head_dim, head_dim)
+    ms_x = np.mean(x * x, axis=-1)
+    denom = np.sqrt(np.mean(uh * uh, axis=-1) + eps2 * (ms_x + eps1)[:, None])
+    return (uh / denom[..., None] * np.asarray(g2, dtype=np.float64)).reshape(M, N)
+
+
+# ---------------------------------------------------------------------------
+# The unfused norm-then-project pipeline the pages compare against: the norm
+# output is materialised in bf16 (one rounding), then multiplied by W.
+# ---------------------------------------------------------------------------
+
+def unfused_norm_then_project(x, g, W, eps):
+    """bf16(RMSNorm(x; g)) . W, the two-kernel baseline with its bf16 intermediate."""
+    xn = bf16_to_f64(f64_to_bf16(rmsnorm(x, g, eps)))
+    return xn @ np.asarray(W, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Convenience wrappers on bf16 bit arrays (what the tests and the bench feed).
+# ---------------------------------------------------------------------------
+
+def reference_output(kind: str, bits: dict, eps: float, *, eps2: float = 0.0, head_dim: int = 0,
+                     rows=None) -> np.ndarray:
+    """Oracle output of a workload from its bf16 input bits, optionally for a subset of rows.
+
+    kind "linear": RMSNorm(x; g) . W.   kind "glu": silu(z_gate) * z_up.
+    kind "postnorm": the full RMSNorm -> linear -> per-head RMSNorm chain with
+    g1 = bits["g"], g2 = bits["g2"], eps1 = eps.
+    """
+    x = bf16_to_f64(bits["x"])
+    if rows is not None:
+        x = x[rows]
+    g = bf16_to_f64(bits["g"])
+    W = bf16_to_f64(bits["w"])
+    if kind == "linear":
+        return norm_then_project(x, g, W, eps)
+    if kind == "glu":
+        return glu_norm_then_project(x, g, W, eps)
+    if kind == "postnorm":
+        return postnorm_full(x, g, W, bf16_to_f64(bits["g2"]), eps, eps2, head_dim)
+    raise ValueError(kind)
+
+
+def exact_operand_output(kind: str, bits: dict, wstar_bits, eps: float, *, eps2: float = 0.0,
+                         head_dim: int = 0, rows=None) -> np.ndarray:
+    """Oracle of the reformulated form on the bf16 W* (given as [d, N] bits).
+
+    Used for fp32 outputs, where the fold's own bf16 rounding of W* would
+    otherwise dominate the comparison.
+    """
+    x = bf16_to_f64(bits["x"])
+    if rows is not None:
+        x = x[rows]
+    Ws = bf16_to_f64(wstar_bits)
+    if kind == "linear":
+        return deferred(x, Ws, eps)
+    if kind == "glu":
+        return glu_deferred(x, Ws, eps)
+    if kind == "postnorm":
+        return postnorm_elided(x, Ws, bf16_to_f64(bits["g2"]), eps2, head_dim)
+    raise ValueError(kind)
+
+
+def rel_err(y, y_ref) -> float:
+    """max |y - y_ref| / max |y_ref|, the parity metric."""
+    y = np.asarray(y, dtype=np.float64)
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    denom = np.max(np.abs(y_ref))
+    return float(np.max(np.abs(y - y_ref)) / denom) if denom > 0 else float(np.max(np.abs(y - y_ref)))

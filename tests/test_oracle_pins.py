@@ -1,0 +1,349 @@
+"""Pins for the fp64 oracle: it is checked against things other than itself.
+
+* hand-worked golden cases (tests/golden/hand_worked.json), derived from the
+  definitions in the FlashNorm abstract by hand;
+* torch's own CPU RMSNorm, SiLU and float32 -> bf16 conversion on the special
+  cases those library routines cover;
+* closed forms (constant rows, d = 1, identity weights, GLU with proportional
+  gate and up columns);
+* invariants the abstract states: folded == unfolded ("exact reformulation"),
+  scale invariance of RMS, and the redundant-norm identity;
+* brute force in exact rational arithmetic (50-digit square roots) on tiny inputs.
+
+The last test plants plausible mistakes in the oracle (on the CPU) and checks
+that every one of them is caught by at least one pin.
+"""
+
+import json
+import os
+from decimal import Decimal, getcontext
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import flashnorm_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_worked.json")
+
+
+def _arr(v):
+    return np.asarray(v, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Pin checks. Each returns a list of failure strings (empty = pass), so the
+# mutation test can run them against a deliberately broken oracle.
+# ---------------------------------------------------------------------------
+
+def check_golden(O):
+    fails = []
+    with open(GOLDEN) as f:
+        data = json.load(f)
+    for c in data["cases"]:
+        op = c["op"]
+        if op == "norm_then_project":
+            y = O.norm_then_project(_arr(c["x"]), _arr(c["g"]), _arr(c["W"]), c["eps"])
+        elif op == "deferred_of_fold":
+            y = O.deferred(_arr(c["x"]), O.fold(_arr(c["W"]), _arr(c["g"])), c["eps"])
+        elif op == "unfused_norm_then_project":
+            y = O.unfused_norm_then_project(_arr(c["x"]), _arr(c["g"]), _arr(c["W"]), c["eps"])
+        elif op == "glu_norm_then_project":
+            y = O.glu_norm_then_project(_arr(c["x"]), _arr(c["g"]), _arr(c["W"]), c["eps"])
+        elif op == "postnorm_full":
+            y = O.postnorm_full(_arr(c["x"]), _arr(c["g"]), _arr(c["W"]), _arr(c["g2"]), c["eps"],
+                                c["eps2"], c["head_dim"])
+        elif op == "postnorm_elided_exact_eps":
+            y = O.postnorm_elided_exact_eps(_arr(c["x"]), _arr(c["Wstar"]), _arr(c["g2"]), c["eps"],
+                                            c["eps2"], c["head_dim"])
+        elif op == "postnorm_elided":
+            y = O.postnorm_elided(_arr(c["x"]), _arr(c["Wstar"]), _arr(c["g2"]), c["eps2"], c["head_dim"])
+        else:
+            raise AssertionError(op)
+        exp = _arr(c["expected"])
+        if y.shape != exp.shape or not np.allclose(y, exp, rtol=1e-14, atol=1e-14):
+            fails.append(f"golden {c['name']}: got {y.tolist()} expected {exp.tolist()}")
+    for c in data["fold_bits"]["cases"]:
+        g = np.array([int(c["g"], 16)], dtype=np.uint16)
+        w = np.array([[int(c["w"], 16)]], dtype=np.uint16)
+        got = int(O.fold_bf16(w, g)[0, 0])
+        if got != int(c["wstar"], 16):
+            fails.append(f"fold bits g={c['g']} w={c['w']}: got {got:#06x} expected {c['wstar']}")
+    return fails
+
+
+def check_torch_rmsnorm(O):
+    rng = np.random.default_rng(1)
+    fails = []
+    for d, eps in ((1, 1e-5), (7, 0.0), (64, 1e-6), (576, 1e-5)):
+        x = rng.standard_normal((5, d)) * np.exp(rng.uniform(-3, 3, (5, 1)))
+        g = rng.uniform(0.5, 1.5, d)
+        ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (d,), torch.from_numpy(g), eps).numpy()
+        if not np.allclose(O.rmsnorm(x, g, eps), ref, rtol=1e-13, atol=0):
+            fails.append(f"rmsnorm vs torch d={d}")
+    return fails
+
+
+def check_torch_silu(O):
+    t = np.linspace(-40, 40, 1001)
+    ref = torch.nn.functional.silu(torch.from_numpy(t)).numpy()
+    return [] if np.allclose(O.silu(t), ref, rtol=1e-14, atol=1e-300) else ["silu vs torch"]
+
+
+def check_torch_bf16(O):
+    """fp32-representable values: RNE to bf16 must equal torch's fp32 -> bf16 cast."""
+    rng = np.random.default_rng(2)
+    bits32 = rng.integers(0, 2**32, size=200000, dtype=np.uint64).astype(np.uint32)
+    # add exact ties and near-ties around a few exponents
+    base = rng.integers(0, 2**16, size=4000, dtype=np.uint64).astype(np.uint32) << np.uint32(16)
+    ties = np.concatenate([base | np.uint32(0x8000), base | np.uint32(0x7FFF), base | np.uint32(0x8001)])
+    bits32 = np.concatenate([bits32, ties])
+    f = bits32.view(np.float32)
+    f = f[np.isfinite(f) & (np.abs(f) < 3.0e38)]
+    ref = torch.from_numpy(f.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = O.f64_to_bf16(f.astype(np.float64))
+    bad = np.nonzero(got != ref)[0]
+    return [] if bad.size == 0 else [f"bf16 RNE vs torch: {bad.size} mismatches, e.g. {f[bad[0]]!r}"]
+
+
+def check_closed_forms(O):
+    fails = []
+    rng = np.random.default_rng(3)
+    # constant row x = c * 1: y_j = c / sqrt(c^2 + eps) * sum_i g_i W_ij
+    d, N, c, eps = 16, 5, -0.7, 1e-3
+    g = rng.uniform(0.5, 1.5, d)
+    W = rng.standard_normal((d, N))
+    y = O.norm_then_project(np.full((1, d), c), g, W, eps)
+    exp = c / np.sqrt(c * c + eps) * (g @ W)
+    if not np.allclose(y[0], exp, rtol=1e-13):
+        fails.append("constant row closed form")
+    # d = 1: y = x / sqrt(x^2 + eps) * g * W
+    x = np.array([[2.5], [-0.25]])
+    y = O.norm_then_project(x, np.array([1.25]), np.array([[3.0, -2.0]]), 0.5)
+    exp = x / np.sqrt(x * x + 0.5) * 1.25 * np.array([[3.0, -2.0]])
+    if not np.allclose(y, exp, rtol=1e-14):
+        fails.append("d=1 closed form")
+    # W = I, g = 1, eps = 0: mean(y^2) = 1 for every row
+    x = rng.standard_normal((4, 32)) * 7.0
+    y = O.norm_then_project(x, np.ones(32), np.eye(32), 0.0)
+    if not np.allclose(np.mean(y * y, axis=1), 1.0, rtol=1e-14):
+        fails.append("identity weights: mean(y^2) != 1")
+    # GLU with up = 2 * gate: y = silu(z) * 2z, z = the linear output on the gate columns
+    Wg = rng.standard_normal((32, 6))
+    x = rng.standard_normal((3, 32))
+    gg = rng.uniform(0.5, 1.5, 32)
+    z = O.norm_then_project(x, gg, Wg, 1e-5)
+    y = O.glu_norm_then_project(x, gg, np.concatenate([Wg, 2 * Wg], axis=1), 1e-5)
+    if not np.allclose(y, 2 * z * (z / (1 + np.exp(-z))), rtol=1e-13):
+        fails.append("GLU up = 2*gate closed form (gate/up order)")
+    return fails
+
+
+def check_invariants(O):
+    fails = []
+    rng = np.random.default_rng(4)
+    M, d, N = 6, 40, 12
+    x = rng.standard_normal((M, d)) * np.exp(rng.uniform(-2, 2, (M, 1)))
+    g = rng.uniform(0.5, 1.5, d)
+    W = rng.standard_normal((d, N)) / np.sqrt(d)
+    eps = 1e-5
+    # (i)+(ii): folded, deferred form equals the unfolded chain
+    if not np.allclose(O.deferred(x, O.fold(W, g), eps), O.norm_then_project(x, g, W, eps), rtol=1e-12, atol=0):
+        fails.append("folded deferred != unfolded")
+    Wgu = rng.standard_normal((d, 2 * N)) / np.sqrt(d)
+    if not np.allclose(O.glu_deferred(x, O.fold(Wgu, g), eps), O.glu_norm_then_project(x, g, Wgu, eps),
+                       rtol=1e-12, atol=1e-300):
+        fails.append("GLU folded deferred != unfolded")
+    # scale invariance at eps = 0; closed form a x / sqrt(a^2 ms + eps) with eps > 0
+    for a in (1e-3, 0.37, 1e3):
+        if not np.allclose(O.norm_then_project(a * x, g, W, 0.0), O.norm_then_project(x, g, W, 0.0),
+                           rtol=1e-12, atol=0):
+            fails.append(f"scale invariance a={a}")
+        ms = np.mean(x * x, axis=1, keepdims=True)
+        if not np.allclose(O.rmsnorm(a * x, g, eps), a * x / np.sqrt(a * a * ms + eps) * g, rtol=1e-12):
+            fails.append(f"eps>0 scaling closed form a={a}")
+    # redundant norm: full chain == elided at eps = 0; == eps-corrected form at eps > 0
+    hd = 4
+    g2 = rng.uniform(0.5, 1.5, hd)
+    full0 = O.postnorm_full(x, g, W, g2, 0.0, 0.0, hd)
+    if not np.allclose(full0, O.postnorm_elided(x, O.fold(W, g), g2, 0.0, hd), rtol=1e-12, atol=0):
+        fails.append("postnorm identity at eps=0")
+    full1 = O.postnorm_full(x, g, W, g2, 1e-2, 3e-2, hd)
+    if not np.allclose(full1, O.postnorm_elided_exact_eps(x, O.fold(W, g), g2, 1e-2, 3e-2, hd),
+                       rtol=1e-12, atol=0):
+        fails.append("postnorm identity with eps correction")
+    return fails
+
+
+def _dsqrt(fr: Fraction) -> Decimal:
+    return (Decimal(fr.numerator) / Decimal(fr.denominator)).sqrt()
+
+
+def _brute_linear(x, g, W, eps):
+    """RMSNorm -> linear in exact rationals, square root to 50 digits, pure Python loops."""
+    out = []
+    for row in x:
+        d = len(row)
+        ms = sum(Fraction(v) * Fraction(v) for v in row) / d + Fraction(eps)
+        inv = Decimal(1) / _dsqrt(ms)
+        n = [Decimal(Fraction(row[i]).numerator) / Decimal(Fraction(row[i]).denominator) * inv
+             * (Decimal(Fraction(g[i]).numerator) / Decimal(Fraction(g[i]).denominator)) for i in range(d)]
+        outrow = []
+        for j in range(len(W[0])):
+            acc = Decimal(0)
+            for i in range(d):
+                w = Fraction(W[i][j])
+                acc += n[i] * (Decimal(w.numerator) / Decimal(w.denominator))
+            outrow.append(float(acc))
+        out.append(outrow)
+    return np.array(out)
+
+
+def check_brute_force(O):
+    getcontext().prec = 50
+    rng = np.random.default_rng(5)
+    fails = []
+    for trial in range(12):
+        M, d, N = rng.integers(1, 4), rng.integers(1, 9), rng.integers(1, 5)
+        # dyadic values (exact in binary) so Fraction sees the very numbers numpy sees
+        x = rng.integers(-64, 65, (M, d)) / 16.0
+        x[0, 0] = 1.5  # no all-zero row
+        g = rng.integers(8, 25, d) / 16.0
+        W = rng.integers(-32, 33, (d, N)) / 32.0
+        eps = float(rng.choice([0.0, 1.0 / 1024, 0.5]))
+        if eps == 0.0 and np.any(np.all(x == 0, axis=1)):
+            continue
+        exp = _brute_linear(x.tolist(), g.tolist(), W.tolist(), eps)
+        y = O.norm_then_project(x, g, W, eps)
+        scale = max(1.0, float(np.max(np.abs(exp))))
+        if np.max(np.abs(y - exp)) > 1e-14 * scale:
+            fails.append(f"brute force trial {trial}")
+    return fails
+
+
+ALL_CHECKS = [check_golden, check_torch_rmsnorm, check_torch_silu, check_torch_bf16,
+              check_closed_forms, check_invariants, check_brute_force]
+
+
+@pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
+def test_oracle_pin(check):
+    fails = check(O)
+    assert not fails, fails
+
+
+def test_reference_output_wrappers():
+    """The bit-array wrappers route to the pinned functions with the right operands."""
+    from flashnorm_inputs import Workload
+
+    wl = Workload("t", "postnorm", 5, 24, 8, 1e-6, head_dim=4, eps2=1e-6, seed=7)
+    bits = wl.draw()
+    x, g, W, g2 = (O.bf16_to_f64(bits[k]) for k in ("x", "g", "w", "g2"))
+    y = O.reference_output("postnorm", bits, 1e-6, eps2=1e-6, head_dim=4)
+    assert np.allclose(y, O.postnorm_full(x, g, W, g2, 1e-6, 1e-6, 4), rtol=1e-15)
+    ws = O.fold_bf16(bits["w"], bits["g"])
+    y2 = O.exact_operand_output("postnorm", bits, ws, 1e-6, eps2=1e-6, head_dim=4, rows=[1, 3])
+    assert np.allclose(y2, O.postnorm_elided(x[[1, 3]], O.bf16_to_f64(ws), g2, 1e-6, 4), rtol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# Planted mistakes: each must be caught by at least one pin.
+# ---------------------------------------------------------------------------
+
+def _mut_mean_d_minus_1(x, eps):
+    x = np.asarray(x, dtype=np.float64)
+    n = max(x.shape[-1] - 1, 1)
+    return 1.0 / np.sqrt(np.sum(x * x, axis=-1) / n + eps)
+
+
+def _mut_eps_outside(x, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return 1.0 / (np.sqrt(np.mean(x * x, axis=-1)) + eps)
+
+
+def _mut_rms_not_inverted(x, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return np.sqrt(np.mean(x * x, axis=-1) + eps)
+
+
+def _mut_drop_gain(x, g, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return x * O.inv_rms(x, eps)[..., None]
+
+
+def _mut_fold_columns(W, g):
+    W = np.asarray(W, dtype=np.float64)
+    return W * np.resize(np.asarray(g, dtype=np.float64), W.shape[1])[None, :]
+
+
+def _mut_silu_sign(t):
+    t = np.asarray(t, dtype=np.float64)
+    return t / (1.0 + np.exp(t))
+
+
+def _mut_glu_swap(x, g, W_gu, eps):
+    z = O.norm_then_project(x, g, W_gu, eps)
+    F = z.shape[1] // 2
+    return O.silu(z[:, F:]) * z[:, :F]
+
+
+def _mut_glu_scale_after(x, Wstar_gu, eps):
+    x = np.asarray(x, dtype=np.float64)
+    r = O.inv_rms(x, eps)[:, None]
+    z = x @ Wstar_gu
+    F = z.shape[1] // 2
+    return r * r * O.silu(z[:, :F]) * z[:, F:]
+
+
+def _mut_rne_truncate(v):
+    v = np.asarray(v, dtype=np.float64).astype(np.float32)
+    return (v.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+def _mut_rne_ties_away(v):
+    v = np.asarray(v, dtype=np.float64)
+    _, e = np.frexp(v)
+    q = np.ldexp(1.0, np.maximum(e - 8, -133))
+    r = np.sign(v) * np.floor(np.abs(v) / q + 0.5) * q
+    return (r.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+def _mut_transpose_product(x, g, W, eps):
+    n = O.rmsnorm(x, g, eps)
+    W = np.asarray(W, dtype=np.float64)
+    return n @ W if W.shape[0] != W.shape[1] else n @ W.T
+
+
+def _mut_postnorm_whole_row(v, g2, eps2, head_dim):
+    M, N = v.shape
+    return O.rmsnorm(v, np.tile(g2, N // head_dim), eps2)
+
+
+MUTANTS = {
+    "mean over d-1": ("inv_rms", _mut_mean_d_minus_1),
+    "eps outside sqrt": ("inv_rms", _mut_eps_outside),
+    "rms not inverted": ("inv_rms", _mut_rms_not_inverted),
+    "gain dropped": ("rmsnorm", _mut_drop_gain),
+    "fold scales columns": ("fold", _mut_fold_columns),
+    "silu sign": ("silu", _mut_silu_sign),
+    "gate/up swapped": ("glu_norm_then_project", _mut_glu_swap),
+    "deferred GLU scale after silu": ("glu_deferred", _mut_glu_scale_after),
+    "bf16 truncation": ("f64_to_bf16", _mut_rne_truncate),
+    "bf16 ties away": ("f64_to_bf16", _mut_rne_ties_away),
+    "W transposed": ("norm_then_project", _mut_transpose_product),
+    "post-norm over whole row": ("_per_head_rmsnorm", _mut_postnorm_whole_row),
+}
+
+
+@pytest.mark.parametrize("name", list(MUTANTS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(O, attr, fn)
+    caught = []
+    for check in ALL_CHECKS:
+        try:
+            if check(O):
+                caught.append(check.__name__)
+        except Exception as e:  # a crash also counts as caught
+            caught.append(f"{check.__name__} raised {type(e).__name__}")
+    assert caught, f"planted mistake '{name}' passed every pin"
