@@ -1,0 +1,161 @@
+/*
+ * flashnorm.h — C ABI of the FlashNorm RMSNorm -> linear library for NVIDIA B200 (sm_100a).
+ *
+ * FlashNorm ("FlashNorm: Fast Normalization for Transformers", Abstract) is an exact reformulation of
+ * RMSNorm followed by a linear layer:
+ *   (i)  the norm gain g is folded into the weights offline:   W* = diag(g) . W
+ *   (ii) the scalar RMS normalisation is deferred to the matmul output:
+ *            y = (x . W*) * 1 / sqrt(mean(x^2) + eps)
+ *        so the row sum of squares and the contraction run at the same time (here: in one kernel,
+ *        on different warps, joined by shared-memory barriers).
+ * It extends to GLU feed-forward layers (the deferred scale goes onto the gate and the up outputs
+ * before SiLU) and to RMSNorm -> linear -> RMSNorm, where the first norm is dropped by the scale
+ * invariance of RMS (same abstract).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are caller-owned DEVICE memory on the current device; the library never
+ *     allocates, frees or keeps them. Pointers must be 16-byte aligned.
+ *   - Element types: activations, weights, gains and the unfused intermediate are bf16 (stored as
+ *     uint16 bit patterns); outputs are bf16 or fp32 as `out_dtype` says. All arithmetic is fp32
+ *     with one round-to-nearest-even conversion per bf16 result.
+ *   - Layouts are row-major. x is [M, d]; y is [M, N] (linear, post-norm) or [M, F] (GLU).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Every call only
+ *     enqueues work on it and returns; nothing synchronises except flashnorm_check_device_error.
+ *   - Arguments are validated before anything is launched; a rejected call launches nothing and
+ *     returns FN_ERR_INVALID_ARG / FN_ERR_ALIGN / FN_ERR_UNSUPPORTED with a message available from
+ *     flashnorm_last_error(). A failed launch returns FN_ERR_CUDA.
+ *   - M == 0 is a valid empty call: nothing is launched and FN_OK is returned.
+ *   - Outputs must not overlap inputs. Results are deterministic (no atomics, no split reductions),
+ *     so identical calls give bitwise identical outputs.
+ *   - Every wait inside a kernel is bounded in time; a wait that runs out records FN_ERR_TIMEOUT in a
+ *     device-side status word (read and cleared by flashnorm_check_device_error) and the kernel
+ *     returns early instead of hanging.
+ */
+#ifndef FLASHNORM_H
+#define FLASHNORM_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FN_API __attribute__((visibility("default")))
+#else
+#define FN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FN_OK = 0,
+  FN_ERR_INVALID_ARG = 1, /* a size, pointer or flag is out of range */
+  FN_ERR_UNSUPPORTED = 2, /* a legal request this build has no kernel for (e.g. head_dim > 512) */
+  FN_ERR_ALIGN = 3,       /* a pointer or a leading dimension is not 16-byte aligned */
+  FN_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (message has the CUDA error) */
+  FN_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out (see flashnorm_check_device_error) */
+} fn_status;
+
+typedef enum { FN_BF16 = 0, FN_F32 = 1 } fn_dtype;
+
+/* Which kernel family a projection runs on. AUTO: the GEMV path for M <= FN_DECODE_MAX_M, the
+ * tensor-core path otherwise. */
+typedef enum { FN_PATH_AUTO = 0, FN_PATH_TENSOR = 1, FN_PATH_GEMV = 2 } fn_path;
+
+#define FN_DECODE_MAX_M 16
+/* GLU weights are stored gate/up interleaved in blocks of this many output columns (see fold). */
+#define FN_GLU_BLOCK 16
+
+/*
+ * flashnorm_fold_weights — step (i), weight folding (FlashNorm Abstract, item i: the norm gain is
+ * multiplied into the projection that follows, so the norm keeps no weights of its own).
+ *   W      bf16 [d, N] row-major, the unfolded projection (y = x . W).
+ *   g      bf16 [d], the RMSNorm gain.
+ *   Wstar  bf16 [N, d] output: Wstar[n][k] = RNE_bf16(g[k] * W[k][n]), i.e. W* stored K-major (its
+ *          transpose, row-major), the operand layout every projection kernel reads. g[k]*W[k][n] is
+ *          exact in fp32, so each element is rounded exactly once.
+ *   glu    0: N output columns in order. 1: N = 2F columns, gate = W[:, 0:F), up = W[:, F:2F); the
+ *          output rows are interleaved in blocks of FN_GLU_BLOCK: rows [32b, 32b+16) hold gate
+ *          columns [16b, 16b+16) and rows [32b+16, 32b+32) the matching up columns. Needs F % 16 == 0.
+ * Folding with g = 1 is an exact transpose; that is how the unfused path gets its K-major W.
+ * Constraints: d >= 8, d % 8 == 0, N >= 8, N % 8 == 0.
+ */
+FN_API fn_status flashnorm_fold_weights(const void* W, const void* g, void* Wstar, int64_t d, int64_t N,
+                                 int glu, void* stream);
+
+/*
+ * flashnorm_linear — steps (i)+(ii): y = (x . W*) * 1/sqrt(mean(x^2) + eps) (FlashNorm Abstract).
+ *   x      bf16 [M, d]; Wstar bf16 [N, d] from flashnorm_fold_weights(glu = 0); y [M, N] of out_dtype.
+ *   For M > 16 one persistent tcgen05 kernel computes x . W* into tensor memory while a separate
+ *   warpgroup sums x^2 per row from the same shared-memory x tiles; the epilogue waits for both and
+ *   scales each row. For M <= 16 a bandwidth-bound GEMV kernel streams W* once.
+ * Constraints: M >= 0, d % 8 == 0, N % 8 == 0, eps >= 0 and finite.
+ */
+FN_API fn_status flashnorm_linear(const void* x, const void* Wstar, void* y, int64_t M, int64_t d, int64_t N,
+                           float eps, int out_dtype, void* stream);
+
+/* Same as flashnorm_linear with the kernel family chosen explicitly (fn_path). */
+FN_API fn_status flashnorm_linear_ex(const void* x, const void* Wstar, void* y, int64_t M, int64_t d, int64_t N,
+                              float eps, int out_dtype, int path, void* stream);
+
+/*
+ * flashnorm_glu — the GLU feed-forward variant (FlashNorm Abstract: the techniques carry over to
+ * gated feed-forward layers): with r = 1/sqrt(mean(x^2) + eps), z = x . W*,
+ *     y[m, j] = silu(r * z[m, gate j]) * (r * z[m, up j]),   silu(t) = t / (1 + exp(-t)).
+ *   x bf16 [M, d]; Wstar_gu bf16 [2F, d] from flashnorm_fold_weights(glu = 1); y [M, F] of out_dtype.
+ * Constraints: as flashnorm_linear, and F % 16 == 0.
+ */
+FN_API fn_status flashnorm_glu(const void* x, const void* Wstar_gu, void* y, int64_t M, int64_t d, int64_t F,
+                        float eps, int out_dtype, void* stream);
+
+FN_API fn_status flashnorm_glu_ex(const void* x, const void* Wstar_gu, void* y, int64_t M, int64_t d, int64_t F,
+                           float eps, int out_dtype, int path, void* stream);
+
+/*
+ * flashnorm_linear_postnorm — redundant-norm removal (FlashNorm Abstract: when a linear layer sits
+ * between two RMSNorms, RMS scale invariance makes the first one unnecessary):
+ *     u = x . W*   (the first norm's gain folded into W*, its 1/rms dropped),
+ *     y[m, h*hd + j] = u[m, h*hd + j] / sqrt(mean_j u[m, h*hd + j]^2 + eps2) * g2[j]
+ *   for each head h of width hd = head_dim.
+ *   x bf16 [M, d]; Wstar bf16 [N, d] (fold with glu = 0); g2 bf16 [head_dim]; y [M, N] of out_dtype.
+ * Constraints: d % 8 == 0, head_dim % 16 == 0, 16 <= head_dim <= 512, N % head_dim == 0, eps2 >= 0.
+ */
+FN_API fn_status flashnorm_linear_postnorm(const void* x, const void* Wstar, const void* g2, void* y, int64_t M,
+                                    int64_t d, int64_t N, int64_t head_dim, float eps2, int out_dtype,
+                                    void* stream);
+
+/*
+ * The unfused baseline the pages compare against (FlashNorm Abstract: its speedups are stated against a
+ * plain norm-then-project pipeline): kernel 1 writes xn = RNE_bf16(x * 1/sqrt(mean(x^2)+eps) * g), kernel 2 runs the
+ * same tensor-core GEMM on xn with no scale. Kept for measuring what folding + deferral buy.
+ *
+ * flashnorm_rmsnorm: x bf16 [M, d], g bf16 [d] -> xn bf16 [M, d] (caller-owned).
+ * flashnorm_linear_unfused: W_kmajor bf16 [N, d] is the UNFOLDED weight transposed (fold with g = 1);
+ *   xn_ws bf16 [M, d] is caller-owned scratch that receives the normalised activations.
+ * flashnorm_glu_unfused: the same for GLU; W_kmajor_gu from fold(glu = 1, g = 1); y [M, F].
+ */
+FN_API fn_status flashnorm_rmsnorm(const void* x, const void* g, void* xn, int64_t M, int64_t d, float eps,
+                            void* stream);
+FN_API fn_status flashnorm_linear_unfused(const void* x, const void* g, const void* W_kmajor, void* xn_ws, void* y,
+                                   int64_t M, int64_t d, int64_t N, float eps, int out_dtype, void* stream);
+FN_API fn_status flashnorm_glu_unfused(const void* x, const void* g, const void* W_kmajor_gu, void* xn_ws, void* y,
+                                int64_t M, int64_t d, int64_t F, float eps, int out_dtype, void* stream);
+
+/*
+ * flashnorm_check_device_error — synchronises `stream`, then reads and clears the device-side status
+ * word of the current device. Returns FN_ERR_TIMEOUT if any kernel of this library gave up on a bounded
+ * wait since the last check, FN_ERR_CUDA if the synchronisation itself failed, FN_OK otherwise.
+ */
+FN_API fn_status flashnorm_check_device_error(void* stream);
+
+/* Static description of a status code. */
+FN_API const char* flashnorm_status_string(int status);
+/* Detail of the most recent failed call on this host thread ("" if none). */
+FN_API const char* flashnorm_last_error(void);
+/* ABI version of this library: major * 10000 + minor * 100 + patch. */
+FN_API int flashnorm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLASHNORM_H */

@@ -1,7 +1,7 @@
 """Plain fp64 CPU oracle for FlashNorm (RMSNorm followed by a linear layer).
 
-TEST INFRASTRUCTURE ONLY. This module is imported by the tests, by the graft
-smoke check and by the CPU-baseline leg of the benchmark. The library itself
+TEST INFRASTRUCTURE ONLY. This module is imported by the tests, by
+__graft_entry__.smoke() and by the CPU-baseline leg of bench.py. The library itself
 never imports it, calls it or falls back to it; it shares no code with the
 CUDA kernels (only the seeded input generator feeds both).
 
@@ -17,12 +17,13 @@ function below states the plainest reading of that prose:
   W* = diag(g) . W.
 * (ii) deferred normalization: the scalar 1/rms is applied to the output of
   the matrix multiplication, y = (x . W*) * 1/sqrt(mean(x^2) + eps).
-* GLU feed-forward variant ("feed-forward networks with GLU variants"): the
-  deferred scale is applied to the gate and the up outputs before SiLU,
-  y = silu(z_gate) * z_up, silu(t) = t / (1 + exp(-t)).
-* Redundant-norm removal ("an RMSNorm followed by a linear layer followed by
-  another RMSNorm allows the first RMSNorm to be eliminated"): linear ->
-  RMSNorm replaces RMSNorm -> linear -> RMSNorm by the scale invariance of RMS.
+* GLU feed-forward variant (the abstract lists gated feed-forward layers among
+  the cases the techniques extend to): the deferred scale is applied to the
+  gate and the up outputs before SiLU, y = silu(z_gate) * z_up,
+  silu(t) = t / (1 + exp(-t)).
+* Redundant-norm removal (with a linear layer between two RMSNorms, the abstract
+  drops the first norm by the scale invariance of RMS): linear -> RMSNorm
+  replaces RMSNorm -> linear -> RMSNorm.
 
 Everything is computed in float64 from inputs given as bf16 bit patterns; the
 only library primitive is numpy's float64 matrix product. No blocking, fusion

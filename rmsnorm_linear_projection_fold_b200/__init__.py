@@ -1,0 +1,264 @@
+"""FlashNorm RMSNorm -> linear on B200: a thin binding of the C ABI in include/flashnorm.h.
+
+Each function here has the name of the C entry point it calls and only marshals arguments: it
+checks that the torch tensors are CUDA bf16 / fp32 and contiguous, allocates outputs the caller did
+not pass, and hands raw pointers plus the current CUDA stream to libflashnorm.so. All arithmetic
+runs in the library's sm_100a kernels; there is no fallback of any kind. If the library is missing,
+importing works but every call raises.
+
+    Wstar = flashnorm_fold_weights(W, g)             # W [d, N] bf16, g [d] bf16 -> W* [N, d]
+    y = flashnorm_linear(x, Wstar, eps)              # x [M, d] bf16 -> y [M, N]
+    Wgu = flashnorm_fold_weights(W_gu, g, glu=True)  # W_gu [d, 2F]: gate | up
+    y = flashnorm_glu(x, Wgu, eps)                   # -> y [M, F]
+    y = flashnorm_linear_postnorm(x, Wstar, g2, head_dim, eps2)
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "FlashNormError",
+    "library_path",
+    "load_library",
+    "flashnorm_fold_weights",
+    "flashnorm_linear",
+    "flashnorm_glu",
+    "flashnorm_linear_postnorm",
+    "flashnorm_rmsnorm",
+    "flashnorm_linear_unfused",
+    "flashnorm_glu_unfused",
+    "flashnorm_check_device_error",
+    "flashnorm_version",
+    "EXPORTED_SYMBOLS",
+]
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG_DIR, "libflashnorm.so")
+
+FN_OK, FN_ERR_INVALID_ARG, FN_ERR_UNSUPPORTED, FN_ERR_ALIGN, FN_ERR_CUDA, FN_ERR_TIMEOUT = range(6)
+FN_BF16, FN_F32 = 0, 1
+PATHS = {"auto": 0, "tensor": 1, "gemv": 2}
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_F = ctypes.c_float
+_INT = ctypes.c_int
+
+# name -> argtypes; restype is fn_status (int) unless listed in _RESTYPES
+_SIGNATURES = {
+    "flashnorm_fold_weights": [_P, _P, _P, _I64, _I64, _INT, _P],
+    "flashnorm_linear": [_P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
+    "flashnorm_linear_ex": [_P, _P, _P, _I64, _I64, _I64, _F, _INT, _INT, _P],
+    "flashnorm_glu": [_P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
+    "flashnorm_glu_ex": [_P, _P, _P, _I64, _I64, _I64, _F, _INT, _INT, _P],
+    "flashnorm_linear_postnorm": [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _F, _INT, _P],
+    "flashnorm_rmsnorm": [_P, _P, _P, _I64, _I64, _F, _P],
+    "flashnorm_linear_unfused": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
+    "flashnorm_glu_unfused": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
+    "flashnorm_check_device_error": [_P],
+    "flashnorm_status_string": [_INT],
+    "flashnorm_last_error": [],
+    "flashnorm_version": [],
+}
+_RESTYPES = {"flashnorm_status_string": ctypes.c_char_p, "flashnorm_last_error": ctypes.c_char_p}
+EXPORTED_SYMBOLS = tuple(_SIGNATURES)
+
+_lib = None
+
+
+class FlashNormError(RuntimeError):
+    """A library call returned a status other than FN_OK."""
+
+    def __init__(self, fn_name: str, status: int, detail: str):
+        self.status = status
+        super().__init__(f"{fn_name} failed with status {status}: {detail}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libflashnorm.so (once). Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise FlashNormError("load_library", -1, f"{_LIB_PATH} is missing; build it with "
+                                 "`python -m rmsnorm_linear_projection_fold_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        for name, args in _SIGNATURES.items():
+            f = getattr(lib, name)
+            f.argtypes = args
+            f.restype = _RESTYPES.get(name, ctypes.c_int)
+        _lib = lib
+    return _lib
+
+
+def _check(name: str, status: int) -> None:
+    if status != FN_OK:
+        lib = load_library()
+        detail = lib.flashnorm_last_error().decode() or lib.flashnorm_status_string(status).decode()
+        raise FlashNormError(name, status, detail)
+
+
+def _stream_ptr(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _need(t: torch.Tensor, name: str, dtype=torch.bfloat16, dim=None) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if dim is not None and t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dimensions, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _out_code(out_dtype) -> int:
+    if out_dtype == torch.bfloat16:
+        return FN_BF16
+    if out_dtype == torch.float32:
+        return FN_F32
+    raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
+
+
+def _output(out, shape, dtype, like):
+    if out is None:
+        return torch.empty(shape, dtype=dtype, device=like.device)
+    _need(out, "out", dtype)
+    if tuple(out.shape) != tuple(shape):
+        raise ValueError(f"out must have shape {tuple(shape)}, got {tuple(out.shape)}")
+    return out
+
+
+def flashnorm_fold_weights(W: torch.Tensor, g: torch.Tensor, glu: bool = False, out=None) -> torch.Tensor:
+    """W* = diag(g) . W rounded once to bf16, stored K-major [N, d] (GLU: gate/up interleaved)."""
+    _need(W, "W", dim=2)
+    _need(g, "g", dim=1)
+    d, N = W.shape
+    if g.shape[0] != d:
+        raise ValueError("g must have d elements")
+    out = _output(out, (N, d), torch.bfloat16, W)
+    lib = load_library()
+    _check("flashnorm_fold_weights",
+           lib.flashnorm_fold_weights(_ptr(W), _ptr(g), _ptr(out), d, N, int(bool(glu)), _stream_ptr(W)))
+    return out
+
+
+def flashnorm_linear(x: torch.Tensor, Wstar: torch.Tensor, eps: float, out_dtype=torch.bfloat16, out=None,
+                     path: str = "auto") -> torch.Tensor:
+    """y = (x . W*) * 1/sqrt(mean(x^2) + eps); x [M, d] bf16, W* [N, d] from fold_weights."""
+    _need(x, "x", dim=2)
+    _need(Wstar, "Wstar", dim=2)
+    M, d = x.shape
+    N = Wstar.shape[0]
+    if Wstar.shape[1] != d:
+        raise ValueError("Wstar must be [N, d] with the d of x")
+    y = _output(out, (M, N), out_dtype, x)
+    lib = load_library()
+    _check("flashnorm_linear", lib.flashnorm_linear_ex(_ptr(x), _ptr(Wstar), _ptr(y), M, d, N, float(eps),
+                                                       _out_code(out_dtype), PATHS[path], _stream_ptr(x)))
+    return y
+
+
+def flashnorm_glu(x: torch.Tensor, Wstar_gu: torch.Tensor, eps: float, out_dtype=torch.bfloat16, out=None,
+                  path: str = "auto") -> torch.Tensor:
+    """y = silu(r * x.W*_gate) * (r * x.W*_up), r = 1/sqrt(mean(x^2)+eps); W*_gu [2F, d] from fold(glu=True)."""
+    _need(x, "x", dim=2)
+    _need(Wstar_gu, "Wstar_gu", dim=2)
+    M, d = x.shape
+    if Wstar_gu.shape[1] != d or Wstar_gu.shape[0] % 2:
+        raise ValueError("Wstar_gu must be [2F, d] with the d of x")
+    F = Wstar_gu.shape[0] // 2
+    y = _output(out, (M, F), out_dtype, x)
+    lib = load_library()
+    _check("flashnorm_glu", lib.flashnorm_glu_ex(_ptr(x), _ptr(Wstar_gu), _ptr(y), M, d, F, float(eps),
+                                                 _out_code(out_dtype), PATHS[path], _stream_ptr(x)))
+    return y
+
+
+def flashnorm_linear_postnorm(x: torch.Tensor, Wstar: torch.Tensor, g2: torch.Tensor, head_dim: int, eps2: float,
+                              out_dtype=torch.bfloat16, out=None) -> torch.Tensor:
+    """Per-head RMSNorm(x . W*; g2, eps2) with the first RMSNorm elided (its gain folded into W*)."""
+    _need(x, "x", dim=2)
+    _need(Wstar, "Wstar", dim=2)
+    _need(g2, "g2", dim=1)
+    M, d = x.shape
+    N = Wstar.shape[0]
+    if Wstar.shape[1] != d:
+        raise ValueError("Wstar must be [N, d] with the d of x")
+    if g2.shape[0] != head_dim:
+        raise ValueError("g2 must have head_dim elements")
+    y = _output(out, (M, N), out_dtype, x)
+    lib = load_library()
+    _check("flashnorm_linear_postnorm",
+           lib.flashnorm_linear_postnorm(_ptr(x), _ptr(Wstar), _ptr(g2), _ptr(y), M, d, N, int(head_dim),
+                                         float(eps2), _out_code(out_dtype), _stream_ptr(x)))
+    return y
+
+
+def flashnorm_rmsnorm(x: torch.Tensor, g: torch.Tensor, eps: float, out=None) -> torch.Tensor:
+    """xn = bf16(x / sqrt(mean(x^2) + eps) * g), the first kernel of the unfused baseline."""
+    _need(x, "x", dim=2)
+    _need(g, "g", dim=1)
+    M, d = x.shape
+    xn = _output(out, (M, d), torch.bfloat16, x)
+    lib = load_library()
+    _check("flashnorm_rmsnorm", lib.flashnorm_rmsnorm(_ptr(x), _ptr(g), _ptr(xn), M, d, float(eps), _stream_ptr(x)))
+    return xn
+
+
+def flashnorm_linear_unfused(x, g, W_kmajor, eps, xn_ws=None, out_dtype=torch.bfloat16, out=None):
+    """Unfused baseline: xn = RMSNorm(x; g) in bf16, then y = xn . W (W_kmajor = fold(W, ones))."""
+    _need(x, "x", dim=2)
+    _need(g, "g", dim=1)
+    _need(W_kmajor, "W_kmajor", dim=2)
+    M, d = x.shape
+    N = W_kmajor.shape[0]
+    xn_ws = _output(xn_ws, (M, d), torch.bfloat16, x)
+    y = _output(out, (M, N), out_dtype, x)
+    lib = load_library()
+    _check("flashnorm_linear_unfused",
+           lib.flashnorm_linear_unfused(_ptr(x), _ptr(g), _ptr(W_kmajor), _ptr(xn_ws), _ptr(y), M, d, N, float(eps),
+                                        _out_code(out_dtype), _stream_ptr(x)))
+    return y
+
+
+def flashnorm_glu_unfused(x, g, W_kmajor_gu, eps, xn_ws=None, out_dtype=torch.bfloat16, out=None):
+    """Unfused GLU baseline: xn = RMSNorm(x; g) in bf16, then silu(xn.W_gate) * (xn.W_up)."""
+    _need(x, "x", dim=2)
+    _need(g, "g", dim=1)
+    _need(W_kmajor_gu, "W_kmajor_gu", dim=2)
+    M, d = x.shape
+    F = W_kmajor_gu.shape[0] // 2
+    xn_ws = _output(xn_ws, (M, d), torch.bfloat16, x)
+    y = _output(out, (M, F), out_dtype, x)
+    lib = load_library()
+    _check("flashnorm_glu_unfused",
+           lib.flashnorm_glu_unfused(_ptr(x), _ptr(g), _ptr(W_kmajor_gu), _ptr(xn_ws), _ptr(y), M, d, F, float(eps),
+                                     _out_code(out_dtype), _stream_ptr(x)))
+    return y
+
+
+def flashnorm_check_device_error(device=None) -> None:
+    """Synchronise the current stream and raise if a kernel gave up on a bounded wait."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+    lib = load_library()
+    s = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    _check("flashnorm_check_device_error", lib.flashnorm_check_device_error(s))
+
+
+def flashnorm_version() -> int:
+    return int(load_library().flashnorm_version())

@@ -1,0 +1,420 @@
+// flashnorm.cu — the C ABI (include/flashnorm.h): argument validation, tile selection, TMA tensor maps
+// and kernel launches for the FlashNorm path on sm_100a. Every computation happens in the kernels of
+// fused_gemm.cuh, gemv.cuh and elementwise.cuh; this file only checks, plans and enqueues.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/flashnorm.h"
+#include "elementwise.cuh"
+#include "fused_gemm.cuh"
+#include "gemv.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+fn_status fail(fn_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+fn_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+
+int device_sm_count(int* dev_out) {
+  static int sms[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  if (sms[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    sms[dev] = v;
+  }
+  *dev_out = dev;
+  return sms[dev];
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda dependency).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn_ptr = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn_ptr = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn_ptr;
+}
+
+// 2-D bf16 K-major operand [rows, k] with a (64 x box_rows) box and 128-byte swizzle.
+fn_status make_operand_map(CUtensorMap* map, const void* ptr, int64_t k, int64_t rows, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(fn::kBK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  return FN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fn_status check_ptr(const void* p, const char* name) {
+  if (p == nullptr) return fail(FN_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(FN_ERR_ALIGN, "%s is not 16-byte aligned", name);
+  return FN_OK;
+}
+
+constexpr int64_t kMaxDim = (int64_t{1} << 31) - 1;
+
+fn_status check_common(const void* x, const void* w, const void* y, int64_t M, int64_t d, float eps, int out_dtype) {
+  if (M < 0 || M > kMaxDim) return fail(FN_ERR_INVALID_ARG, "M = %lld out of range", (long long)M);
+  if (d < 8 || d > kMaxDim || d % 8 != 0)
+    return fail(FN_ERR_INVALID_ARG, "d = %lld must be a positive multiple of 8", (long long)d);
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return fail(FN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (out_dtype != FN_BF16 && out_dtype != FN_F32) return fail(FN_ERR_INVALID_ARG, "out_dtype %d unknown", out_dtype);
+  fn_status st;
+  if (M > 0) {
+    if ((st = check_ptr(x, "x")) != FN_OK) return st;
+    if ((st = check_ptr(y, "y")) != FN_OK) return st;
+  }
+  if ((st = check_ptr(w, "W*")) != FN_OK) return st;
+  return FN_OK;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Tensor-core path
+// ------------------------------------------------------------------------------------------------
+
+// Accumulator width: fewest waves of tiles over the SMs, weighted by the tile width plus a fixed
+// per-tile cost (the x tile and the epilogue do not shrink with bn).
+int choose_bn(int64_t M, int64_t n_rows, int sms, int step) {
+  const int64_t m_tiles = (M + fn::kBM - 1) / fn::kBM;
+  const int64_t n_cap = ((n_rows + step - 1) / step) * step;
+  const int top = n_cap < 256 ? static_cast<int>(n_cap) : 256;
+  int best = top;
+  int64_t best_cost = INT64_MAX;
+  for (int bn = top; bn >= step && (bn >= 64 || bn == top); bn -= step) {
+    const int64_t tiles = m_tiles * ((n_rows + bn - 1) / bn);
+    const int64_t waves = (tiles + sms - 1) / sms;
+    const int64_t cost = waves * (bn + 64);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
+template <int MAX_BN, int STAGES, int EPI, bool SCALE, bool OUT_F32>
+fn_status launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw, const fn::GemmParams& p, int sms, int dev,
+                        cudaStream_t stream) {
+  auto kern = fn::k_fused_gemm<MAX_BN, STAGES, EPI, SCALE, OUT_F32>;
+  constexpr int smem = fn::gemm_smem_bytes<MAX_BN, STAGES>();
+  static bool configured[kMaxDevices] = {false};
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    configured[dev] = true;
+  }
+  const int tiles = p.num_m_tiles * p.num_n_tiles;
+  const int grid = tiles < sms ? tiles : sms;
+  kern<<<grid, fn::gemm_threads(SCALE), smem, stream>>>(tx, tw, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fused GEMM launch");
+  return FN_OK;
+}
+
+// epi: fn::EpiKind; scale: apply the deferred 1/rms (sum of squares warpgroup on).
+fn_status run_tensor_path(const void* x, const void* w, void* y, const void* g2, int64_t M, int64_t d,
+                          int64_t n_rows, int64_t n_out, int64_t head_dim, float eps, int out_dtype, int epi,
+                          bool scale, cudaStream_t stream) {
+  int dev = 0;
+  const int sms = device_sm_count(&dev);
+  if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
+  int bn;
+  if (epi == fn::EPI_POSTNORM) {
+    bn = head_dim <= 256 ? static_cast<int>((256 / head_dim) * head_dim) : static_cast<int>(head_dim);
+    if (bn > n_rows) bn = static_cast<int>(n_rows);  // n_rows is a multiple of head_dim
+  } else {
+    bn = choose_bn(M, n_rows, sms, epi == fn::EPI_GLU ? 32 : 16);
+  }
+  CUtensorMap tx, tw;
+  fn_status st = make_operand_map(&tx, x, d, M, fn::kBM);
+  if (st != FN_OK) return st;
+  st = make_operand_map(&tw, w, d, n_rows, bn <= 256 ? bn : bn / 2);
+  if (st != FN_OK) return st;
+
+  fn::GemmParams p;
+  p.y = y;
+  p.g2 = static_cast<const uint16_t*>(g2);
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(d);
+  p.n_out = static_cast<int>(n_out);
+  p.ldy = static_cast<int>(n_out);
+  p.bn = bn;
+  p.head_dim = static_cast<int>(head_dim);
+  p.num_m_tiles = static_cast<int>((M + fn::kBM - 1) / fn::kBM);
+  p.num_n_tiles = static_cast<int>((n_rows + bn - 1) / bn);
+  p.eps = eps;
+  const bool f32 = out_dtype == FN_F32;
+
+#define FN_LAUNCH(MAXBN, ST, EPI, SC)                                                        \
+  (f32 ? launch_gemm_t<MAXBN, ST, EPI, SC, true>(tx, tw, p, sms, dev, stream)               \
+       : launch_gemm_t<MAXBN, ST, EPI, SC, false>(tx, tw, p, sms, dev, stream))
+  if (epi == fn::EPI_LINEAR) return scale ? FN_LAUNCH(256, 4, fn::EPI_LINEAR, true) : FN_LAUNCH(256, 4, fn::EPI_LINEAR, false);
+  if (epi == fn::EPI_GLU) return scale ? FN_LAUNCH(256, 4, fn::EPI_GLU, true) : FN_LAUNCH(256, 4, fn::EPI_GLU, false);
+  if (bn <= 256) return FN_LAUNCH(256, 4, fn::EPI_POSTNORM, false);
+  return FN_LAUNCH(512, 2, fn::EPI_POSTNORM, false);
+#undef FN_LAUNCH
+}
+
+// ------------------------------------------------------------------------------------------------
+// GEMV (decode) path
+// ------------------------------------------------------------------------------------------------
+
+template <int MT, int R, bool GLU, bool OUT_F32>
+fn_status launch_gemv_t(const void* x, const void* w, void* y, int64_t M, int64_t d, int64_t n_units, float eps,
+                        int sms, int dev, cudaStream_t stream) {
+  auto kern = fn::k_gemv<MT, R, GLU, OUT_F32>;
+  const int smem = fn::gemv_smem_bytes<MT>(static_cast<int>(d));
+  static int configured[kMaxDevices] = {0};
+  if (smem > 48 * 1024 && configured[dev] < smem) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (gemv)");
+    configured[dev] = smem;
+  }
+  const int64_t groups = (n_units + R - 1) / R;
+  const int64_t blocks_needed = (groups + 7) / 8;
+  int per_sm = (228 * 1024) / (smem + 1024);
+  if (per_sm > 8) per_sm = 8;
+  if (per_sm < 1) per_sm = 1;
+  int64_t grid = static_cast<int64_t>(sms) * per_sm;
+  if (blocks_needed < grid) grid = blocks_needed;
+  kern<<<static_cast<unsigned>(grid), fn::kGemvThreads, smem, stream>>>(
+      static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w), y, static_cast<int>(M), static_cast<int>(d),
+      static_cast<int>(n_units), static_cast<int>(n_units), eps);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");
+  return FN_OK;
+}
+
+constexpr int kGemvSmemLimit = 227 * 1024;
+
+int gemv_mt(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
+
+bool gemv_fits(int64_t M, int64_t d) {
+  return static_cast<int64_t>(gemv_mt(M)) * d * 2 + 64 <= kGemvSmemLimit;
+}
+
+fn_status run_gemv(const void* x, const void* w, void* y, int64_t M, int64_t d, int64_t n_units, float eps,
+                   int out_dtype, bool glu, cudaStream_t stream) {
+  int dev = 0;
+  const int sms = device_sm_count(&dev);
+  if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
+  const bool f32 = out_dtype == FN_F32;
+  const int mt = gemv_mt(M);
+#define FN_GEMV(MT, R)                                                                                       \
+  (glu ? (f32 ? launch_gemv_t<MT, R, true, true>(x, w, y, M, d, n_units, eps, sms, dev, stream)             \
+              : launch_gemv_t<MT, R, true, false>(x, w, y, M, d, n_units, eps, sms, dev, stream))           \
+       : (f32 ? launch_gemv_t<MT, R, false, true>(x, w, y, M, d, n_units, eps, sms, dev, stream)            \
+              : launch_gemv_t<MT, R, false, false>(x, w, y, M, d, n_units, eps, sms, dev, stream)))
+  switch (mt) {
+    case 1: return FN_GEMV(1, 4);
+    case 2: return FN_GEMV(2, 4);
+    case 4: return FN_GEMV(4, 2);
+    case 8: return FN_GEMV(8, 2);
+    default: return FN_GEMV(16, 1);
+  }
+#undef FN_GEMV
+}
+
+fn_status projection(const void* x, const void* w, void* y, int64_t M, int64_t d, int64_t n_rows, int64_t n_out,
+                     float eps, int out_dtype, int path, bool glu, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (path != FN_PATH_AUTO && path != FN_PATH_TENSOR && path != FN_PATH_GEMV)
+    return fail(FN_ERR_INVALID_ARG, "path %d unknown", path);
+  if (M == 0) return FN_OK;
+  bool use_gemv = path == FN_PATH_GEMV || (path == FN_PATH_AUTO && M <= FN_DECODE_MAX_M && gemv_fits(M, d));
+  if (use_gemv) {
+    if (M > FN_DECODE_MAX_M) return fail(FN_ERR_UNSUPPORTED, "GEMV path takes M <= %d", FN_DECODE_MAX_M);
+    if (!gemv_fits(M, d)) return fail(FN_ERR_UNSUPPORTED, "GEMV path: x [%lld, %lld] does not fit in shared memory",
+                                      (long long)M, (long long)d);
+    return run_gemv(x, w, y, M, d, n_out, eps, out_dtype, glu, s);
+  }
+  return run_tensor_path(x, w, y, nullptr, M, d, n_rows, n_out, 0, eps, out_dtype,
+                         glu ? fn::EPI_GLU : fn::EPI_LINEAR, true, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+fn_status flashnorm_fold_weights(const void* W, const void* g, void* Wstar, int64_t d, int64_t N, int glu,
+                                 void* stream) {
+  g_last_error[0] = '\0';
+  if (d < 8 || d > kMaxDim || d % 8 != 0) return fail(FN_ERR_INVALID_ARG, "d = %lld must be a positive multiple of 8", (long long)d);
+  if (N < 8 || N > kMaxDim || N % 8 != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a positive multiple of 8", (long long)N);
+  if (glu != 0 && glu != 1) return fail(FN_ERR_INVALID_ARG, "glu must be 0 or 1");
+  if (glu && (N % 32 != 0)) return fail(FN_ERR_INVALID_ARG, "GLU fold needs N = 2F with F %% 16 == 0");
+  fn_status st;
+  if ((st = check_ptr(W, "W")) != FN_OK) return st;
+  if ((st = check_ptr(g, "g")) != FN_OK) return st;
+  if ((st = check_ptr(Wstar, "Wstar")) != FN_OK) return st;
+  dim3 grid(static_cast<unsigned>((N + fn::kFoldTile - 1) / fn::kFoldTile),
+            static_cast<unsigned>((d + fn::kFoldTile - 1) / fn::kFoldTile));
+  if (grid.y > 65535) return fail(FN_ERR_UNSUPPORTED, "d too large for the fold grid");
+  fn::k_fold<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(W), static_cast<const uint16_t*>(g), static_cast<uint16_t*>(Wstar),
+      static_cast<int>(d), static_cast<int>(N), glu);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fold launch");
+  return FN_OK;
+}
+
+fn_status flashnorm_linear_ex(const void* x, const void* Wstar, void* y, int64_t M, int64_t d, int64_t N, float eps,
+                              int out_dtype, int path, void* stream) {
+  g_last_error[0] = '\0';
+  fn_status st = check_common(x, Wstar, y, M, d, eps, out_dtype);
+  if (st != FN_OK) return st;
+  if (N < 8 || N > kMaxDim || N % 8 != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a positive multiple of 8", (long long)N);
+  return projection(x, Wstar, y, M, d, N, N, eps, out_dtype, path, false, stream);
+}
+
+fn_status flashnorm_linear(const void* x, const void* Wstar, void* y, int64_t M, int64_t d, int64_t N, float eps,
+                           int out_dtype, void* stream) {
+  return flashnorm_linear_ex(x, Wstar, y, M, d, N, eps, out_dtype, FN_PATH_AUTO, stream);
+}
+
+fn_status flashnorm_glu_ex(const void* x, const void* Wstar_gu, void* y, int64_t M, int64_t d, int64_t F, float eps,
+                           int out_dtype, int path, void* stream) {
+  g_last_error[0] = '\0';
+  fn_status st = check_common(x, Wstar_gu, y, M, d, eps, out_dtype);
+  if (st != FN_OK) return st;
+  if (F < 16 || F > kMaxDim / 2 || F % 16 != 0) return fail(FN_ERR_INVALID_ARG, "F = %lld must be a positive multiple of 16", (long long)F);
+  return projection(x, Wstar_gu, y, M, d, 2 * F, F, eps, out_dtype, path, true, stream);
+}
+
+fn_status flashnorm_glu(const void* x, const void* Wstar_gu, void* y, int64_t M, int64_t d, int64_t F, float eps,
+                        int out_dtype, void* stream) {
+  return flashnorm_glu_ex(x, Wstar_gu, y, M, d, F, eps, out_dtype, FN_PATH_AUTO, stream);
+}
+
+fn_status flashnorm_linear_postnorm(const void* x, const void* Wstar, const void* g2, void* y, int64_t M, int64_t d,
+                                    int64_t N, int64_t head_dim, float eps2, int out_dtype, void* stream) {
+  g_last_error[0] = '\0';
+  fn_status st = check_common(x, Wstar, y, M, d, eps2, out_dtype);
+  if (st != FN_OK) return st;
+  if (head_dim < 16 || head_dim % 16 != 0) return fail(FN_ERR_INVALID_ARG, "head_dim = %lld must be a positive multiple of 16", (long long)head_dim);
+  if (head_dim > 512) return fail(FN_ERR_UNSUPPORTED, "head_dim = %lld > 512 (one tensor memory)", (long long)head_dim);
+  if (head_dim > 256 && head_dim % 32 != 0) return fail(FN_ERR_UNSUPPORTED, "head_dim in (256, 512] must be a multiple of 32");
+  if (N < head_dim || N > kMaxDim || N % head_dim != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a multiple of head_dim", (long long)N);
+  if ((st = check_ptr(g2, "g2")) != FN_OK) return st;
+  if (M == 0) return FN_OK;
+  return run_tensor_path(x, Wstar, y, g2, M, d, N, N, head_dim, eps2, out_dtype, fn::EPI_POSTNORM, false,
+                         static_cast<cudaStream_t>(stream));
+}
+
+fn_status flashnorm_rmsnorm(const void* x, const void* g, void* xn, int64_t M, int64_t d, float eps, void* stream) {
+  g_last_error[0] = '\0';
+  if (M < 0 || M > kMaxDim) return fail(FN_ERR_INVALID_ARG, "M out of range");
+  if (d < 8 || d > kMaxDim || d % 8 != 0) return fail(FN_ERR_INVALID_ARG, "d must be a positive multiple of 8");
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return fail(FN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  fn_status st;
+  if ((st = check_ptr(g, "g")) != FN_OK) return st;
+  if (M == 0) return FN_OK;
+  if ((st = check_ptr(x, "x")) != FN_OK) return st;
+  if ((st = check_ptr(xn, "xn")) != FN_OK) return st;
+  const int64_t blocks = (M + 7) / 8;
+  fn::k_rmsnorm<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(g), static_cast<uint16_t*>(xn),
+      static_cast<int>(M), static_cast<int>(d), eps);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
+  return FN_OK;
+}
+
+static fn_status unfused(const void* x, const void* g, const void* Wk, void* xn_ws, void* y, int64_t M, int64_t d,
+                         int64_t n_rows, int64_t n_out, float eps, int out_dtype, bool glu, void* stream) {
+  fn_status st = check_common(x, Wk, y, M, d, eps, out_dtype);
+  if (st != FN_OK) return st;
+  if ((st = check_ptr(g, "g")) != FN_OK) return st;
+  if (M == 0) return FN_OK;
+  if ((st = check_ptr(xn_ws, "xn_ws")) != FN_OK) return st;
+  st = flashnorm_rmsnorm(x, g, xn_ws, M, d, eps, stream);
+  if (st != FN_OK) return st;
+  return run_tensor_path(xn_ws, Wk, y, nullptr, M, d, n_rows, n_out, 0, 0.0f, out_dtype,
+                         glu ? fn::EPI_GLU : fn::EPI_LINEAR, false, static_cast<cudaStream_t>(stream));
+}
+
+fn_status flashnorm_linear_unfused(const void* x, const void* g, const void* W_kmajor, void* xn_ws, void* y,
+                                   int64_t M, int64_t d, int64_t N, float eps, int out_dtype, void* stream) {
+  g_last_error[0] = '\0';
+  if (N < 8 || N > kMaxDim || N % 8 != 0) return fail(FN_ERR_INVALID_ARG, "N must be a positive multiple of 8");
+  return unfused(x, g, W_kmajor, xn_ws, y, M, d, N, N, eps, out_dtype, false, stream);
+}
+
+fn_status flashnorm_glu_unfused(const void* x, const void* g, const void* W_kmajor_gu, void* xn_ws, void* y,
+                                int64_t M, int64_t d, int64_t F, float eps, int out_dtype, void* stream) {
+  g_last_error[0] = '\0';
+  if (F < 16 || F > kMaxDim / 2 || F % 16 != 0) return fail(FN_ERR_INVALID_ARG, "F must be a positive multiple of 16");
+  return unfused(x, g, W_kmajor_gu, xn_ws, y, M, d, 2 * F, F, eps, out_dtype, true, stream);
+}
+
+fn_status flashnorm_check_device_error(void* stream) {
+  g_last_error[0] = '\0';
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int h = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&h, fn::g_device_status, sizeof(h), 0, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  if (h != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbolAsync(fn::g_device_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+    if (h & fn::kStatusTimeout) return fail(FN_ERR_TIMEOUT, "a kernel gave up on a bounded wait");
+  }
+  return FN_OK;
+}
+
+const char* flashnorm_status_string(int status) {
+  switch (status) {
+    case FN_OK: return "FN_OK";
+    case FN_ERR_INVALID_ARG: return "FN_ERR_INVALID_ARG: an argument is out of range";
+    case FN_ERR_UNSUPPORTED: return "FN_ERR_UNSUPPORTED: no kernel for this request";
+    case FN_ERR_ALIGN: return "FN_ERR_ALIGN: a pointer is not 16-byte aligned";
+    case FN_ERR_CUDA: return "FN_ERR_CUDA: a CUDA call failed";
+    case FN_ERR_TIMEOUT: return "FN_ERR_TIMEOUT: a device-side wait ran out";
+    default: return "unknown status";
+  }
+}
+
+const char* flashnorm_last_error(void) { return g_last_error; }
+
+int flashnorm_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,96 @@
+"""The C-ABI library: it loads without a GPU, exports every entry point the header declares, and
+rejects bad arguments on the host before it would touch the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import rmsnorm_linear_projection_fold_b200 as fn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "flashnorm.h")
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^FN_API\s+[\w\s\*]+?\b(flashnorm_\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from rmsnorm_linear_projection_fold_b200 import build
+
+    build.build()
+    return fn.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_symbols()
+    for required in ("flashnorm_fold_weights", "flashnorm_linear", "flashnorm_glu", "flashnorm_linear_postnorm"):
+        assert required in names
+    # the binding knows every declared entry point, and nothing undeclared
+    assert set(names) == set(fn.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.flashnorm_version() >= 100
+    for s in range(6):
+        assert lib.flashnorm_status_string(s).startswith(b"FN_")
+
+
+# Fake, aligned, never-dereferenced addresses: every call below must be rejected on the host.
+P = ctypes.c_void_p(1 << 20)
+P_MISALIGNED = ctypes.c_void_p((1 << 20) + 2)
+NULL = ctypes.c_void_p(0)
+
+
+@pytest.mark.parametrize("args,expected", [
+    ((P, P, P, 4, 7, 960, 1e-5, 0, 0, NULL), fn.FN_ERR_INVALID_ARG),      # d % 8 != 0
+    ((P, P, P, 4, 576, 964, 1e-5, 0, 0, NULL), fn.FN_ERR_INVALID_ARG),    # N % 8 != 0
+    ((P, P, P, -1, 576, 960, 1e-5, 0, 0, NULL), fn.FN_ERR_INVALID_ARG),   # M < 0
+    ((P, P, P, 4, 576, 960, -1.0, 0, 0, NULL), fn.FN_ERR_INVALID_ARG),    # eps < 0
+    ((P, P, P, 4, 576, 960, float("nan"), 0, 0, NULL), fn.FN_ERR_INVALID_ARG),
+    ((P, P, P, 4, 576, 960, 1e-5, 7, 0, NULL), fn.FN_ERR_INVALID_ARG),    # out dtype
+    ((P, P, P, 4, 576, 960, 1e-5, 0, 9, NULL), fn.FN_ERR_INVALID_ARG),    # path
+    ((NULL, P, P, 4, 576, 960, 1e-5, 0, 0, NULL), fn.FN_ERR_INVALID_ARG),  # x NULL
+    ((P_MISALIGNED, P, P, 4, 576, 960, 1e-5, 0, 0, NULL), fn.FN_ERR_ALIGN),
+    ((P, P, P, 64, 576, 960, 1e-5, 0, 2, NULL), fn.FN_ERR_UNSUPPORTED),   # GEMV forced with M > 16
+    ((P, P, P, 0, 576, 960, 1e-5, 0, 0, NULL), fn.FN_OK),                # empty call: nothing launched
+])
+def test_linear_validation(lib, args, expected):
+    assert lib.flashnorm_linear_ex(*args) == expected
+    if expected != fn.FN_OK:
+        assert lib.flashnorm_last_error() != b""
+
+
+def test_glu_postnorm_fold_validation(lib):
+    # GLU: F must be a multiple of 16
+    assert lib.flashnorm_glu_ex(P, P, P, 4, 576, 24, 1e-5, 0, 0, NULL) == fn.FN_ERR_INVALID_ARG
+    # post-norm: head_dim limits and N % head_dim
+    assert lib.flashnorm_linear_postnorm(P, P, P, P, 4, 576, 1024, 1024, 1e-6, 0, NULL) == fn.FN_ERR_UNSUPPORTED
+    assert lib.flashnorm_linear_postnorm(P, P, P, P, 4, 576, 1000, 8, 1e-6, 0, NULL) == fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_linear_postnorm(P, P, P, P, 4, 576, 960, 128, 1e-6, 0, NULL) == fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_linear_postnorm(P, P, P, NULL, 4, 576, 512, 128, 1e-6, 0, NULL) == fn.FN_ERR_INVALID_ARG
+    # fold: sizes, flags, GLU needs N = 2F with F % 16 == 0
+    assert lib.flashnorm_fold_weights(P, P, P, 576, 12, 0, NULL) == fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_fold_weights(P, P, P, 576, 960, 2, NULL) == fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_fold_weights(P, P, P, 576, 48, 1, NULL) == fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_fold_weights(P, P, P_MISALIGNED, 576, 960, 0, NULL) == fn.FN_ERR_ALIGN
+    # unfused: the workspace pointer is checked
+    assert lib.flashnorm_linear_unfused(P, P, P, NULL, P, 4, 576, 960, 1e-5, 0, NULL) == fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_rmsnorm(P, P, P, 4, 12, 1e-5, NULL) == fn.FN_ERR_INVALID_ARG
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+
+    x = torch.zeros(4, 16, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fn.flashnorm_linear(x, torch.zeros(16, 16, dtype=torch.bfloat16), 1e-5)
