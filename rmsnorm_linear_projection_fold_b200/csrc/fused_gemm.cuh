@@ -11,7 +11,11 @@
 // Concurrency Challenges"); here the join is explicit and on-chip:
 //   * each shared-memory stage is released only after BOTH of its consumers are done with it (the
 //     MMA's commit and one arrival per sum-of-squares warp), so TMA never overwrites an x tile that
-//     the reduction has not read;
+//     the reduction has not read. The reduction reads with ordinary (generic-proxy) loads while TMA
+//     writes through the async proxy, so each reduction warp also issues a proxy fence before its
+//     arrival; without it the refill could overtake the reads, and the rows' 1/rms picked up parts
+//     of the next k-block (seen on tiles after a CTA's first: the stale-buffer race of the pages,
+//     moved on-chip);
 //   * the epilogue waits on both the accumulator-ready barrier and the rms-ready barrier of the
 //     same tile before it scales anything.
 //
@@ -369,8 +373,6 @@ __global__ void __launch_bounds__(gemm_threads(SCALE), 1)
     uint32_t ph = 0;
     int sb = 0;
     uint32_t sb_ph = 0;
-    const float inv_k = 1.0f / static_cast<float>(p.K);
-    (void)inv_k;
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
@@ -396,6 +398,9 @@ __global__ void __launch_bounds__(gemm_threads(SCALE), 1)
           f = bf16lo_to_f32(w.w); a2 = fmaf(f, f, a2);
           f = bf16hi_to_f32(w.w); a3 = fmaf(f, f, a3);
         }
+        // The generic-proxy reads above must be ordered before the TMA (async proxy) refill of this
+        // stage that our arrival permits.
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
         if (++s == STAGES) {

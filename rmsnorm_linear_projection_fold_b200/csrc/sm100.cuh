@@ -83,6 +83,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Order this thread's generic-proxy accesses of shared memory before later async-proxy (TMA /
+// tensor core) accesses of it. A warp that has READ a TMA-filled stage with ordinary loads must
+// execute this before it releases the stage: the mbarrier hand-off alone does not order the reads
+// against the next TMA write into that stage, and without it the refill can land while the reads
+// are still in flight.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Named barrier over a subset of the CTA's warps.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
