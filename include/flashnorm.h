@@ -141,6 +141,28 @@ FN_API fn_status flashnorm_glu_unfused(const void* x, const void* g, const void*
                                 int64_t M, int64_t d, int64_t F, float eps, int out_dtype, void* stream);
 
 /*
+ * flashnorm_linear_unfused_noalloc — flashnorm_linear_unfused without a caller-supplied workspace.
+ * The paper has no counterpart to this entry point; it exists for callers that cannot provide one:
+ * a drop-in norm+projection op whose interface carries only inputs and outputs, or a caller whose
+ * device memory is all handed out by its own pool allocator, so an extra cudaMalloc would fail (and
+ * cudaMalloc may synchronise the device, which a latency-bound loop cannot afford).
+ * The normalised activations go to a scratch array that is part of the library's device image
+ * (16 MiB of bf16, FN_NOALLOC_MAX_ELEMS elements), which every GPU that loads the library keeps until
+ * the process exits. This call allocates nothing: no cudaMalloc, cudaFree or allocating routine.
+ *   Arguments and results as flashnorm_linear_unfused; M * d must not exceed FN_NOALLOC_MAX_ELEMS
+ *   (larger requests return FN_ERR_UNSUPPORTED and launch nothing).
+ *   The first call on a device looks up the scratch array's device address on that device (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls share the one array and it keeps the previous call's contents (every call overwrites
+ *   the rows it uses before reading them). Calls whose kernels overlap on the GPU -- on different
+ *   streams, or from different host threads -- race on it; serialise them.
+ */
+#define FN_NOALLOC_MAX_ELEMS (1LL << 23)
+FN_API fn_status flashnorm_linear_unfused_noalloc(const void* x, const void* g, const void* W_kmajor, void* y,
+                                                  int64_t M, int64_t d, int64_t N, float eps, int out_dtype,
+                                                  void* stream);
+
+/*
  * flashnorm_check_device_error — synchronises `stream`, then reads and clears the device-side status
  * word of the current device. Returns FN_ERR_TIMEOUT if any kernel of this library gave up on a bounded
  * wait since the last check, FN_ERR_CUDA if the synchronisation itself failed, FN_OK otherwise.

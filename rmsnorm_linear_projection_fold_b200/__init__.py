@@ -31,6 +31,8 @@ __all__ = [
     "flashnorm_rmsnorm",
     "flashnorm_linear_unfused",
     "flashnorm_glu_unfused",
+    "flashnorm_linear_unfused_noalloc",
+    "NOALLOC_MAX_ELEMS",
     "flashnorm_check_device_error",
     "flashnorm_version",
     "EXPORTED_SYMBOLS",
@@ -41,6 +43,7 @@ _LIB_PATH = os.path.join(_PKG_DIR, "libflashnorm.so")
 
 FN_OK, FN_ERR_INVALID_ARG, FN_ERR_UNSUPPORTED, FN_ERR_ALIGN, FN_ERR_CUDA, FN_ERR_TIMEOUT = range(6)
 FN_BF16, FN_F32 = 0, 1
+NOALLOC_MAX_ELEMS = 1 << 23  # FN_NOALLOC_MAX_ELEMS in include/flashnorm.h
 PATHS = {"auto": 0, "tensor": 1, "gemv": 2}
 
 _P = ctypes.c_void_p
@@ -59,6 +62,7 @@ _SIGNATURES = {
     "flashnorm_rmsnorm": [_P, _P, _P, _I64, _I64, _F, _P],
     "flashnorm_linear_unfused": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_glu_unfused": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
+    "flashnorm_linear_unfused_noalloc": [_P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_check_device_error": [_P],
     "flashnorm_status_string": [_INT],
     "flashnorm_last_error": [],
@@ -249,6 +253,27 @@ def flashnorm_glu_unfused(x, g, W_kmajor_gu, eps, xn_ws=None, out_dtype=torch.bf
     _check("flashnorm_glu_unfused",
            lib.flashnorm_glu_unfused(_ptr(x), _ptr(g), _ptr(W_kmajor_gu), _ptr(xn_ws), _ptr(y), M, d, F, float(eps),
                                      _out_code(out_dtype), _stream_ptr(x)))
+    return y
+
+
+def flashnorm_linear_unfused_noalloc(x, g, W_kmajor, eps, out_dtype=torch.bfloat16, out=None):
+    """flashnorm_linear_unfused with the library's own fixed scratch instead of a workspace argument.
+
+    For callers that cannot allocate device memory on this path (no workspace in their interface, or
+    all memory owned by their own pool). M * d must be at most NOALLOC_MAX_ELEMS. Calls share one
+    scratch array per device: calls that overlap on the GPU race, so keep them on one stream. Passing
+    `out` makes the whole call allocation-free on the Python side too.
+    """
+    _need(x, "x", dim=2)
+    _need(g, "g", dim=1)
+    _need(W_kmajor, "W_kmajor", dim=2)
+    M, d = x.shape
+    N = W_kmajor.shape[0]
+    y = _output(out, (M, N), out_dtype, x)
+    lib = load_library()
+    _check("flashnorm_linear_unfused_noalloc",
+           lib.flashnorm_linear_unfused_noalloc(_ptr(x), _ptr(g), _ptr(W_kmajor), _ptr(y), M, d, N, float(eps),
+                                                _out_code(out_dtype), _stream_ptr(x)))
     return y
 
 

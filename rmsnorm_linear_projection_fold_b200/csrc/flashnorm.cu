@@ -383,6 +383,55 @@ fn_status flashnorm_glu_unfused(const void* x, const void* g, const void* W_kmaj
   return unfused(x, g, W_kmajor_gu, xn_ws, y, M, d, 2 * F, F, eps, out_dtype, true, stream);
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// Unfused baseline without a caller workspace. The scratch for the normalised activations lives in
+// this file's device image; host code reaches it only through the address that cudaGetSymbolAddress
+// returns on the current device (the symbol itself is a host-side stand-in, not a device pointer).
+// ------------------------------------------------------------------------------------------------
+static __device__ __align__(256) uint16_t g_noalloc_xn[FN_NOALLOC_MAX_ELEMS];
+
+namespace {
+
+// Device address of g_noalloc_xn on the current device, looked up once per device.
+fn_status noalloc_scratch(void** out) {
+  static void* addr[kMaxDevices] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FN_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_xn);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return FN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fn_status flashnorm_linear_unfused_noalloc(const void* x, const void* g, const void* W_kmajor, void* y, int64_t M,
+                                           int64_t d, int64_t N, float eps, int out_dtype, void* stream) {
+  g_last_error[0] = '\0';
+  if (N < 8 || N > kMaxDim || N % 8 != 0) return fail(FN_ERR_INVALID_ARG, "N must be a positive multiple of 8");
+  fn_status st = check_common(x, W_kmajor, y, M, d, eps, out_dtype);
+  if (st != FN_OK) return st;
+  if (M > 0 && M > FN_NOALLOC_MAX_ELEMS / d)
+    return fail(FN_ERR_UNSUPPORTED, "no-alloc scratch holds %lld elements; M * d = %lld is larger",
+                (long long)FN_NOALLOC_MAX_ELEMS, (long long)(M * d));
+  if (M == 0) return FN_OK;
+  void* xn = nullptr;
+  if ((st = noalloc_scratch(&xn)) != FN_OK) return st;
+  return unfused(x, g, W_kmajor, xn, y, M, d, N, N, eps, out_dtype, false, stream);
+}
+
 fn_status flashnorm_check_device_error(void* stream) {
   g_last_error[0] = '\0';
   cudaStream_t s = static_cast<cudaStream_t>(stream);
