@@ -141,7 +141,7 @@ fn_status launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw, const fn::
   }
   const int tiles = p.num_m_tiles * p.num_n_tiles;
   const int grid = tiles < sms ? tiles : sms;
-  kern<<<grid, fn::gemm_threads(SCALE), smem, stream>>>(tx, tw, p);
+  kern<<<grid, fn::gemm_threads(EPI, SCALE), smem, stream>>>(tx, tw, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fused GEMM launch");
   return FN_OK;

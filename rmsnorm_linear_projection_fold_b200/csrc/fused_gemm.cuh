@@ -19,11 +19,13 @@
 //   * the epilogue waits on both the accumulator-ready barrier and the rms-ready barrier of the
 //     same tile before it scales anything.
 //
-// Warp roles (320 threads with the reduction warpgroup, 192 without):
+// Warp roles:
 //   warp 0      TMA producer: x tile [128 x 64] and W* tile [bn x 64] per k-block into a smem ring
 //   warp 1      TMEM allocator; one lane issues tcgen05.mma and the commits
-//   warps 2-5   epilogue: tcgen05.ld from TMEM, scale / SwiGLU / per-head RMSNorm, global stores
-//   warps 6-9   sum of squares of x per row (only when the deferred scale is used)
+//   epilogue    8 warps (4 for POSTNORM): tcgen05.ld from TMEM, scale / SwiGLU / per-head RMSNorm,
+//               global stores. Warp w may only read TMEM lanes 32*(w%4)..+31, so two warps share
+//               each lane quarter and split the tile's columns between them.
+//   reduction   4 warps, sum of squares of x per row (only when the deferred scale is used)
 //
 // Epilogues: LINEAR  y = r * acc
 //            GLU     y = silu(r * acc_gate) * (r * acc_up)   (gate/up interleaved in blocks of 16 cols)
@@ -61,14 +63,27 @@ struct GemmSmem {
   static constexpr int kBStageBytes = MAX_BN * kBK * 2;
 };
 
-__host__ __device__ constexpr int gemm_threads(bool scale) { return scale ? 320 : 192; }
+// Epilogue warps: two per TMEM lane quarter, except the per-head post-norm, whose row norms need
+// all of a head's columns in one thread.
+__host__ __device__ constexpr int gemm_epi_warps(int epi) { return epi == 2 /* EPI_POSTNORM */ ? 4 : 8; }
+__host__ __device__ constexpr int gemm_threads(int epi, bool scale) {
+  return 64 + 32 * gemm_epi_warps(epi) + (scale ? 128 : 0);
+}
 
 template <int MAX_BN, int STAGES>
 __host__ __device__ constexpr int gemm_smem_bytes() {
   return 1024 /* alignment slack */ + STAGES * (kAStageBytes + MAX_BN * kBK * 2) + 4096 /* barriers etc. */;
 }
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+// silu(z) = z * sigmoid(z), with exp and the reciprocal taken on the special-function unit:
+// sigmoid(z) = 1 / (1 + 2^(-z * log2(e))). Relative error ~1e-6; the limits are exact (z -> -inf
+// gives 2^+inf = inf and rcp(inf) = 0; z -> +inf gives rcp(1) = 1).
+__device__ __forceinline__ float silu_f(float z) {
+  float e, s;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(e) : "f"(-z * 1.4426950408889634f));
+  asm("rcp.approx.f32 %0, %1;" : "=f"(s) : "f"(1.0f + e));
+  return z * s;
+}
 
 // Store 16 consecutive output values of one row (bf16 or fp32), masking whole 8-column groups.
 template <bool OUT_F32>
@@ -100,11 +115,13 @@ __device__ __forceinline__ void store16(void* y, int ldy, int row, int col, int 
 }
 
 template <int MAX_BN, int STAGES, int EPI, bool SCALE, bool OUT_F32>
-__global__ void __launch_bounds__(gemm_threads(SCALE), 1)
+__global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
     k_fused_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, GemmParams p) {
   constexpr int kAccBufs = (MAX_BN <= 256) ? 2 : 1;
   constexpr int kBStage = MAX_BN * kBK * 2;
   constexpr int kSsWarps = SCALE ? 4 : 0;
+  constexpr int kEpiWarps = gemm_epi_warps(EPI);
+  constexpr int kEpiFirst = 2, kSsFirst = 2 + kEpiWarps;
 
   extern __shared__ uint8_t smem_raw[];
   // Stage buffers must sit on 1024-byte boundaries (the 128-byte swizzle repeats every 8 rows).
@@ -135,9 +152,9 @@ __global__ void __launch_bounds__(gemm_threads(SCALE), 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], kEpiWarps);
       mbar_init(&ss_full[b], kBM);
-      mbar_init(&ss_empty[b], kBM);
+      mbar_init(&ss_empty[b], 32 * kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -263,16 +280,17 @@ __global__ void __launch_bounds__(gemm_threads(SCALE), 1)
         }
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < kSsFirst) {
     // ------------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    const int q = warp & 3;                    // TMEM lane quarter this warp may read
+    const int half = (warp - kEpiFirst) >> 2;  // which of the two warps on this quarter
     const int row_in_tile = q * 32 + lane;
     if (EPI == EPI_POSTNORM) {
-      for (int i = threadIdx.x - 64; i < p.head_dim; i += 128) {
+      for (int i = threadIdx.x - 32 * kEpiFirst; i < p.head_dim; i += 32 * kEpiWarps) {
         const uint32_t b = p.g2[i];
         g2s[i] = __uint_as_float(b << 16);
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(1, 32 * kEpiWarps);
     }
     int acc = 0;
     uint32_t acc_ph = 0;
@@ -297,20 +315,30 @@ __global__ void __launch_bounds__(gemm_threads(SCALE), 1)
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * MAX_BN);
 
       if (EPI == EPI_LINEAR) {
+        // this warp's 16-column chunks: every other one, two per TMEM wait
         const int col0 = nt * bn;
-        for (int c = 0; c < bn; c += 16) {
-          uint32_t v[16];
-          tmem_ld16(t_row + c, v);
+        for (int c = half * 16; c < bn; c += 64) {
+          const bool two = c + 32 < bn;
+          uint32_t v0[16], v1[16];
+          tmem_ld16(t_row + c, v0);
+          if (two) tmem_ld16(t_row + c + 32, v1);
           tmem_ld_wait();
-          reg_fence16(v);
+          reg_fence16(v0);
           float o[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(v[j]) * r;
+          for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(v0[j]) * r;
           if (row_ok) store16<OUT_F32>(p.y, p.ldy, row, col0 + c, p.n_out, o);
+          if (two) {
+            reg_fence16(v1);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(v1[j]) * r;
+            if (row_ok) store16<OUT_F32>(p.y, p.ldy, row, col0 + c + 32, p.n_out, o);
+          }
         }
       } else if (EPI == EPI_GLU) {
+        // this warp's (gate, up) pairs of 16 columns: every other pair
         const int col0 = nt * (bn / 2);
-        for (int c = 0; c < bn; c += 32) {
+        for (int c = half * 32; c < bn; c += 64) {
           uint32_t gt[16], up[16];
           tmem_ld16(t_row + c, gt);
           tmem_ld16(t_row + c + 16, up);
