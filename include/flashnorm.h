@@ -57,9 +57,13 @@ typedef enum {
 
 typedef enum { FN_BF16 = 0, FN_F32 = 1 } fn_dtype;
 
-/* Which kernel family a projection runs on. AUTO: the GEMV path for M <= FN_DECODE_MAX_M, the
- * tensor-core path otherwise. */
-typedef enum { FN_PATH_AUTO = 0, FN_PATH_TENSOR = 1, FN_PATH_GEMV = 2 } fn_path;
+/* Which kernel family a projection runs on.
+ *   FN_PATH_TENSOR  the persistent prefill kernel (128-row tiles of x, any M)
+ *   FN_PATH_GEMV    the CUDA-core GEMV (M <= FN_DECODE_MAX_M)
+ *   FN_PATH_DECODE  the tensor-core decode kernel: W* rows on the MMA's M side, the tokens on its
+ *                   N side, W* streamed once by TMA (M <= FN_DECODE_MAX_M)
+ *   FN_PATH_AUTO    a decode kernel for M <= FN_DECODE_MAX_M, the prefill kernel otherwise */
+typedef enum { FN_PATH_AUTO = 0, FN_PATH_TENSOR = 1, FN_PATH_GEMV = 2, FN_PATH_DECODE = 3 } fn_path;
 
 #define FN_DECODE_MAX_M 16
 /* GLU weights are stored gate/up interleaved in blocks of this many output columns (see fold). */

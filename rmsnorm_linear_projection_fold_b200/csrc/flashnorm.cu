@@ -11,9 +11,11 @@
 #include <mutex>
 
 #include "../../include/flashnorm.h"
+#include "decode_tc.cuh"
 #include "elementwise.cuh"
 #include "fused_gemm.cuh"
 #include "gemv.cuh"
+#include "postnorm_cluster.cuh"
 
 namespace {
 
@@ -192,6 +194,71 @@ fn_status run_tensor_path(const void* x, const void* w, void* y, const void* g2,
 }
 
 // ------------------------------------------------------------------------------------------------
+// Wide-head post-norm: one cluster of (head_dim / 128) x KS CTAs per 128-row tile and head
+// ------------------------------------------------------------------------------------------------
+
+template <bool OUT_F32>
+fn_status launch_postnorm_cluster_t(const CUtensorMap& tx, const CUtensorMap& tw, const fn::PostnormClusterParams& p,
+                                    int ctas, int dev, cudaStream_t stream) {
+  auto kern = fn::k_postnorm_cluster<OUT_F32>;
+  constexpr int smem = fn::postnorm_cluster_smem_bytes();
+  static bool configured[kMaxDevices] = {false};
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (post-norm cluster)");
+    configured[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
+  cfg.blockDim = dim3(fn::kPnThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(p.cn * p.ks);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
+  if (e != cudaSuccess) return cuda_fail(e, "post-norm cluster launch");
+  return FN_OK;
+}
+
+fn_status run_postnorm_cluster(const void* x, const void* w, const void* g2, void* y, int64_t M, int64_t d, int64_t N,
+                               int64_t head_dim, float eps2, int out_dtype, cudaStream_t stream) {
+  int dev = 0;
+  const int sms = device_sm_count(&dev);
+  if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
+  fn::PostnormClusterParams p;
+  p.y = y;
+  p.g2 = static_cast<const uint16_t*>(g2);
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(d);
+  p.N = static_cast<int>(N);
+  p.head_dim = static_cast<int>(head_dim);
+  p.num_m_tiles = static_cast<int>((M + 127) / 128);
+  p.cn = static_cast<int>(head_dim / fn::kPnCols);
+  p.eps2 = eps2;
+  const int64_t heads = N / head_dim;
+  const int64_t num_kb = (d + 63) / 64;
+  // Split K while that still adds SMs: at most 8 CTAs per cluster, about one CTA per SM.
+  int ks = 1;
+  if (p.cn * 2 <= 8 && p.num_m_tiles * heads * p.cn * 2 <= sms && num_kb >= 2) ks = 2;
+  p.ks = ks;
+  const int64_t ctas = p.num_m_tiles * heads * p.cn * ks;
+  if (ctas > INT32_MAX) return fail(FN_ERR_UNSUPPORTED, "too many tiles");
+  CUtensorMap tx, tw;
+  fn_status st = make_operand_map(&tx, x, d, M, 128);
+  if (st != FN_OK) return st;
+  st = make_operand_map(&tw, w, d, N, fn::kPnCols);
+  if (st != FN_OK) return st;
+  return out_dtype == FN_F32 ? launch_postnorm_cluster_t<true>(tx, tw, p, static_cast<int>(ctas), dev, stream)
+                             : launch_postnorm_cluster_t<false>(tx, tw, p, static_cast<int>(ctas), dev, stream);
+}
+
+// ------------------------------------------------------------------------------------------------
 // GEMV (decode) path
 // ------------------------------------------------------------------------------------------------
 
@@ -251,12 +318,86 @@ fn_status run_gemv(const void* x, const void* w, void* y, int64_t M, int64_t d, 
 #undef FN_GEMV
 }
 
+// ------------------------------------------------------------------------------------------------
+// Tensor-core decode path
+// ------------------------------------------------------------------------------------------------
+
+template <int STAGES, int KSPLIT, bool GLU, bool OUT_F32>
+fn_status launch_decode_t(const CUtensorMap& tw, const CUtensorMap& tx, const fn::DecodeParams& p, int slabs,
+                          int dev, cudaStream_t stream) {
+  auto kern = fn::k_decode_tc<STAGES, KSPLIT, GLU, OUT_F32>;
+  constexpr int smem = fn::decode_smem_bytes<STAGES, KSPLIT>();
+  static bool configured[kMaxDevices] = {false};
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (decode)");
+    configured[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(slabs * KSPLIT), 1, 1);
+  cfg.blockDim = dim3(fn::kDecThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = KSPLIT;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, p);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return FN_OK;
+}
+
+fn_status run_decode_tc(const void* x, const void* w, void* y, int64_t M, int64_t d, int64_t n_rows, int64_t n_out,
+                        float eps, int out_dtype, bool glu, cudaStream_t stream) {
+  int dev = 0;
+  const int sms = device_sm_count(&dev);
+  if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
+  const int64_t slabs = (n_rows + fn::kDecRows - 1) / fn::kDecRows;
+  const int64_t num_kb = (d + 63) / 64;
+  // Split K across a cluster when the slabs alone would leave most SMs without a W* stream.
+  int ksplit = 1;
+  if (slabs * 2 <= sms && num_kb >= 2) ksplit = 2;
+  if (slabs * 4 <= sms && num_kb >= 4) ksplit = 4;
+  CUtensorMap tw, tx;
+  fn_status st = make_operand_map(&tw, w, d, n_rows, fn::kDecRows);
+  if (st != FN_OK) return st;
+  st = make_operand_map(&tx, x, d, M, fn::kDecTok);
+  if (st != FN_OK) return st;
+  fn::DecodeParams p;
+  p.y = y;
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(d);
+  p.n_rows = static_cast<int>(n_rows);
+  p.n_out = static_cast<int>(n_out);
+  p.ldy = static_cast<int>(n_out);
+  p.ksplit = ksplit;
+  p.eps = eps;
+  const int sl = static_cast<int>(slabs);
+  const bool f32 = out_dtype == FN_F32;
+#define FN_DEC(ST, KS)                                                                                          \
+  (glu ? (f32 ? launch_decode_t<ST, KS, true, true>(tw, tx, p, sl, dev, stream)                              \
+              : launch_decode_t<ST, KS, true, false>(tw, tx, p, sl, dev, stream))                            \
+       : (f32 ? launch_decode_t<ST, KS, false, true>(tw, tx, p, sl, dev, stream)                             \
+              : launch_decode_t<ST, KS, false, false>(tw, tx, p, sl, dev, stream)))
+  if (ksplit == 1) return FN_DEC(12, 1);
+  if (ksplit == 2) return FN_DEC(5, 2);
+  return FN_DEC(3, 4);
+#undef FN_DEC
+}
+
 fn_status projection(const void* x, const void* w, void* y, int64_t M, int64_t d, int64_t n_rows, int64_t n_out,
                      float eps, int out_dtype, int path, bool glu, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (path != FN_PATH_AUTO && path != FN_PATH_TENSOR && path != FN_PATH_GEMV)
+  if (path != FN_PATH_AUTO && path != FN_PATH_TENSOR && path != FN_PATH_GEMV && path != FN_PATH_DECODE)
     return fail(FN_ERR_INVALID_ARG, "path %d unknown", path);
   if (M == 0) return FN_OK;
+  if (path == FN_PATH_DECODE) {
+    if (M > FN_DECODE_MAX_M) return fail(FN_ERR_UNSUPPORTED, "decode path takes M <= %d", FN_DECODE_MAX_M);
+    return run_decode_tc(x, w, y, M, d, n_rows, n_out, eps, out_dtype, glu, s);
+  }
   bool use_gemv = path == FN_PATH_GEMV || (path == FN_PATH_AUTO && M <= FN_DECODE_MAX_M && gemv_fits(M, d));
   if (use_gemv) {
     if (M > FN_DECODE_MAX_M) return fail(FN_ERR_UNSUPPORTED, "GEMV path takes M <= %d", FN_DECODE_MAX_M);
@@ -333,6 +474,8 @@ fn_status flashnorm_linear_postnorm(const void* x, const void* Wstar, const void
   if (N < head_dim || N > kMaxDim || N % head_dim != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a multiple of head_dim", (long long)N);
   if ((st = check_ptr(g2, "g2")) != FN_OK) return st;
   if (M == 0) return FN_OK;
+  if (head_dim > 256 && head_dim % fn::kPnCols == 0)
+    return run_postnorm_cluster(x, Wstar, g2, y, M, d, N, head_dim, eps2, out_dtype, static_cast<cudaStream_t>(stream));
   return run_tensor_path(x, Wstar, y, g2, M, d, N, N, head_dim, eps2, out_dtype, fn::EPI_POSTNORM, false,
                          static_cast<cudaStream_t>(stream));
 }

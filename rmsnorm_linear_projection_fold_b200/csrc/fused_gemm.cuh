@@ -173,7 +173,13 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Tile schedule: the tiles are numbered row-block-major (t -> m = t / num_n, n = t % num_n) and each
+  // CTA takes one contiguous, balanced range of them. Consecutive tiles of a CTA then mostly share
+  // their 128 rows of x, so the reduction warps compute a row's 1/rms once per row block and reuse
+  // it, and the x tiles they reload stay hot in L2.
   const int num_tiles = p.num_m_tiles * p.num_n_tiles;
+  const int t_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * num_tiles / gridDim.x);
+  const int t_end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * num_tiles / gridDim.x);
   const int num_kb = (p.K + kBK - 1) / kBK;
   const int bn = p.bn;
 
@@ -186,9 +192,9 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
       uint32_t ph = 0;
       int issued = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int m0 = (t % p.num_m_tiles) * kBM;
-        const int n0 = (t / p.num_m_tiles) * bn;
+      for (int t = t_begin; t < t_end && ok; ++t) {
+        const int m0 = (t / p.num_n_tiles) * kBM;
+        const int n0 = (t % p.num_n_tiles) * bn;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
@@ -234,7 +240,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
       int acc = 0;
       uint32_t acc_ph = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int t = t_begin; t < t_end && ok; ++t) {
         if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -296,9 +302,9 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
     uint32_t acc_ph = 0;
     int sb = 0;
     uint32_t sb_ph = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      const int mt = t % p.num_m_tiles;
-      const int nt = t / p.num_m_tiles;
+    for (int t = t_begin; t < t_end; ++t) {
+      const int mt = t / p.num_n_tiles;
+      const int nt = t % p.num_n_tiles;
       if (!mbar_wait(&acc_full[acc], acc_ph, abort_flag)) break;
       tc_fence_after_sync();
       float r = 1.0f;
@@ -402,9 +408,15 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
     int sb = 0;
     uint32_t sb_ph = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+    int last_m = -1;  // row block whose 1/rms this thread holds in `r_row`
+    float r_row = 0.0f;
+    for (int t = t_begin; t < t_end && ok; ++t) {
+      const int mt = t / p.num_n_tiles;
+      const bool fresh = mt != last_m;  // same for the whole CTA
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
       for (int kb = 0; kb < num_kb; ++kb) {
+        // Every stage is still waited for and released (the stage barriers count these arrivals),
+        // but it is only read when this row block's sum of squares is not known yet.
         if (!mbar_wait(&full[s], ph, abort_flag)) {
           ok = false;
           break;
@@ -415,6 +427,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
         const uint8_t* line = sA + s * kAStageBytes + row_in_tile * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
+          if (!fresh) break;
           const uint4 w = *reinterpret_cast<const uint4*>(line + (((c ^ lane) & 7) << 4));
           float f;
           f = bf16lo_to_f32(w.x); a0 = fmaf(f, f, a0);
@@ -437,9 +450,13 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
         }
       }
       if (!ok) break;
+      if (fresh) {
+        const float ss = (a0 + a1) + (a2 + a3);
+        r_row = 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps);
+        last_m = mt;
+      }
       if (!mbar_wait(&ss_empty[sb], sb_ph ^ 1u, abort_flag)) break;
-      const float ss = (a0 + a1) + (a2 + a3);
-      rinv[sb * kBM + row_in_tile] = 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps);
+      rinv[sb * kBM + row_in_tile] = r_row;
       mbar_arrive(&ss_full[sb]);
       sb ^= 1;
       if (sb == 0) sb_ph ^= 1u;

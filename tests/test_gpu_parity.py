@@ -109,6 +109,12 @@ LINEAR_CASES = [
     (4, 4096, 1024, "gemv"),
     (16, 4096, 1024, "gemv"),
     (7, 264, 136, "gemv"),       # odd sizes on the GEMV path
+    (1, 4096, 1024, "decode"),   # tensor-core decode: 8 slabs -> K split over a 4-CTA cluster
+    (4, 4096, 12288, "decode"),  # 96 slabs, no split
+    (16, 4096, 1024, "decode"),
+    (7, 576, 960, "decode"),     # partial last slab
+    (5, 72, 136, "decode"),      # 2 k-blocks split over 2 CTAs, ragged K and N
+    (16, 128, 200, "decode"),    # 2 k-blocks, 2 slabs
 ]
 
 
@@ -135,6 +141,9 @@ GLU_CASES = [
     (1, 4096, 512, "gemv"),
     (16, 4096, 512, "gemv"),
     (5, 576, 1536, "auto"),
+    (1, 4096, 512, "decode"),
+    (16, 576, 1536, "decode"),
+    (3, 4096, 11008, "decode"),
 ]
 
 
@@ -158,8 +167,12 @@ POSTNORM_CASES = [
     (300, 512, 512, 128),
     (200, 256, 1024, 256),
     (64, 640, 384, 384),
-    (150, 5120, 512, 512),
+    (150, 5120, 512, 512),       # cluster of 4 column slices x 2 K ranges
     (40, 128, 64, 16),
+    (130, 256, 1024, 512),       # two 512-wide heads, ragged M
+    (300, 320, 768, 384),        # two 384-wide heads: 3 slices x 2 K ranges
+    (2048, 576, 512, 512),       # 16 row tiles, cluster split
+    (64, 320, 320, 320),         # 320-wide head: single-CTA 512-column path
 ]
 
 
@@ -299,7 +312,7 @@ def test_empty_and_zero_rows():
     bits["x"][[0, 17, 39]] = 0  # all-zero rows
     x = to_dev(bits["x"])
     ws = _fold(bits, False)
-    for path in ("tensor", "gemv"):
+    for path in ("tensor", "gemv", "decode"):
         xx = x if path == "tensor" else x[:16].contiguous()
         y = fn.flashnorm_linear(xx, ws, 1e-5, path=path)
         torch.cuda.synchronize()
@@ -344,3 +357,19 @@ def test_many_tiles_per_cta_all_rows(kind, M, d, N):
         y32 = f(x, ws, 1e-6, out_dtype=torch.float32)
         torch.cuda.synchronize()
         assert O.rel_err(to_host_f64(y32), ex) <= F32_TOL
+
+
+@pytest.mark.parametrize("name", ["llama7b_qkv_m1", "llama7b_qkv_m4", "llama7b_qkv_m16"])
+@pytest.mark.parametrize("path", ["gemv", "decode"])
+def test_decode_paths_full_size(name, path):
+    """Both decode kernels at the full Llama-7B QKV size, every output checked."""
+    wl = I.WORKLOADS[name]
+    bits = wl.draw()
+    ws = _fold(bits, False)
+    y16 = fn.flashnorm_linear(to_dev(bits["x"]), ws, wl.eps, path=path)
+    y32 = fn.flashnorm_linear(to_dev(bits["x"]), ws, wl.eps, out_dtype=torch.float32, path=path)
+    torch.cuda.synchronize()
+    ref = O.reference_output("linear", bits, wl.eps)
+    ref_exact = _exact("linear", bits, wl.eps)
+    check_bf16(to_host_f64(y16), ref, ref_exact)
+    assert O.rel_err(to_host_f64(y32), ref_exact) <= F32_TOL
