@@ -91,6 +91,22 @@ def _peaks() -> dict:
             "source": "fallback"}
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest `value` over all ranks (a device-timed duration: the slowest rank sets the time)."""
+    if world <= 1:
+        return float(value)
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, world: int, ms_per_step: float, scale: float) -> float:
+    """Whole-job throughput: every rank processes its own batch of `units_per_rank` per step."""
+    return units_per_rank * world / (ms_per_step * 1e-3) * scale
+
+
 def _is_decode(wls) -> bool:
     return all(w.M <= 16 for w in wls)
 
@@ -289,10 +305,8 @@ def run_ours(args, rank, world, device_index):
         wall = time.perf_counter() - t0
     fn.flashnorm_check_device_error()
     dom_ms = sum(a.elapsed_time(b) for a, b in marks) / len(marks)
+    total_ms = max_over_ranks(total_ms, world, "cuda")
     if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
         torch.distributed.barrier()
     ms_per_step = total_ms / args.steps
 
@@ -322,17 +336,14 @@ def run_ours(args, rank, world, device_index):
         e2e_step(i)
     torch.cuda.synchronize()
     e2e_ms, _ = _time_back_to_back(torch, k_e2e, e2e_step)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, "cuda")
     h2d = sum(p.x[0].numel() * 2 for p in projs)
     d2h = sum(p.y[0].numel() * 2 for p in projs)
 
     units = _units(wls)
     scale = _scale(wls)
     metric, unit = _metric(wls)
-    value = units * world / (ms_per_step * 1e-3) * scale
+    value = weak_scaling_value(units, world, ms_per_step, scale)
     peaks = _peaks()
     w_dom = wls[dom]
     if _is_decode(wls):
@@ -378,7 +389,7 @@ def run_ours(args, rank, world, device_index):
             "parallelism": f"dp{world} (independent batches per GPU)",
         },
         "roofline": roof,
-        "e2e": {"value": units * world / (e2e_ms / k_e2e * 1e-3) * scale, "unit": unit,
+        "e2e": {"value": weak_scaling_value(units, world, e2e_ms / k_e2e, scale), "unit": unit,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e},
         "gpu_launches": args.steps * sum(p.launches() for p in projs),
         "clocks": sampler.summary(),

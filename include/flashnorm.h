@@ -58,12 +58,19 @@ typedef enum {
 typedef enum { FN_BF16 = 0, FN_F32 = 1 } fn_dtype;
 
 /* Which kernel family a projection runs on.
- *   FN_PATH_TENSOR  the persistent prefill kernel (128-row tiles of x, any M)
+ *   FN_PATH_TENSOR  the persistent prefill kernel, one CTA per 128-row tile (any M)
+ *   FN_PATH_PAIR    the persistent prefill kernel on CTA pairs: one 2-SM MMA per 256-row tile
  *   FN_PATH_GEMV    the CUDA-core GEMV (M <= FN_DECODE_MAX_M)
  *   FN_PATH_DECODE  the tensor-core decode kernel: W* rows on the MMA's M side, the tokens on its
  *                   N side, W* streamed once by TMA (M <= FN_DECODE_MAX_M)
- *   FN_PATH_AUTO    a decode kernel for M <= FN_DECODE_MAX_M, the prefill kernel otherwise */
-typedef enum { FN_PATH_AUTO = 0, FN_PATH_TENSOR = 1, FN_PATH_GEMV = 2, FN_PATH_DECODE = 3 } fn_path;
+ *   FN_PATH_AUTO    DECODE for M <= FN_DECODE_MAX_M, PAIR for M > 128, TENSOR otherwise */
+typedef enum {
+  FN_PATH_AUTO = 0,
+  FN_PATH_TENSOR = 1,
+  FN_PATH_GEMV = 2,
+  FN_PATH_DECODE = 3,
+  FN_PATH_PAIR = 4
+} fn_path;
 
 #define FN_DECODE_MAX_M 16
 /* GLU weights are stored gate/up interleaved in blocks of this many output columns (see fold). */

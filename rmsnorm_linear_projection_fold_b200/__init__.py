@@ -44,7 +44,7 @@ _LIB_PATH = os.path.join(_PKG_DIR, "libflashnorm.so")
 FN_OK, FN_ERR_INVALID_ARG, FN_ERR_UNSUPPORTED, FN_ERR_ALIGN, FN_ERR_CUDA, FN_ERR_TIMEOUT = range(6)
 FN_BF16, FN_F32 = 0, 1
 NOALLOC_MAX_ELEMS = 1 << 23  # FN_NOALLOC_MAX_ELEMS in include/flashnorm.h
-PATHS = {"auto": 0, "tensor": 1, "gemv": 2, "decode": 3}
+PATHS = {"auto": 0, "tensor": 1, "gemv": 2, "decode": 3, "pair": 4}
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64

@@ -14,6 +14,7 @@
 #include "decode_tc.cuh"
 #include "elementwise.cuh"
 #include "fused_gemm.cuh"
+#include "fused_gemm_pair.cuh"
 #include "gemv.cuh"
 #include "postnorm_cluster.cuh"
 
@@ -147,6 +148,71 @@ fn_status launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw, const fn::
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fused GEMM launch");
   return FN_OK;
+}
+
+// ---- CTA-pair (2-SM MMA) variant ------------------------------------------------------------------
+
+template <int STAGES, int EPI, bool SCALE, bool OUT_F32>
+fn_status launch_gemm_pair_t(const CUtensorMap& tx, const CUtensorMap& tw, const fn::GemmParams& p, int sms, int dev,
+                             cudaStream_t stream) {
+  auto kern = fn::k_fused_gemm_pair<STAGES, EPI, SCALE, OUT_F32>;
+  constexpr int smem = fn::gemm_pair_smem_bytes<STAGES>();
+  static bool configured[kMaxDevices] = {false};
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (pair GEMM)");
+    configured[dev] = true;
+  }
+  const int tiles = p.num_m_tiles * p.num_n_tiles;
+  const int pairs = tiles < sms / 2 ? tiles : sms / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(fn::gemm_threads(EPI, SCALE), 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
+  if (e != cudaSuccess) return cuda_fail(e, "pair GEMM launch");
+  return FN_OK;
+}
+
+fn_status run_pair_path(const void* x, const void* w, void* y, int64_t M, int64_t d, int64_t n_rows, int64_t n_out,
+                        float eps, int out_dtype, int epi, bool scale, cudaStream_t stream) {
+  int dev = 0;
+  const int sms = device_sm_count(&dev);
+  if (sms <= 1) return fail(FN_ERR_CUDA, "cannot query the current device");
+  // pair tiles are 256 rows; the choice of width counts pairs of SMs
+  const int bn = choose_bn((M + 1) / 2, n_rows, sms / 2, 32);
+  CUtensorMap tx, tw;
+  fn_status st = make_operand_map(&tx, x, d, M, fn::kBM);
+  if (st != FN_OK) return st;
+  st = make_operand_map(&tw, w, d, n_rows, bn / 2);
+  if (st != FN_OK) return st;
+  fn::GemmParams p;
+  p.y = y;
+  p.g2 = nullptr;
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(d);
+  p.n_out = static_cast<int>(n_out);
+  p.ldy = static_cast<int>(n_out);
+  p.bn = bn;
+  p.head_dim = 0;
+  p.num_m_tiles = static_cast<int>((M + 2 * fn::kBM - 1) / (2 * fn::kBM));
+  p.num_n_tiles = static_cast<int>((n_rows + bn - 1) / bn);
+  p.eps = eps;
+  const bool f32 = out_dtype == FN_F32;
+#define FN_PAIR(EPI, SC)                                                                                        \
+  (f32 ? launch_gemm_pair_t<fn::kPairStages, EPI, SC, true>(tx, tw, p, sms, dev, stream)                       \
+       : launch_gemm_pair_t<fn::kPairStages, EPI, SC, false>(tx, tw, p, sms, dev, stream))
+  if (epi == fn::EPI_LINEAR) return scale ? FN_PAIR(fn::EPI_LINEAR, true) : FN_PAIR(fn::EPI_LINEAR, false);
+  return scale ? FN_PAIR(fn::EPI_GLU, true) : FN_PAIR(fn::EPI_GLU, false);
+#undef FN_PAIR
 }
 
 // epi: fn::EpiKind; scale: apply the deferred 1/rms (sum of squares warpgroup on).
@@ -391,14 +457,19 @@ fn_status run_decode_tc(const void* x, const void* w, void* y, int64_t M, int64_
 fn_status projection(const void* x, const void* w, void* y, int64_t M, int64_t d, int64_t n_rows, int64_t n_out,
                      float eps, int out_dtype, int path, bool glu, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (path != FN_PATH_AUTO && path != FN_PATH_TENSOR && path != FN_PATH_GEMV && path != FN_PATH_DECODE)
+  if (path != FN_PATH_AUTO && path != FN_PATH_TENSOR && path != FN_PATH_GEMV && path != FN_PATH_DECODE &&
+      path != FN_PATH_PAIR)
     return fail(FN_ERR_INVALID_ARG, "path %d unknown", path);
   if (M == 0) return FN_OK;
   if (path == FN_PATH_DECODE) {
     if (M > FN_DECODE_MAX_M) return fail(FN_ERR_UNSUPPORTED, "decode path takes M <= %d", FN_DECODE_MAX_M);
     return run_decode_tc(x, w, y, M, d, n_rows, n_out, eps, out_dtype, glu, s);
   }
-  bool use_gemv = path == FN_PATH_GEMV || (path == FN_PATH_AUTO && M <= FN_DECODE_MAX_M && gemv_fits(M, d));
+  if (path == FN_PATH_PAIR || (path == FN_PATH_AUTO && M > fn::kBM))
+    return run_pair_path(x, w, y, M, d, n_rows, n_out, eps, out_dtype, glu ? fn::EPI_GLU : fn::EPI_LINEAR, true, s);
+  if (path == FN_PATH_AUTO && M <= FN_DECODE_MAX_M)
+    return run_decode_tc(x, w, y, M, d, n_rows, n_out, eps, out_dtype, glu, s);
+  bool use_gemv = path == FN_PATH_GEMV;
   if (use_gemv) {
     if (M > FN_DECODE_MAX_M) return fail(FN_ERR_UNSUPPORTED, "GEMV path takes M <= %d", FN_DECODE_MAX_M);
     if (!gemv_fits(M, d)) return fail(FN_ERR_UNSUPPORTED, "GEMV path: x [%lld, %lld] does not fit in shared memory",
@@ -508,6 +579,10 @@ static fn_status unfused(const void* x, const void* g, const void* Wk, void* xn_
   if ((st = check_ptr(xn_ws, "xn_ws")) != FN_OK) return st;
   st = flashnorm_rmsnorm(x, g, xn_ws, M, d, eps, stream);
   if (st != FN_OK) return st;
+  // the same GEMM kernel the fused path would pick, with the deferred scale switched off
+  if (M > fn::kBM)
+    return run_pair_path(xn_ws, Wk, y, M, d, n_rows, n_out, 0.0f, out_dtype, glu ? fn::EPI_GLU : fn::EPI_LINEAR,
+                         false, static_cast<cudaStream_t>(stream));
   return run_tensor_path(xn_ws, Wk, y, nullptr, M, d, n_rows, n_out, 0, 0.0f, out_dtype,
                          glu ? fn::EPI_GLU : fn::EPI_LINEAR, false, static_cast<cudaStream_t>(stream));
 }

@@ -1,0 +1,339 @@
+// fused_gemm_pair.cuh — the FlashNorm prefill kernel on CTA pairs (tcgen05 cta_group::2).
+//
+// Same computation and warp roles as fused_gemm.cuh (deferred normalisation of "FlashNorm: Fast
+// Normalization for Transformers", Abstract, item ii: x . W* on the tensor cores, sum of x^2 per row
+// on a separate warpgroup from the same staged x tiles, joined in the epilogue), but two CTAs of a
+// cluster share each MMA of M = 256 rows:
+//   * each CTA stages its own 128 rows of x and HALF of the tile's W* rows (split along N), so the W*
+//     bytes a CTA moves per MMA are halved and a stage shrinks from 48 KB to 32 KB (six stages fit);
+//   * the leader CTA (cluster rank 0) issues the pair MMA; both CTAs' TMA loads report to the
+//     leader's stage barrier, and the leader's commits arrive on both CTAs' barriers (commit
+//     multicast; every TMA load is an ordinary single-CTA fetch);
+//   * each CTA's tensor memory holds the accumulator of its own 128 rows, read by its own epilogue;
+//   * each CTA's sum-of-squares warps read only their own x tile; the leader forwards "stage landed"
+//     to both CTAs once the whole pair stage is in, and each stage is released only after the MMA
+//     and the CTA's own reduction warps are done with it (the explicit join of the 1-SM kernel).
+#pragma once
+
+#include "fused_gemm.cuh"
+
+namespace fn {
+
+constexpr int kPairStages = 6;
+constexpr int kPairBHalfRows = 128;                       // W* rows per CTA per stage, at most
+constexpr int kPairBStage = kPairBHalfRows * kBK * 2;     // 16 KB
+
+template <int STAGES>
+__host__ __device__ constexpr int gemm_pair_smem_bytes() {
+  return 1024 + STAGES * (kAStageBytes + kPairBStage) + 4096;
+}
+
+// p.num_m_tiles counts 256-row pair tiles; p.bn is the pair tile width (W* rows), each CTA holding bn/2.
+template <int STAGES, int EPI, bool SCALE, bool OUT_F32>
+__global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
+    k_fused_gemm_pair(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                      GemmParams p) {
+  constexpr int kSsWarps = SCALE ? 4 : 0;
+  constexpr int kEpiWarps = gemm_epi_warps(EPI);
+  constexpr int kEpiFirst = 2, kSsFirst = 2 + kEpiWarps;
+  static_assert(EPI != EPI_POSTNORM, "the pair kernel has no per-head post-norm epilogue");
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * kAStageBytes;
+  uint8_t* tail = sB + STAGES * kPairBStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tail);  // used in the leader
+  uint64_t* empty = full + STAGES;
+  uint64_t* xfull = empty + STAGES;                     // "x tile of this stage has landed" (reduction)
+  uint64_t* acc_full = xfull + STAGES;                  // [2]
+  uint64_t* acc_empty = acc_full + 2;                   // [2], used in the leader
+  uint64_t* ss_full = acc_empty + 2;                    // [2]
+  uint64_t* ss_empty = ss_full + 2;                     // [2]
+  uint64_t* drain = ss_empty + 2;                       // [1]
+  float* rinv = reinterpret_cast<float*>(drain + 1);    // [2][128]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rinv + 2 * kBM);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x) >> 5, 0);
+  const int lane = static_cast<int>(threadIdx.x) & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);  // the leader's expect-tx arrival covers both CTAs' bytes
+      mbar_init(&empty[s], 1 + kSsWarps);
+      mbar_init(&xfull[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 2 * kEpiWarps);
+      mbar_init(&ss_full[b], kBM);
+      mbar_init(&ss_empty[b], 32 * kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before either touches the other's
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = p.num_m_tiles * p.num_n_tiles;
+  const int cl = static_cast<int>(blockIdx.x) >> 1;
+  const int ncl = static_cast<int>(gridDim.x) >> 1;
+  const int t_begin = static_cast<int>(static_cast<long long>(cl) * num_tiles / ncl);
+  const int t_end = static_cast<int>(static_cast<long long>(cl + 1) * num_tiles / ncl);
+  const int num_kb = (p.K + kBK - 1) / kBK;
+  const int bn = p.bn;
+  const int half = bn / 2;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      // per CTA; the leader announces the whole pair stage, the peer's loads only complete on it
+      const uint32_t stage_bytes = static_cast<uint32_t>(kAStageBytes + half * kBK * 2);
+      int s = 0;
+      uint32_t ph = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = t_begin; t < t_end && ok; ++t) {
+        const int m0 = (t / p.num_n_tiles) * (2 * kBM) + static_cast<int>(rank) * kBM;
+        const int n0 = (t % p.num_n_tiles) * bn + static_cast<int>(rank) * half;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_cluster(&empty[s], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t leader_full = dsmem_addr(&full[s], 0);
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * stage_bytes);
+          tma_load_2d_pair(sA + s * kAStageBytes, &tm_x, leader_full, kb * kBK, m0);
+          tma_load_2d_pair(sB + s * kPairBStage, &tm_w, leader_full, kb * kBK, n0);
+          ++issued;
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok && leader) {
+        // Gave up: let the pair's copies still in flight land (bounded) before shared memory goes.
+        const int pending = issued < STAGES ? issued : STAGES;
+        for (int i = 1; i <= pending; ++i) {
+          int st = s - i;
+          uint32_t pp = ph;
+          if (st < 0) {
+            st += STAGES;
+            pp ^= 1u;
+          }
+          const unsigned long long t0 = globaltimer_ns();
+          while (!mbar_try_wait_cluster(&full[st], pp) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ pair MMA issuer (leader)
+    if (lane == 0 && leader) {
+      const uint32_t idesc = make_idesc_bf16(2 * kBM, bn);
+      int s = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t acc_ph = 0;
+      bool ok = true;
+      for (int t = t_begin; t < t_end && ok; ++t) {
+        if (!mbar_wait_cluster(&acc_empty[acc], acc_ph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_cluster(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          if (SCALE) {  // both CTAs' reduction warps may read their x tiles now
+            mbar_arrive(&xfull[s]);
+            mbar_arrive_remote(dsmem_addr(&xfull[s], 1));
+          }
+          const uint32_t a_addr = smem_u32(sA + s * kAStageBytes);
+          const uint32_t b_addr = smem_u32(sB + s * kPairBStage);
+#pragma unroll
+          for (int k = 0; k < kBK / kMmaK; ++k)
+            tc_mma_bf16_pair(d_tmem, make_sdesc_sw128(a_addr + k * kMmaK * 2),
+                             make_sdesc_sw128(b_addr + k * kMmaK * 2), idesc, (kb | k) != 0 ? 1u : 0u);
+          tc_commit_pair_mc(&empty[s], 0x3);  // frees stage s in both CTAs once read
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(&acc_full[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_ph ^= 1u;
+      }
+      if (!ok) {
+        tc_commit_pair_mc(drain, 0x1);
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else if (warp < kSsFirst) {
+    // ------------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const int hh = (warp - kEpiFirst) >> 2;  // which of the two warps on this lane quarter
+    const int row_in_tile = q * 32 + lane;
+    const uint32_t leader_acc_empty0 = dsmem_addr(&acc_empty[0], 0);
+    const uint32_t leader_acc_empty1 = dsmem_addr(&acc_empty[1], 0);
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    int sb = 0;
+    uint32_t sb_ph = 0;
+    for (int t = t_begin; t < t_end; ++t) {
+      const int mt = t / p.num_n_tiles;
+      const int nt = t % p.num_n_tiles;
+      if (!mbar_wait_cluster(&acc_full[acc], acc_ph, abort_flag)) break;
+      tc_fence_after_sync();
+      float r = 1.0f;
+      if (SCALE) {
+        if (!mbar_wait(&ss_full[sb], sb_ph, abort_flag)) break;
+        r = rinv[sb * kBM + row_in_tile];
+        mbar_arrive(&ss_empty[sb]);
+        sb ^= 1;
+        if (sb == 0) sb_ph ^= 1u;
+      }
+      const int row = mt * (2 * kBM) + static_cast<int>(rank) * kBM + row_in_tile;
+      const bool row_ok = row < p.M;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * 256);
+      if (EPI == EPI_LINEAR) {
+        const int col0 = nt * bn;
+        for (int c = hh * 16; c < bn; c += 64) {
+          const bool two = c + 32 < bn;
+          uint32_t v0[16], v1[16];
+          tmem_ld16(t_row + c, v0);
+          if (two) tmem_ld16(t_row + c + 32, v1);
+          tmem_ld_wait();
+          reg_fence16(v0);
+          float o[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(v0[j]) * r;
+          if (row_ok) store16<OUT_F32>(p.y, p.ldy, row, col0 + c, p.n_out, o);
+          if (two) {
+            reg_fence16(v1);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(v1[j]) * r;
+            if (row_ok) store16<OUT_F32>(p.y, p.ldy, row, col0 + c + 32, p.n_out, o);
+          }
+        }
+      } else {  // EPI_GLU
+        const int col0 = nt * (bn / 2);
+        for (int c = hh * 32; c < bn; c += 64) {
+          uint32_t gt[16], up[16];
+          tmem_ld16(t_row + c, gt);
+          tmem_ld16(t_row + c + 16, up);
+          tmem_ld_wait();
+          reg_fence16(gt);
+          reg_fence16(up);
+          float o[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float zg = __uint_as_float(gt[j]) * r;
+            const float zu = __uint_as_float(up[j]) * r;
+            o[j] = silu_f(zg) * zu;
+          }
+          if (row_ok) store16<OUT_F32>(p.y, p.ldy, row, col0 + c / 2, p.n_out, o);
+        }
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(&acc_empty[acc]);
+        else
+          mbar_arrive_remote(acc == 0 ? leader_acc_empty0 : leader_acc_empty1);
+      }
+      acc ^= 1;
+      if (acc == 0) acc_ph ^= 1u;
+    }
+  } else if (SCALE) {
+    // ------------------------------------------------------------------ sum of squares (both CTAs)
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    int s = 0;
+    uint32_t ph = 0;
+    int sb = 0;
+    uint32_t sb_ph = 0;
+    int last_m = -1;
+    float r_row = 0.0f;
+    bool ok = true;
+    for (int t = t_begin; t < t_end && ok; ++t) {
+      const int mt = t / p.num_n_tiles;
+      const bool fresh = mt != last_m;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait_cluster(&xfull[s], ph, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* line = sA + s * kAStageBytes + row_in_tile * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if (!fresh) break;
+          const uint4 w = *reinterpret_cast<const uint4*>(line + (((c ^ lane) & 7) << 4));
+          float f;
+          f = bf16lo_to_f32(w.x); a0 = fmaf(f, f, a0);
+          f = bf16hi_to_f32(w.x); a1 = fmaf(f, f, a1);
+          f = bf16lo_to_f32(w.y); a2 = fmaf(f, f, a2);
+          f = bf16hi_to_f32(w.y); a3 = fmaf(f, f, a3);
+          f = bf16lo_to_f32(w.z); a0 = fmaf(f, f, a0);
+          f = bf16hi_to_f32(w.z); a1 = fmaf(f, f, a1);
+          f = bf16lo_to_f32(w.w); a2 = fmaf(f, f, a2);
+          f = bf16hi_to_f32(w.w); a3 = fmaf(f, f, a3);
+        }
+        fence_proxy_async_smem();  // reads above before the TMA refill our arrival permits
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (fresh) {
+        const float ss = (a0 + a1) + (a2 + a3);
+        r_row = 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps);
+        last_m = mt;
+      }
+      if (!mbar_wait(&ss_empty[sb], sb_ph ^ 1u, abort_flag)) break;
+      rinv[sb * kBM + row_in_tile] = r_row;
+      mbar_arrive(&ss_full[sb]);
+      sb ^= 1;
+      if (sb == 0) sb_ph ^= 1u;
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  tc_fence_before_sync();
+  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while the other may still signal its barriers
+  tc_fence_after_sync();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
+}
+
+}  // namespace fn

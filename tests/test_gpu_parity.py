@@ -109,6 +109,11 @@ LINEAR_CASES = [
     (4, 4096, 1024, "gemv"),
     (16, 4096, 1024, "gemv"),
     (7, 264, 136, "gemv"),       # odd sizes on the GEMV path
+    (333, 576, 960, "pair"),     # 2-SM MMA: two 256-row pair tiles, the second ragged
+    (200, 4096, 512, "pair"),
+    (130, 72, 200, "pair"),      # ragged K and N; the peer CTA's rows are mostly past M
+    (17, 576, 960, "pair"),      # the peer CTA's rows are all past M
+    (2048, 576, 12288, "tensor"),  # many tiles per CTA on the 1-SM kernel
     (1, 4096, 1024, "decode"),   # tensor-core decode: 8 slabs -> K split over a 4-CTA cluster
     (4, 4096, 12288, "decode"),  # 96 slabs, no split
     (16, 4096, 1024, "decode"),
@@ -141,6 +146,8 @@ GLU_CASES = [
     (1, 4096, 512, "gemv"),
     (16, 4096, 512, "gemv"),
     (5, 576, 1536, "auto"),
+    (257, 576, 256, "pair"),
+    (600, 576, 1536, "pair"),
     (1, 4096, 512, "decode"),
     (16, 576, 1536, "decode"),
     (3, 4096, 11008, "decode"),
@@ -342,9 +349,10 @@ def test_invalid_arguments_raise():
         fn.flashnorm_linear(x, w, 1e-5, path="gemv")  # GEMV takes M <= 16
 
 
+@pytest.mark.parametrize("path", ["pair", "tensor"])
 @pytest.mark.parametrize("kind,M,d,N", [("linear", 2048, 576, 12288), ("glu", 2048, 576, 6144),
                                          ("linear", 8192, 576, 960)])
-def test_many_tiles_per_cta_all_rows(kind, M, d, N):
+def test_many_tiles_per_cta_all_rows(kind, M, d, N, path):
     """Every row, with several tiles per persistent CTA, three launches. A race between the
     sum-of-squares warps' shared-memory reads and the TMA refill of the same stage once corrupted
     1/rms on tiles after a CTA's first; only an all-rows fp32 check catches it reliably."""
@@ -354,7 +362,7 @@ def test_many_tiles_per_cta_all_rows(kind, M, d, N):
     ex = O.exact_operand_output(kind, bits, O.fold_bf16(bits["w"], bits["g"]), 1e-6)
     f = fn.flashnorm_linear if kind == "linear" else fn.flashnorm_glu
     for _ in range(3):
-        y32 = f(x, ws, 1e-6, out_dtype=torch.float32)
+        y32 = f(x, ws, 1e-6, out_dtype=torch.float32, path=path)
         torch.cuda.synchronize()
         assert O.rel_err(to_host_f64(y32), ex) <= F32_TOL
 
