@@ -63,7 +63,7 @@ typedef enum { FN_BF16 = 0, FN_F32 = 1 } fn_dtype;
  *   FN_PATH_GEMV    the CUDA-core GEMV (M <= FN_DECODE_MAX_M)
  *   FN_PATH_DECODE  the tensor-core decode kernel: W* rows on the MMA's M side, the tokens on its
  *                   N side, W* streamed once by TMA (M <= FN_DECODE_MAX_M)
- *   FN_PATH_AUTO    DECODE for M <= FN_DECODE_MAX_M, TENSOR otherwise */
+ *   FN_PATH_AUTO    DECODE for M <= FN_DECODE_MAX_M, PAIR for M > 128, TENSOR otherwise */
 typedef enum {
   FN_PATH_AUTO = 0,
   FN_PATH_TENSOR = 1,

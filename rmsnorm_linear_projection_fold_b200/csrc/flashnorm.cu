@@ -465,8 +465,8 @@ fn_status projection(const void* x, const void* w, void* y, int64_t M, int64_t d
     if (M > FN_DECODE_MAX_M) return fail(FN_ERR_UNSUPPORTED, "decode path takes M <= %d", FN_DECODE_MAX_M);
     return run_decode_tc(x, w, y, M, d, n_rows, n_out, eps, out_dtype, glu, s);
   }
-  // The pair kernel is correct but not yet faster than the 1-CTA kernel: only an explicit request uses it.
-  if (path == FN_PATH_PAIR)
+  // Prefill: CTA pairs (2-SM MMA) whenever there is more than one 128-row tile of x.
+  if (path == FN_PATH_PAIR || (path == FN_PATH_AUTO && M > fn::kBM))
     return run_pair_path(x, w, y, M, d, n_rows, n_out, eps, out_dtype, glu ? fn::EPI_GLU : fn::EPI_LINEAR, true, s);
   if (path == FN_PATH_AUTO && M <= FN_DECODE_MAX_M)
     return run_decode_tc(x, w, y, M, d, n_rows, n_out, eps, out_dtype, glu, s);
@@ -581,6 +581,9 @@ static fn_status unfused(const void* x, const void* g, const void* Wk, void* xn_
   st = flashnorm_rmsnorm(x, g, xn_ws, M, d, eps, stream);
   if (st != FN_OK) return st;
   // the same GEMM kernel the fused path picks, with the deferred scale switched off
+  if (M > fn::kBM)
+    return run_pair_path(xn_ws, Wk, y, M, d, n_rows, n_out, 0.0f, out_dtype, glu ? fn::EPI_GLU : fn::EPI_LINEAR,
+                         false, static_cast<cudaStream_t>(stream));
   return run_tensor_path(xn_ws, Wk, y, nullptr, M, d, n_rows, n_out, 0, 0.0f, out_dtype,
                          glu ? fn::EPI_GLU : fn::EPI_LINEAR, false, static_cast<cudaStream_t>(stream));
 }

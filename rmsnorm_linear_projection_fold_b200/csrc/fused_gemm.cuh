@@ -415,9 +415,11 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
       const bool fresh = mt != last_m;  // same for the whole CTA
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
       for (int kb = 0; kb < num_kb; ++kb) {
-        // Every stage is still waited for and released (the stage barriers count these arrivals),
-        // but it is only read when this row block's sum of squares is not known yet.
-        if (!mbar_wait(&full[s], ph, abort_flag)) {
+        // Every stage use still gets this warp's release (the stage barriers count it). When the row
+        // block's sum of squares is already known, the warp does not read the stage and releases it as
+        // soon as the stage's previous use has completed, i.e. before it is even refilled, so that it
+        // never delays the refill; otherwise it waits for the data and reads it.
+        if (!(fresh ? mbar_wait(&full[s], ph, abort_flag) : mbar_wait(&empty[s], ph ^ 1u, abort_flag))) {
           ok = false;
           break;
         }

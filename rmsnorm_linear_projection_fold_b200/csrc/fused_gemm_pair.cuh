@@ -287,7 +287,10 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
       const bool fresh = mt != last_m;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
       for (int kb = 0; kb < num_kb; ++kb) {
-        if (!mbar_wait_cluster(&xfull[s], ph, abort_flag)) {
+        // As in the 1-CTA kernel: with this row block's 1/rms already known, release each stage use as
+        // soon as its previous use has completed, without reading it (off the refill's critical path).
+        if (!(fresh ? mbar_wait_cluster(&xfull[s], ph, abort_flag)
+                    : mbar_wait_cluster(&empty[s], ph ^ 1u, abort_flag))) {
           ok = false;
           break;
         }

@@ -93,9 +93,14 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ---- cluster-scope mbarrier operations (CTA pairs of the 2-SM MMA) ----------------------------
-// Arrive on an mbarrier in another CTA of the cluster (address from dsmem_addr()).
+// Arrive on an mbarrier in another CTA of the cluster (address from dsmem_addr()). CTA-scope release,
+// as CUTLASS's cluster barriers use: a cluster-scope release here makes the arriving thread wait for
+// its outstanding asynchronous work (issued MMAs, commits) and serialised the pair pipeline (a
+// 2x slowdown, measured). What the receiver needs is ordered by other means: TMA data by the
+// transaction count of the barrier the MMA issuer waited on, tensor-memory reads by
+// tcgen05.wait::ld + tcgen05.fence::before_thread_sync before the arrival.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_addr, uint32_t bytes) {
