@@ -62,6 +62,7 @@ DEFAULT_WORKLOAD = "smollm2_prefill_m8192"
 # if the CUDA sources hash differently now, traffic is reported as null.
 NCU_TRAFFIC = {
     # workload: (bytes per launch, sha256[:16] of the csrc/*.cu* sources at capture time, profile file)
+    "smollm2_prefill_m8192": (13077504, "376fc8fb0e36e66e", "profiles/fused_gemm_pair_smollm2_ffn_m8192.md"),
 }
 
 L2_BYTES = 126 * 1000 * 1000
