@@ -54,6 +54,8 @@ BENCH_WORKLOADS = {
     "llama7b_qkv_m2048": ["llama7b_qkv_m2048"],
     "llama7b_ffn_m2048": ["llama7b_ffn_m2048"],
     "mla_latent_m2048": ["mla_latent_m2048"],
+    "gemma_qkvnorm_hd256_m2048": ["gemma_qkvnorm_hd256_m2048"],
+    "gemma_qkvnorm_hd128_m2048": ["gemma_qkvnorm_hd128_m2048"],
 }
 DEFAULT_WORKLOAD = "smollm2_prefill_m8192"
 

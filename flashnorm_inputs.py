@@ -124,6 +124,12 @@ WORKLOADS = {
     "llama7b_ffn_m2048": Workload("llama7b_ffn_m2048", "glu", 2048, 4096, 11008, 1e-6, seed=BASE_SEED + 3),
     "mla_latent_m2048": Workload("mla_latent_m2048", "postnorm", 2048, 5120, 512, 1e-6,
                                  head_dim=512, eps2=1e-6, seed=BASE_SEED + 4),
+    # Per-head QKV normalisation at Gemma-like widths (model dimension 2560, 16 heads of 256 or 32 of
+    # 128 over the concatenated q/k/v projections): the pre-attention RMSNorm is elided.
+    "gemma_qkvnorm_hd256_m2048": Workload("gemma_qkvnorm_hd256_m2048", "postnorm", 2048, 2560, 4096, 1e-6,
+                                          head_dim=256, eps2=1e-6, seed=BASE_SEED + 5),
+    "gemma_qkvnorm_hd128_m2048": Workload("gemma_qkvnorm_hd128_m2048", "postnorm", 2048, 2560, 4096, 1e-6,
+                                          head_dim=128, eps2=1e-6, seed=BASE_SEED + 6),
 }
 
 

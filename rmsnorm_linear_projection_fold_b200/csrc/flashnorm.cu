@@ -187,8 +187,10 @@ fn_status run_pair_path(const void* x, const void* w, void* y, int64_t M, int64_
   int dev = 0;
   const int sms = device_sm_count(&dev);
   if (sms <= 1) return fail(FN_ERR_CUDA, "cannot query the current device");
-  // pair tiles are 256 rows; the choice of width counts pairs of SMs
-  const int bn = choose_bn((M + 1) / 2, n_rows, sms / 2, 32);
+  // Pair tiles are 256 rows; the choice of width counts pairs of SMs. A tile's output columns are a
+  // whole number of the epilogue's 64-byte chunks (32 bf16 outputs, i.e. 64 W* rows for the GLU).
+  const int bn = choose_bn((M + 1) / 2, n_rows, sms / 2,
+                           epi == fn::EPI_GLU ? 2 * fn::pair_chunk_cols(out_dtype == FN_F32) : 32);
   CUtensorMap tx, tw;
   fn_status st = make_operand_map(&tx, x, d, M, fn::kBM);
   if (st != FN_OK) return st;

@@ -12,7 +12,10 @@
 //   * each CTA's tensor memory holds the accumulator of its own 128 rows, read by its own epilogue;
 //   * each CTA's sum-of-squares warps read only their own x tile; the leader forwards "stage landed"
 //     to both CTAs once the whole pair stage is in, and each stage is released only after the MMA
-//     and the CTA's own reduction warps are done with it (the explicit join of the 1-SM kernel).
+//     and the CTA's own reduction warps are done with it (the explicit join of the 1-SM kernel);
+//   * the epilogue stages each warp's 32 rows x 64 bytes of output in swizzled shared memory and writes
+//     them back row-contiguously (8 rows x 64 bytes per warp store) instead of every lane storing its
+//     own row (32 cache lines per warp store, which made the epilogue as long as a short-K tile).
 #pragma once
 
 #include "fused_gemm.cuh"
@@ -20,13 +23,18 @@
 namespace fn {
 
 constexpr int kPairStages = 6;
+constexpr int kPairStageOutBytes = 32 * 64;  // per epilogue warp: 32 rows x 64 bytes of y
 constexpr int kPairBHalfRows = 128;                       // W* rows per CTA per stage, at most
 constexpr int kPairBStage = kPairBHalfRows * kBK * 2;     // 16 KB
 
 template <int STAGES>
 __host__ __device__ constexpr int gemm_pair_smem_bytes() {
-  return 1024 + STAGES * (kAStageBytes + kPairBStage) + 4096;
+  return 1024 + STAGES * (kAStageBytes + kPairBStage) + 8 * kPairStageOutBytes + 4096;
 }
+
+// Output columns per staged chunk (64 bytes of a row). The pair kernel's tile width is chosen so that
+// every tile's output columns are a whole number of chunks.
+__host__ __device__ constexpr int pair_chunk_cols(bool out_f32) { return out_f32 ? 16 : 32; }
 
 // p.num_m_tiles counts 256-row pair tiles; p.bn is the pair tile width (W* rows), each CTA holding bn/2.
 template <int STAGES, int EPI, bool SCALE, bool OUT_F32>
@@ -43,7 +51,8 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kAStageBytes;
-  uint8_t* tail = sB + STAGES * kPairBStage;
+  uint8_t* sOut = sB + STAGES * kPairBStage;  // [8 epilogue warps][32 rows x 64 B], swizzled
+  uint8_t* tail = sOut + 8 * kPairStageOutBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(tail);  // used in the leader
   uint64_t* empty = full + STAGES;
   uint64_t* xfull = empty + STAGES;                     // "x tile of this stage has landed" (reduction)
@@ -218,47 +227,97 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
         sb ^= 1;
         if (sb == 0) sb_ph ^= 1u;
       }
-      const int row = mt * (2 * kBM) + static_cast<int>(rank) * kBM + row_in_tile;
-      const bool row_ok = row < p.M;
+      // rows of this warp's lane quarter in y, and its staging buffer
+      const int qrow0 = mt * (2 * kBM) + static_cast<int>(rank) * kBM + q * 32;
+      uint8_t* stage_out = sOut + (warp - kEpiFirst) * kPairStageOutBytes;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * 256);
-      if (EPI == EPI_LINEAR) {
-        const int col0 = nt * bn;
-        for (int c = hh * 16; c < bn; c += 64) {
-          const bool two = c + 32 < bn;
-          uint32_t v0[16], v1[16];
-          tmem_ld16(t_row + c, v0);
-          if (two) tmem_ld16(t_row + c + 32, v1);
-          tmem_ld_wait();
-          reg_fence16(v0);
-          float o[16];
+      constexpr int CC = pair_chunk_cols(OUT_F32);
+      constexpr int kEsz = OUT_F32 ? 4 : 2;
+      const int ocols = EPI == EPI_GLU ? bn / 2 : bn;
+      const int ocol0 = nt * ocols;
+      // 16-byte piece j (0..3) of row r sits at r*64 + ((j ^ (r >> 1)) & 3) * 16: conflict-free both for
+      // a quarter-warp writing one piece of eight rows and for one reading two whole rows.
+      auto put16 = [&](int j, uint4 v) {
+        *reinterpret_cast<uint4*>(stage_out + lane * 64 + (((j ^ (lane >> 1)) & 3) << 4)) = v;
+      };
+      for (int ch = hh; ch * CC < ocols && ocol0 + ch * CC < p.n_out; ch += 2) {
+        if (EPI == EPI_LINEAR) {
+          if (OUT_F32) {  // 16 columns -> 4 pieces
+            uint32_t v0[16];
+            tmem_ld16(t_row + ch * CC, v0);
+            tmem_ld_wait();
+            reg_fence16(v0);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(v0[j]) * r;
-          if (row_ok) store16<OUT_F32>(p.y, p.ldy, row, col0 + c, p.n_out, o);
-          if (two) {
+            for (int j = 0; j < 4; ++j)
+              put16(j, make_uint4(__float_as_uint(__uint_as_float(v0[4 * j]) * r),
+                                  __float_as_uint(__uint_as_float(v0[4 * j + 1]) * r),
+                                  __float_as_uint(__uint_as_float(v0[4 * j + 2]) * r),
+                                  __float_as_uint(__uint_as_float(v0[4 * j + 3]) * r)));
+          } else {  // 32 columns -> 4 pieces
+            uint32_t v0[16], v1[16];
+            tmem_ld16(t_row + ch * CC, v0);
+            tmem_ld16(t_row + ch * CC + 16, v1);
+            tmem_ld_wait();
+            reg_fence16(v0);
             reg_fence16(v1);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(v1[j]) * r;
-            if (row_ok) store16<OUT_F32>(p.y, p.ldy, row, col0 + c + 32, p.n_out, o);
+            for (int j = 0; j < 2; ++j) {
+              put16(j, make_uint4(pack_bf16x2(__uint_as_float(v0[8 * j]) * r, __uint_as_float(v0[8 * j + 1]) * r),
+                                  pack_bf16x2(__uint_as_float(v0[8 * j + 2]) * r, __uint_as_float(v0[8 * j + 3]) * r),
+                                  pack_bf16x2(__uint_as_float(v0[8 * j + 4]) * r, __uint_as_float(v0[8 * j + 5]) * r),
+                                  pack_bf16x2(__uint_as_float(v0[8 * j + 6]) * r, __uint_as_float(v0[8 * j + 7]) * r)));
+              put16(2 + j, make_uint4(pack_bf16x2(__uint_as_float(v1[8 * j]) * r, __uint_as_float(v1[8 * j + 1]) * r),
+                                      pack_bf16x2(__uint_as_float(v1[8 * j + 2]) * r, __uint_as_float(v1[8 * j + 3]) * r),
+                                      pack_bf16x2(__uint_as_float(v1[8 * j + 4]) * r, __uint_as_float(v1[8 * j + 5]) * r),
+                                      pack_bf16x2(__uint_as_float(v1[8 * j + 6]) * r, __uint_as_float(v1[8 * j + 7]) * r)));
+            }
           }
-        }
-      } else {  // EPI_GLU
-        const int col0 = nt * (bn / 2);
-        for (int c = hh * 32; c < bn; c += 64) {
-          uint32_t gt[16], up[16];
-          tmem_ld16(t_row + c, gt);
-          tmem_ld16(t_row + c + 16, up);
-          tmem_ld_wait();
-          reg_fence16(gt);
-          reg_fence16(up);
-          float o[16];
+        } else {
+          // CC output columns = CC/16 (gate 16, up 16) pairs of accumulator columns
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float zg = __uint_as_float(gt[j]) * r;
-            const float zu = __uint_as_float(up[j]) * r;
-            o[j] = silu_f(zg) * zu;
+          for (int b = 0; b < CC / 16; ++b) {
+            uint32_t gt[16], up[16];
+            const int acol = 2 * (ch * CC) + 32 * b;
+            tmem_ld16(t_row + acol, gt);
+            tmem_ld16(t_row + acol + 16, up);
+            tmem_ld_wait();
+            reg_fence16(gt);
+            reg_fence16(up);
+            float o[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float zg = __uint_as_float(gt[j]) * r;
+              const float zu = __uint_as_float(up[j]) * r;
+              o[j] = silu_f(zg) * zu;
+            }
+            if (OUT_F32) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                put16(j, make_uint4(__float_as_uint(o[4 * j]), __float_as_uint(o[4 * j + 1]),
+                                    __float_as_uint(o[4 * j + 2]), __float_as_uint(o[4 * j + 3])));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+                put16(2 * b + j, make_uint4(pack_bf16x2(o[8 * j], o[8 * j + 1]), pack_bf16x2(o[8 * j + 2], o[8 * j + 3]),
+                                            pack_bf16x2(o[8 * j + 4], o[8 * j + 5]), pack_bf16x2(o[8 * j + 6], o[8 * j + 7])));
+            }
           }
-          if (row_ok) store16<OUT_F32>(p.y, p.ldy, row, col0 + c / 2, p.n_out, o);
         }
+        __syncwarp();
+        // write back: lane l copies piece (l & 3) of rows 8i + (l >> 2); a 16-byte piece lies wholly inside
+        // or wholly past column n_out (n_out is a multiple of 8).
+        const int seg = lane & 3;
+        const int col = ocol0 + ch * CC + seg * (16 / kEsz);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int rr = 8 * i + (lane >> 2);
+          const uint4 v = *reinterpret_cast<const uint4*>(stage_out + rr * 64 + (((seg ^ (rr >> 1)) & 3) << 4));
+          const int row = qrow0 + rr;
+          if (row < p.M && col < p.n_out)
+            *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.y) +
+                                      (static_cast<size_t>(row) * p.ldy + col) * kEsz) = v;
+        }
+        __syncwarp();  // the staging buffer is read before the next chunk overwrites it
       }
       tc_fence_before_sync();
       __syncwarp();

@@ -238,7 +238,8 @@ def test_folded_unfolded_oracle_agree_smollm2_m64():
 
 # ------------------------------------------------------------------------------------------ full sizes, sampled
 FULL = ["smollm2_qkv_m8192", "smollm2_ffn_m8192", "llama7b_qkv_m1", "llama7b_qkv_m4", "llama7b_qkv_m16",
-        "llama7b_qkv_m2048", "llama7b_ffn_m2048", "mla_latent_m2048"]
+        "llama7b_qkv_m2048", "llama7b_ffn_m2048", "mla_latent_m2048", "gemma_qkvnorm_hd256_m2048",
+        "gemma_qkvnorm_hd128_m2048"]
 
 
 @pytest.mark.parametrize("name", FULL)
