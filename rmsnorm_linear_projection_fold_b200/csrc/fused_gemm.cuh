@@ -77,11 +77,13 @@ __host__ __device__ constexpr int gemm_smem_bytes() {
 
 // silu(z) = z * sigmoid(z), with exp and the reciprocal taken on the special-function unit:
 // sigmoid(z) = 1 / (1 + 2^(-z * log2(e))). Relative error ~1e-6; the limits are exact (z -> -inf
-// gives 2^+inf = inf and rcp(inf) = 0; z -> +inf gives rcp(1) = 1).
+// gives 2^+inf = inf and rcp(inf) = 0; z -> +inf gives rcp(1) = 1). The flush-to-zero forms are one
+// SFU instruction each; flushing only matters where 2^(-z log2 e) is subnormal (z > 87), and there
+// 1 + e is 1 either way.
 __device__ __forceinline__ float silu_f(float z) {
   float e, s;
-  asm("ex2.approx.f32 %0, %1;" : "=f"(e) : "f"(-z * 1.4426950408889634f));
-  asm("rcp.approx.f32 %0, %1;" : "=f"(s) : "f"(1.0f + e));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-z * 1.4426950408889634f));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(s) : "f"(1.0f + e));
   return z * s;
 }
 

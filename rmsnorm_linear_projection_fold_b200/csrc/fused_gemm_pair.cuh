@@ -240,7 +240,9 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
       auto put16 = [&](int j, uint4 v) {
         *reinterpret_cast<uint4*>(stage_out + lane * 64 + (((j ^ (lane >> 1)) & 3) << 4)) = v;
       };
-      for (int ch = hh; ch * CC < ocols && ocol0 + ch * CC < p.n_out; ch += 2) {
+      // The two warps of a lane quarter take alternate chunks; which one starts alternates from tile to
+      // tile, so an odd chunk count does not always land on the same warp.
+      for (int ch = (hh + t - t_begin) & 1; ch * CC < ocols && ocol0 + ch * CC < p.n_out; ch += 2) {
         if (EPI == EPI_LINEAR) {
           if (OUT_F32) {  // 16 columns -> 4 pieces
             uint32_t v0[16];
