@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dep_wait();  // the previous kernel's outputs (our inputs, or buffers we overwrite) are complete
 
   if (warp == 0) {
     if (lane == 0) {
@@ -111,6 +112,18 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (++s == STAGES) {
           s = 0;
           ph ^= 1u;
+        }
+      }
+      grid_dep_launch();  // all loads issued: the next kernel may be scheduled onto SMs as they free up
+      if (ok) {
+        // Wait for the release of the last use of every stage, so that no arrival on this CTA's barriers
+        // (an MMA commit completes asynchronously) is still in flight when the CTA exits.
+        for (int i = 0; i < STAGES; ++i) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) break;
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
       }
       if (!ok) {

@@ -28,6 +28,7 @@ __global__ void __launch_bounds__(256) k_fold(const uint16_t* __restrict__ W, co
   const int k0 = blockIdx.y * kFoldTile;
   const int n0 = blockIdx.x * kFoldTile;
   const int F = N / 2;
+  grid_dep_wait();
   // load: 64 rows (k) x 8 chunks of 8 columns (n)
   for (int i = threadIdx.x; i < kFoldTile * 8; i += 256) {
     const int kk = i >> 3, ch = i & 7;
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const uint16_t* __restrict__ x,
                                                  uint16_t* __restrict__ xn, int M, int K, float eps) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + warp;
+  grid_dep_wait();
   if (row >= M) return;
   const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(row) * K);
   const uint4* gr = reinterpret_cast<const uint4*>(g);

@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/flashnorm.h"
 #include "decode_tc.cuh"
@@ -47,6 +48,35 @@ int device_sm_count(int* dev_out) {
   }
   *dev_out = dev;
   return sms[dev];
+}
+
+// Every kernel is launched with programmatic stream serialization: it may be scheduled while the
+// previous kernel of the stream drains, runs its prologue (barriers, tensor memory), and then waits in
+// the kernel (griddepcontrol.wait) for that kernel's completion before it touches global memory.
+// cluster > 1 adds a cluster dimension.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          unsigned cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda dependency).
@@ -144,8 +174,8 @@ fn_status launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw, const fn::
   }
   const int tiles = p.num_m_tiles * p.num_n_tiles;
   const int grid = tiles < sms ? tiles : sms;
-  kern<<<grid, fn::gemm_threads(EPI, SCALE), smem, stream>>>(tx, tw, p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(fn::gemm_threads(EPI, SCALE)), smem,
+                                stream, 1, tx, tw, p);
   if (e != cudaSuccess) return cuda_fail(e, "fused GEMM launch");
   return FN_OK;
 }
@@ -165,19 +195,8 @@ fn_status launch_gemm_pair_t(const CUtensorMap& tx, const CUtensorMap& tw, const
   }
   const int tiles = p.num_m_tiles * p.num_n_tiles;
   const int pairs = tiles < sms / 2 ? tiles : sms / 2;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
-  cfg.blockDim = dim3(fn::gemm_threads(EPI, SCALE), 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
+  cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(2 * pairs)), dim3(fn::gemm_threads(EPI, SCALE)),
+                                smem, stream, 2, tx, tw, p);
   if (e != cudaSuccess) return cuda_fail(e, "pair GEMM launch");
   return FN_OK;
 }
@@ -277,19 +296,8 @@ fn_status launch_postnorm_cluster_t(const CUtensorMap& tx, const CUtensorMap& tw
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (post-norm cluster)");
     configured[dev] = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
-  cfg.blockDim = dim3(fn::kPnThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(p.cn * p.ks);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
+  cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(ctas)), dim3(fn::kPnThreads), smem, stream,
+                                static_cast<unsigned>(p.cn * p.ks), tx, tw, p);
   if (e != cudaSuccess) return cuda_fail(e, "post-norm cluster launch");
   return FN_OK;
 }
@@ -348,10 +356,10 @@ fn_status launch_gemv_t(const void* x, const void* w, void* y, int64_t M, int64_
   if (per_sm < 1) per_sm = 1;
   int64_t grid = static_cast<int64_t>(sms) * per_sm;
   if (blocks_needed < grid) grid = blocks_needed;
-  kern<<<static_cast<unsigned>(grid), fn::kGemvThreads, smem, stream>>>(
-      static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w), y, static_cast<int>(M), static_cast<int>(d),
-      static_cast<int>(n_units), static_cast<int>(n_units), eps);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(fn::kGemvThreads),
+                                static_cast<size_t>(smem), stream, 1, static_cast<const uint16_t*>(x),
+                                static_cast<const uint16_t*>(w), y, static_cast<int>(M), static_cast<int>(d),
+                                static_cast<int>(n_units), static_cast<int>(n_units), eps);
   if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");
   return FN_OK;
 }
@@ -401,19 +409,8 @@ fn_status launch_decode_t(const CUtensorMap& tw, const CUtensorMap& tx, const fn
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (decode)");
     configured[dev] = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(slabs * KSPLIT), 1, 1);
-  cfg.blockDim = dim3(fn::kDecThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = KSPLIT;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, p);
+  cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(slabs * KSPLIT)), dim3(fn::kDecThreads), smem,
+                                stream, KSPLIT, tw, tx, p);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return FN_OK;
 }
@@ -501,10 +498,9 @@ fn_status flashnorm_fold_weights(const void* W, const void* g, void* Wstar, int6
   dim3 grid(static_cast<unsigned>((N + fn::kFoldTile - 1) / fn::kFoldTile),
             static_cast<unsigned>((d + fn::kFoldTile - 1) / fn::kFoldTile));
   if (grid.y > 65535) return fail(FN_ERR_UNSUPPORTED, "d too large for the fold grid");
-  fn::k_fold<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint16_t*>(W), static_cast<const uint16_t*>(g), static_cast<uint16_t*>(Wstar),
-      static_cast<int>(d), static_cast<int>(N), glu);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(fn::k_fold, grid, dim3(256), 0, static_cast<cudaStream_t>(stream), 1,
+                                static_cast<const uint16_t*>(W), static_cast<const uint16_t*>(g),
+                                static_cast<uint16_t*>(Wstar), static_cast<int>(d), static_cast<int>(N), glu);
   if (e != cudaSuccess) return cuda_fail(e, "fold launch");
   return FN_OK;
 }
@@ -565,10 +561,10 @@ fn_status flashnorm_rmsnorm(const void* x, const void* g, void* xn, int64_t M, i
   if ((st = check_ptr(x, "x")) != FN_OK) return st;
   if ((st = check_ptr(xn, "xn")) != FN_OK) return st;
   const int64_t blocks = (M + 7) / 8;
-  fn::k_rmsnorm<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(g), static_cast<uint16_t*>(xn),
-      static_cast<int>(M), static_cast<int>(d), eps);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(fn::k_rmsnorm, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                                static_cast<cudaStream_t>(stream), 1, static_cast<const uint16_t*>(x),
+                                static_cast<const uint16_t*>(g), static_cast<uint16_t*>(xn), static_cast<int>(M),
+                                static_cast<int>(d), eps);
   if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
   return FN_OK;
 }

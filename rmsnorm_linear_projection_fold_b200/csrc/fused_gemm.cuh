@@ -174,6 +174,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dep_wait();  // the previous kernel's outputs (our inputs, or buffers we overwrite) are complete
 
   // Tile schedule: the tiles are numbered row-block-major (t -> m = t / num_n, n = t % num_n) and each
   // CTA takes one contiguous, balanced range of them. Consecutive tiles of a CTA then mostly share
@@ -208,6 +209,18 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
           tma_load_2d(b_dst, &tm_w, &full[s], kb * kBK, n0);
           if (bn > 256) tma_load_2d(b_dst + box_rows * kBK * 2, &tm_w, &full[s], kb * kBK, n0 + box_rows);
           ++issued;
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      grid_dep_launch();  // all loads issued: the next kernel may be scheduled onto SMs as they free up
+      if (ok) {
+        // Wait for the release of the last use of every stage, so that no arrival on this CTA's barriers
+        // (an MMA commit completes asynchronously) is still in flight when the CTA exits.
+        for (int i = 0; i < STAGES; ++i) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) break;
           if (++s == STAGES) {
             s = 0;
             ph ^= 1u;

@@ -99,6 +99,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
   cluster_sync_all();  // both CTAs' barriers exist before either touches the other's
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dep_wait();  // the previous kernel's outputs (our inputs, or buffers we overwrite) are complete
 
   const int num_tiles = p.num_m_tiles * p.num_n_tiles;
   const int cl = static_cast<int>(blockIdx.x) >> 1;
@@ -131,6 +132,18 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
           tma_load_2d_pair(sA + s * kAStageBytes, &tm_x, leader_full, kb * kBK, m0);
           tma_load_2d_pair(sB + s * kPairBStage, &tm_w, leader_full, kb * kBK, n0);
           ++issued;
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      grid_dep_launch();  // all loads issued: the next kernel may be scheduled onto SMs as they free up
+      if (ok) {
+        // Wait for the release of the last use of every stage, so that no arrival on this CTA's barriers
+        // (an MMA commit completes asynchronously) is still in flight when the CTA exits.
+        for (int i = 0; i < STAGES; ++i) {
+          if (!mbar_wait_cluster(&empty[s], ph ^ 1u, abort_flag)) break;
           if (++s == STAGES) {
             s = 0;
             ph ^= 1u;

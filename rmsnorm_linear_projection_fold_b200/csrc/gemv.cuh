@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(kGemvThreads) k_gemv(const uint16_t* __restric
   float* rs = reinterpret_cast<float*>(reinterpret_cast<uint16_t*>(smem_v) + MT * K);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kc = K >> 3;
+  grid_dep_wait();
 
   for (int i = threadIdx.x; i < MT * kc; i += kGemvThreads) {
     const int m = i / kc, c = i - m * kc;

@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(kPnThreads, 1)
     tmem_alloc(tmem_slot, kPnCols);
     tmem_relinquish();
   }
+  grid_dep_wait();  // the previous kernel's outputs (our inputs, or buffers we overwrite) are complete
   for (int i = static_cast<int>(threadIdx.x); i < p.head_dim; i += kPnThreads)
     g2s[i] = __uint_as_float(static_cast<uint32_t>(p.g2[i]) << 16);
   tc_fence_before_sync();
@@ -122,6 +123,18 @@ __global__ void __launch_bounds__(kPnThreads, 1)
         if (++s == kPnStages) {
           s = 0;
           ph ^= 1u;
+        }
+      }
+      grid_dep_launch();  // all loads issued: the next kernel may be scheduled onto SMs as they free up
+      if (ok) {
+        // Wait for the release of the last use of every stage, so that no arrival on this CTA's barriers
+        // (an MMA commit completes asynchronously) is still in flight when the CTA exits.
+        for (int i = 0; i < kPnStages; ++i) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) break;
+          if (++s == kPnStages) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
       }
       if (!ok) {

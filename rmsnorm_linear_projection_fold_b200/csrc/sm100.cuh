@@ -227,6 +227,16 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
       : "memory");
 }
 
+// Programmatic dependent launch. A kernel launched with programmatic stream serialization may start
+// while the previous kernel in its stream is still running: it sets up its barriers and tensor memory,
+// then waits here until that kernel has completed and its writes are visible, before touching global
+// memory. Without the launch attribute the wait returns at once.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next kernel of the stream (if launched as above) be scheduled once every CTA of this grid
+// has issued it or exited. Only scheduling moves earlier; the next kernel still waits for our completion.
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
