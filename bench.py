@@ -47,6 +47,8 @@ import flashnorm_inputs as I  # noqa: E402
 # ----------------------------------------------------------------------------------------------
 BENCH_WORKLOADS = {
     "smollm2_prefill_m8192": ["smollm2_qkv_m8192", "smollm2_ffn_m8192"],
+    "smollm2_qkv_m8192": ["smollm2_qkv_m8192"],
+    "smollm2_ffn_m8192": ["smollm2_ffn_m8192"],
     "smollm2_qkv_m64": ["smollm2_qkv_m64"],
     "llama7b_qkv_m1": ["llama7b_qkv_m1"],
     "llama7b_qkv_m4": ["llama7b_qkv_m4"],

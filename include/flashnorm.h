@@ -180,6 +180,16 @@ FN_API fn_status flashnorm_linear_unfused_noalloc(const void* x, const void* g, 
  */
 FN_API fn_status flashnorm_check_device_error(void* stream);
 
+/*
+ * flashnorm_selftest_timeout — exercises the failure path without faulting anything: launches one
+ * thread that waits on a device barrier nothing will complete, bounded by `limit_us` microseconds
+ * (and as many thousand SM cycles), then synchronises `stream` and reads the status word like
+ * flashnorm_check_device_error. A working library returns FN_ERR_TIMEOUT here and leaves the word
+ * cleared and the CUDA context usable for the next call. limit_us must be in [1, 1e7]. (The pages
+ * have no counterpart: this checks the library's own bounded waits.)
+ */
+FN_API fn_status flashnorm_selftest_timeout(int64_t limit_us, void* stream);
+
 /* Static description of a status code. */
 FN_API const char* flashnorm_status_string(int status);
 /* Detail of the most recent failed call on this host thread ("" if none). */

@@ -34,6 +34,7 @@ __all__ = [
     "flashnorm_linear_unfused_noalloc",
     "NOALLOC_MAX_ELEMS",
     "flashnorm_check_device_error",
+    "flashnorm_selftest_timeout",
     "flashnorm_version",
     "EXPORTED_SYMBOLS",
 ]
@@ -64,6 +65,7 @@ _SIGNATURES = {
     "flashnorm_glu_unfused": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_linear_unfused_noalloc": [_P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_check_device_error": [_P],
+    "flashnorm_selftest_timeout": [_I64, _P],
     "flashnorm_status_string": [_INT],
     "flashnorm_last_error": [],
     "flashnorm_version": [],
@@ -283,6 +285,15 @@ def flashnorm_check_device_error(device=None) -> None:
     lib = load_library()
     s = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     _check("flashnorm_check_device_error", lib.flashnorm_check_device_error(s))
+
+
+def flashnorm_selftest_timeout(limit_us: int = 20000, device=None) -> int:
+    """Run the bounded-wait self-test; returns the status the library reported (FN_ERR_TIMEOUT when the
+    failure path works). Does not raise for that status."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+    lib = load_library()
+    s = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    return int(lib.flashnorm_selftest_timeout(int(limit_us), s))
 
 
 def flashnorm_version() -> int:

@@ -71,6 +71,21 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // One warp per row, 8 rows per block. Pass 1 sums squares, pass 2 (L1/L2 hits) scales and stores.
+// Failure-detection self-test: one thread waits on an mbarrier that nothing will ever arrive at. The
+// bounded wait runs out after limit_ns (and as many SM cycles), records the timeout in the device
+// status word and the kernel returns normally.
+__global__ void __launch_bounds__(32) k_wait_selftest(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    mbar_init_fence();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) mbar_wait_limited(&bar, 0, &abort_flag, limit_ns, static_cast<long long>(limit_ns));
+}
+
 __global__ void __launch_bounds__(256) k_rmsnorm(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g,
                                                  uint16_t* __restrict__ xn, int M, int K, float eps) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

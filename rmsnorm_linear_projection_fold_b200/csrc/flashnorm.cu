@@ -667,6 +667,16 @@ fn_status flashnorm_check_device_error(void* stream) {
   return FN_OK;
 }
 
+fn_status flashnorm_selftest_timeout(int64_t limit_us, void* stream) {
+  g_last_error[0] = '\0';
+  if (limit_us < 1 || limit_us > 10000000) return fail(FN_ERR_INVALID_ARG, "limit_us must be in [1, 1e7]");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_kernel(fn::k_wait_selftest, dim3(1), dim3(32), 0, s, 1,
+                                static_cast<unsigned long long>(limit_us) * 1000ull);
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return flashnorm_check_device_error(stream);
+}
+
 const char* flashnorm_status_string(int status) {
   switch (status) {
     case FN_OK: return "FN_OK";

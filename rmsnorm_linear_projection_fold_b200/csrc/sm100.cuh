@@ -15,8 +15,17 @@ __device__ unsigned int g_device_status;
 constexpr unsigned int kStatusTimeout = 1u;
 
 // A wait that has not completed after this long is treated as a hang: the kernel records the
-// timeout and returns. Real waits in these kernels last microseconds.
+// timeout and returns. Real waits in these kernels last microseconds. Expiry needs BOTH the global
+// nanosecond timer and this SM's cycle counter to have run past their limits (2 s, and 2e9 cycles:
+// 1 s at the maximum SM clock), so that a discontinuity of either counter cannot end a live wait.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr long long kWaitLimitCycles = 2000000000ll;
+
+__device__ __forceinline__ long long sm_clock() {
+  long long c;
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(c));
+  return c;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -69,12 +78,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
+  const long long c0 = sm_clock();
   uint32_t n = 0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((++n & 31u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs && sm_clock() - c0 > kWaitLimitCycles) {
+        *abort_flag = 1;
+        atomicOr(&g_device_status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// The same bounded wait with limits given at run time (used by the timeout self-test).
+__device__ __forceinline__ bool mbar_wait_limited(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  unsigned long long limit_ns, long long limit_cycles) {
+  const unsigned long long t0 = globaltimer_ns();
+  const long long c0 = sm_clock();
+  uint32_t n = 0;
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++n & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > limit_ns && sm_clock() - c0 > limit_cycles) {
         *abort_flag = 1;
         atomicOr(&g_device_status, kStatusTimeout);
         return false;
@@ -126,12 +155,13 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
+  const long long c0 = sm_clock();
   uint32_t n = 0;
   while (true) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((++n & 31u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs && sm_clock() - c0 > kWaitLimitCycles) {
         *abort_flag = 1;
         atomicOr(&g_device_status, kStatusTimeout);
         return false;

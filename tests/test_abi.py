@@ -94,3 +94,8 @@ def test_binding_rejects_cpu_tensors():
     x = torch.zeros(4, 16, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         fn.flashnorm_linear(x, torch.zeros(16, 16, dtype=torch.bfloat16), 1e-5)
+
+
+@pytest.mark.parametrize("limit_us", [0, -5, 10_000_001])
+def test_selftest_timeout_rejects_bad_limits(lib, limit_us):
+    assert lib.flashnorm_selftest_timeout(limit_us, NULL) == fn.FN_ERR_INVALID_ARG
