@@ -75,16 +75,31 @@ __host__ __device__ constexpr int gemm_smem_bytes() {
   return 1024 /* alignment slack */ + STAGES * (kAStageBytes + MAX_BN * kBK * 2) + 4096 /* barriers etc. */;
 }
 
-// silu(z) = z * sigmoid(z), with exp and the reciprocal taken on the special-function unit:
-// sigmoid(z) = 1 / (1 + 2^(-z * log2(e))). Relative error ~1e-6; the limits are exact (z -> -inf
-// gives 2^+inf = inf and rcp(inf) = 0; z -> +inf gives rcp(1) = 1). The flush-to-zero forms are one
-// SFU instruction each; flushing only matters where 2^(-z log2 e) is subnormal (z > 87), and there
-// 1 + e is 1 either way.
-__device__ __forceinline__ float silu_f(float z) {
+// The SwiGLU output with the deferred scale r = 1/rms applied to gate and up:
+//   silu(r g) (r u) = g u r^2 sigmoid(r g) = g u / ((1 + 2^(-r log2(e) g)) / r^2).
+// With the per-row constants c = -r log2(e) and q = 1/r^2 (= mean(x^2) + eps) this is one multiply,
+// one SFU exp, one fused multiply-add, one SFU reciprocal and two multiplies per output: two issue
+// slots fewer than scaling gate and up first, in an epilogue whose speed is set by its instruction
+// count. sigmoid(t) = 1 / (1 + 2^(-t log2(e))) with both the exp and the reciprocal on the
+// special-function unit (flush-to-zero forms, one instruction each; relative error ~1e-6). Limits:
+// r g -> -inf gives 2^+inf = inf and an output of 0; r g -> +inf gives g u r^2.
+struct GluRow {
+  float c;  // -r * log2(e)
+  float q;  // 1 / r^2
+};
+
+__device__ __forceinline__ GluRow glu_row(float r) {
+  GluRow k;
+  k.c = -r * 1.4426950408889634f;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(k.q) : "f"(r * r));
+  return k;
+}
+
+__device__ __forceinline__ float swiglu_deferred(float g, float u, GluRow k) {
   float e, s;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-z * 1.4426950408889634f));
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(s) : "f"(1.0f + e));
-  return z * s;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(g * k.c));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(s) : "f"(fmaf(e, k.q, k.q)));
+  return (g * u) * s;
 }
 
 // Store 16 consecutive output values of one row (bf16 or fp32), masking whole 8-column groups.
@@ -367,12 +382,9 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
           reg_fence16(gt);
           reg_fence16(up);
           float o[16];
+          const GluRow k = glu_row(r);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float zg = __uint_as_float(gt[j]) * r;
-            const float zu = __uint_as_float(up[j]) * r;
-            o[j] = silu_f(zg) * zu;
-          }
+          for (int j = 0; j < 16; ++j) o[j] = swiglu_deferred(__uint_as_float(gt[j]), __uint_as_float(up[j]), k);
           if (row_ok) store16<OUT_F32>(p.y, p.ldy, row, col0 + c / 2, p.n_out, o);
         }
       } else {  // EPI_POSTNORM

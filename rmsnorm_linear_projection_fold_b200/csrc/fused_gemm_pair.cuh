@@ -240,6 +240,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
         sb ^= 1;
         if (sb == 0) sb_ph ^= 1u;
       }
+      const GluRow kr = glu_row(r);
       // rows of this warp's lane quarter in y, and its staging buffer
       const int qrow0 = mt * (2 * kBM) + static_cast<int>(rank) * kBM + q * 32;
       uint8_t* stage_out = sOut + (warp - kEpiFirst) * kPairStageOutBytes;
@@ -300,11 +301,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
             reg_fence16(up);
             float o[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float zg = __uint_as_float(gt[j]) * r;
-              const float zu = __uint_as_float(up[j]) * r;
-              o[j] = silu_f(zg) * zu;
-            }
+            for (int j = 0; j < 16; ++j) o[j] = swiglu_deferred(__uint_as_float(gt[j]), __uint_as_float(up[j]), kr);
             if (OUT_F32) {
 #pragma unroll
               for (int j = 0; j < 4; ++j)
