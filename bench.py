@@ -60,6 +60,7 @@ BENCH_WORKLOADS = {
     "mla_latent_m2048": ["mla_latent_m2048"],
     "gemma_qkvnorm_hd256_m2048": ["gemma_qkvnorm_hd256_m2048"],
     "gemma_qkvnorm_hd128_m2048": ["gemma_qkvnorm_hd128_m2048"],
+    "gemma_qkvnorm_rope_hd256_m2048": ["gemma_qkvnorm_rope_hd256_m2048"],
 }
 DEFAULT_WORKLOAD = "smollm2_prefill_m8192"
 
@@ -230,7 +231,10 @@ class Projection:
             self.wk = [wk0] + [wk0.clone() for _ in range(copies - 1)]
             self.xn = [torch.empty(wl.M, wl.d, dtype=torch.bfloat16, device="cuda") for _ in range(copies)]
         del W
-        self.g2 = _to_dev(b["g2"], torch) if wl.kind == "postnorm" else None
+        self.g2 = _to_dev(b["g2"], torch) if wl.kind in ("postnorm", "postnorm_rope") else None
+        if wl.kind == "postnorm_rope":  # the (cos, sin) table and the row positions are set up once
+            self.rope_cs = fn.flashnorm_rope_table(wl.M, wl.head_dim, wl.rope_base)
+            self.positions = torch.from_numpy(wl.positions()).cuda()
         self.x_host = torch.from_numpy(np.ascontiguousarray(b["x"]).view(np.int16)).view(torch.bfloat16).pin_memory()
         self.y_host = torch.empty(wl.M, wl.N, dtype=torch.bfloat16).pin_memory()
 
@@ -241,6 +245,9 @@ class Projection:
             fn.flashnorm_linear(x, self.ws[r], wl.eps, out=self.y[r])
         elif wl.kind == "glu":
             fn.flashnorm_glu(x, self.ws[r], wl.eps, out=self.y[r])
+        elif wl.kind == "postnorm_rope":
+            fn.flashnorm_linear_postnorm_rope(x, self.ws[r], self.g2, self.rope_cs, self.positions, wl.head_dim,
+                                              wl.n_rope_heads, wl.eps2, out=self.y[r])
         else:
             fn.flashnorm_linear_postnorm(x, self.ws[r], self.g2, wl.head_dim, wl.eps2, out=self.y[r])
 
@@ -432,13 +439,19 @@ def time_oracle(workload: str, budget_s: float):
     draws = [w.draw() for w in wls]
     # a bounded row sample: at most 1024 rows per projection per pass (all rows for small M)
     rows = [np.arange(min(w.M, 1024)) for w in wls]
-    O.reference_output(wls[0].kind, draws[0], wls[0].eps, eps2=wls[0].eps2, head_dim=wls[0].head_dim,
-                       rows=rows[0][:8])  # warm-up
+
+    def oracle(w, b, r):
+        if w.kind == "postnorm_rope":
+            return O.reference_postnorm_rope(b, w.eps, w.eps2, w.head_dim, w.positions(), w.n_rope_heads,
+                                             w.rope_base, rows=r)
+        return O.reference_output(w.kind, b, w.eps, eps2=w.eps2, head_dim=w.head_dim, rows=r)
+
+    oracle(wls[0], draws[0], rows[0][:8])  # warm-up
     done_units, passes = 0.0, 0
     t0 = time.perf_counter()
     while True:
         for w, b, r in zip(wls, draws, rows):
-            O.reference_output(w.kind, b, w.eps, eps2=w.eps2, head_dim=w.head_dim, rows=r)
+            oracle(w, b, r)
             if _is_decode(wls):
                 done_units += 2 * w.d * w.w_cols
             else:

@@ -76,7 +76,7 @@ class Workload:
     """One synthetic problem: shapes, epsilon and the variant it exercises."""
 
     name: str
-    kind: str  # "linear" | "glu" | "postnorm"
+    kind: str  # "linear" | "glu" | "postnorm" | "postnorm_rope"
     M: int
     d: int
     N: int  # linear: output columns; glu: F (W has 2F columns); postnorm: latent width
@@ -84,6 +84,8 @@ class Workload:
     head_dim: int = 0  # postnorm only
     eps2: float = 0.0  # postnorm only
     seed: int = BASE_SEED
+    n_rope_heads: int = 0  # postnorm_rope: heads of a row that are rotated (the q and k heads come first)
+    rope_base: float = 10000.0
 
     @property
     def w_cols(self) -> int:
@@ -96,8 +98,16 @@ class Workload:
 
     @property
     def bytes(self) -> int:
-        """Algorithmic HBM bytes: read x and W* once, write y once (bf16)."""
-        return 2 * (self.M * self.d + self.d * self.w_cols + self.M * self.N)
+        """Algorithmic HBM bytes: read x and W* once, write y once (bf16); with RoPE also each row's
+        position and its fp32 (cos, sin) table row."""
+        b = 2 * (self.M * self.d + self.d * self.w_cols + self.M * self.N)
+        if self.kind == "postnorm_rope":
+            b += 4 * self.M + 4 * self.M * self.head_dim
+        return b
+
+    def positions(self) -> np.ndarray:
+        """Positions of the rows (postnorm_rope): a prefill of M tokens, 0 .. M-1, int32."""
+        return np.arange(self.M, dtype=np.int32)
 
     def draw(self) -> dict:
         """All inputs of this workload as bf16 bit arrays."""
@@ -106,7 +116,7 @@ class Workload:
             "g": gain(self.d, self.seed),
             "w": weight(self.d, self.w_cols, self.seed),
         }
-        if self.kind == "postnorm":
+        if self.kind in ("postnorm", "postnorm_rope"):
             out["g2"] = gain(self.head_dim, self.seed, tag="g2")
         return out
 
@@ -130,6 +140,10 @@ WORKLOADS = {
                                           head_dim=256, eps2=1e-6, seed=BASE_SEED + 5),
     "gemma_qkvnorm_hd128_m2048": Workload("gemma_qkvnorm_hd128_m2048", "postnorm", 2048, 2560, 4096, 1e-6,
                                           head_dim=128, eps2=1e-6, seed=BASE_SEED + 6),
+    # The same with RoPE fused after the per-head norm on the query and key heads (8 q + 4 k heads of 256,
+    # then 4 value heads), positions 0 .. 2047 of a prefill.
+    "gemma_qkvnorm_rope_hd256_m2048": Workload("gemma_qkvnorm_rope_hd256_m2048", "postnorm_rope", 2048, 2560, 4096,
+                                               1e-6, head_dim=256, eps2=1e-6, seed=BASE_SEED + 5, n_rope_heads=12),
 }
 
 

@@ -135,6 +135,36 @@ FN_API fn_status flashnorm_linear_postnorm(const void* x, const void* Wstar, con
                                     void* stream);
 
 /*
+ * flashnorm_linear_postnorm_rope — flashnorm_linear_postnorm followed, in the same epilogue, by rotary
+ * position embedding of the normalised query/key heads. The FlashNorm Abstract lists RoPE-based
+ * attention among the cases the technique extends to, and the paper builds on RoFormer; the rotation is
+ * RoFormer's: features (2i, 2i+1) of a head of the row at position p are rotated by the angle
+ * p * base^(-2i/head_dim):
+ *     y[2i]   = v[2i] cos - v[2i+1] sin,     y[2i+1] = v[2i] sin + v[2i+1] cos,
+ *   where v is the post-norm output of that head. Only the first n_rope_heads heads of a row are rotated
+ *   (in a fused q/k/v projection: the query and key heads); the others are only normalised.
+ *   rope_cs   fp32 [max_pos][head_dim / 2][2], (cos, sin) of pair i at position p, e.g. from
+ *             flashnorm_rope_table; 16-byte aligned; caller-owned device memory.
+ *   positions int32 [M], device memory, 4-byte aligned: the position of each row. A position outside
+ *             [0, max_pos) is not read from the table: the row's rotated heads are written as NaN and
+ *             the next flashnorm_check_device_error returns FN_ERR_INVALID_ARG.
+ * Other arguments and constraints as for flashnorm_linear_postnorm; head_dim of 384 or 512 (the
+ * cluster kernel) returns FN_ERR_UNSUPPORTED; 0 <= n_rope_heads <= N / head_dim; max_pos >= 1.
+ */
+FN_API fn_status flashnorm_linear_postnorm_rope(const void* x, const void* Wstar, const void* g2, const void* rope_cs,
+                                                const void* positions, void* y, int64_t M, int64_t d, int64_t N,
+                                                int64_t head_dim, int64_t n_rope_heads, int64_t max_pos, float eps2,
+                                                int out_dtype, void* stream);
+
+/*
+ * flashnorm_rope_table — fills rope_cs (fp32 [max_pos][head_dim / 2][2], caller-owned device memory,
+ * 16-byte aligned) with cos and sin of p * base^(-2i/head_dim), computed in double precision and
+ * rounded once to fp32. head_dim even, max_pos >= 1, base > 1 (RoFormer uses 10000). Asynchronous on
+ * `stream`.
+ */
+FN_API fn_status flashnorm_rope_table(void* rope_cs, int64_t max_pos, int64_t head_dim, double base, void* stream);
+
+/*
  * The unfused baseline the pages compare against (FlashNorm Abstract: its speedups are stated against a
  * plain norm-then-project pipeline): kernel 1 writes xn = RNE_bf16(x * 1/sqrt(mean(x^2)+eps) * g), kernel 2 runs the
  * same tensor-core GEMM on xn with no scale. Kept for measuring what folding + deferral buy.

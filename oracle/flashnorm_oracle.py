@@ -24,6 +24,9 @@ function below states the plainest reading of that prose:
 * Redundant-norm removal (with a linear layer between two RMSNorms, the abstract
   drops the first norm by the scale invariance of RMS): linear -> RMSNorm
   replaces RMSNorm -> linear -> RMSNorm.
+* RoPE on the normalised query/key heads (the abstract names RoPE-based
+  attention; the paper builds on RoFormer): pairs (2i, 2i+1) of a head rotated
+  by pos * base^(-2i/head_dim), RoFormer's own pairing.
 
 Everything is computed in float64 from inputs given as bf16 bit patterns; the
 only library primitive is numpy's float64 matrix product. No blocking, fusion
@@ -189,6 +192,52 @@ def postnorm_elided_exact_eps(x, Wstar1, g2, eps1, eps2, head_dim):
 
 
 # ---------------------------------------------------------------------------
+# Rotary position embedding on the normalised heads. The abstract lists RoPE-based
+# attention among the cases the techniques extend to, and the paper builds on
+# "RoFormer: Enhanced Transformer with Rotary Position Embedding" (mlsanity page,
+# "Builds on"). The pages give no formula; the reading taken is RoFormer's own:
+# the features of a head are paired as (2i, 2i+1), i = 0 .. head_dim/2 - 1, and
+# pair i of the token at position p is rotated by the angle p * base^(-2i/head_dim).
+# In a fused q/k/v projection with per-head normalisation, the rotation applies
+# to the query and key heads (the first n_rope_heads heads of a row); the value
+# heads are only normalised.
+# ---------------------------------------------------------------------------
+
+def rope_table(max_pos: int, head_dim: int, base: float) -> np.ndarray:
+    """(cos, sin) of the rotation angles, float64 [max_pos, head_dim/2, 2]."""
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    inv_freq = np.power(float(base), -2.0 * i / head_dim)
+    ang = np.arange(max_pos, dtype=np.float64)[:, None] * inv_freq[None, :]
+    return np.stack([np.cos(ang), np.sin(ang)], axis=-1)
+
+
+def apply_rope(v, cs, positions, head_dim: int, n_rope_heads: int) -> np.ndarray:
+    """Rotate pairs (2i, 2i+1) of the first n_rope_heads heads of every row of v [M, N].
+
+    cs is a (cos, sin) table [max_pos, head_dim/2, 2] (any float type; widened to
+    float64) and positions [M] the position of each row.
+    """
+    v = np.array(v, dtype=np.float64, copy=True)
+    M, N = v.shape
+    cs = np.asarray(cs, dtype=np.float64)[np.asarray(positions, dtype=np.int64)]  # [M, hd/2, 2]
+    c, s = cs[..., 0], cs[..., 1]
+    vh = v.reshape(M, N // head_dim, head_dim)
+    for h in range(min(n_rope_heads, N // head_dim)):
+        a = vh[:, h, 0::2].copy()
+        b = vh[:, h, 1::2].copy()
+        vh[:, h, 0::2] = a * c - b * s
+        vh[:, h, 1::2] = a * s + b * c
+    return vh.reshape(M, N)
+
+
+def postnorm_rope_full(x, g1, W, g2, eps1, eps2, head_dim, positions, n_rope_heads, base):
+    """The full chain with RoPE: rotate(per-head RMSNorm(RMSNorm(x; g1) . W; g2)), exact trig."""
+    v = postnorm_full(x, g1, W, g2, eps1, eps2, head_dim)
+    table = rope_table(int(np.max(positions)) + 1, head_dim, base)
+    return apply_rope(v, table, positions, head_dim, n_rope_heads)
+
+
+# ---------------------------------------------------------------------------
 # The unfused norm-then-project pipeline the pages compare against: the norm
 # output is materialised in bf16 (one rounding), then multiplied by W.
 # ---------------------------------------------------------------------------
@@ -243,6 +292,28 @@ def exact_operand_output(kind: str, bits: dict, wstar_bits, eps: float, *, eps2:
     if kind == "postnorm":
         return postnorm_elided(x, Ws, bf16_to_f64(bits["g2"]), eps2, head_dim)
     raise ValueError(kind)
+
+
+def reference_postnorm_rope(bits: dict, eps: float, eps2: float, head_dim: int, positions, n_rope_heads: int,
+                            base: float, rows=None) -> np.ndarray:
+    """Oracle of the full RMSNorm -> linear -> per-head RMSNorm -> RoPE chain (first norm kept)."""
+    x = bf16_to_f64(bits["x"])
+    pos = np.asarray(positions)
+    if rows is not None:
+        x, pos = x[rows], pos[rows]
+    return postnorm_rope_full(x, bf16_to_f64(bits["g"]), bf16_to_f64(bits["w"]), bf16_to_f64(bits["g2"]), eps, eps2,
+                              head_dim, pos, n_rope_heads, base)
+
+
+def exact_operand_postnorm_rope(bits: dict, wstar_bits, eps2: float, head_dim: int, positions, n_rope_heads: int,
+                                table, rows=None) -> np.ndarray:
+    """The elided post-norm on the bf16 W*, rotated with the given (cos, sin) table: the fp32-output bar."""
+    x = bf16_to_f64(bits["x"])
+    pos = np.asarray(positions)
+    if rows is not None:
+        x, pos = x[rows], pos[rows]
+    u = postnorm_elided(x, bf16_to_f64(wstar_bits), bf16_to_f64(bits["g2"]), eps2, head_dim)
+    return apply_rope(u, table, pos, head_dim, n_rope_heads)
 
 
 def rel_err(y, y_ref) -> float:

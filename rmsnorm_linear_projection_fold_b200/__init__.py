@@ -28,6 +28,8 @@ __all__ = [
     "flashnorm_linear",
     "flashnorm_glu",
     "flashnorm_linear_postnorm",
+    "flashnorm_linear_postnorm_rope",
+    "flashnorm_rope_table",
     "flashnorm_rmsnorm",
     "flashnorm_linear_unfused",
     "flashnorm_glu_unfused",
@@ -60,6 +62,8 @@ _SIGNATURES = {
     "flashnorm_glu": [_P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_glu_ex": [_P, _P, _P, _I64, _I64, _I64, _F, _INT, _INT, _P],
     "flashnorm_linear_postnorm": [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _F, _INT, _P],
+    "flashnorm_linear_postnorm_rope": [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64, _F, _INT, _P],
+    "flashnorm_rope_table": [_P, _I64, _I64, ctypes.c_double, _P],
     "flashnorm_rmsnorm": [_P, _P, _P, _I64, _I64, _F, _P],
     "flashnorm_linear_unfused": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_glu_unfused": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
@@ -212,6 +216,52 @@ def flashnorm_linear_postnorm(x: torch.Tensor, Wstar: torch.Tensor, g2: torch.Te
     _check("flashnorm_linear_postnorm",
            lib.flashnorm_linear_postnorm(_ptr(x), _ptr(Wstar), _ptr(g2), _ptr(y), M, d, N, int(head_dim),
                                          float(eps2), _out_code(out_dtype), _stream_ptr(x)))
+    return y
+
+
+def flashnorm_rope_table(max_pos: int, head_dim: int, base: float = 10000.0, device=None, out=None) -> torch.Tensor:
+    """(cos, sin) of the rotary angles p * base^(-2i/head_dim), fp32 [max_pos, head_dim/2, 2], on the GPU."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+    if out is None:
+        out = torch.empty(max_pos, head_dim // 2, 2, dtype=torch.float32, device=dev)
+    else:
+        _need(out, "out", torch.float32)
+        if tuple(out.shape) != (max_pos, head_dim // 2, 2):
+            raise ValueError("out must be [max_pos, head_dim / 2, 2]")
+    lib = load_library()
+    _check("flashnorm_rope_table",
+           lib.flashnorm_rope_table(_ptr(out), int(max_pos), int(head_dim), float(base), _stream_ptr(out)))
+    return out
+
+
+def flashnorm_linear_postnorm_rope(x: torch.Tensor, Wstar: torch.Tensor, g2: torch.Tensor, rope_cs: torch.Tensor,
+                                   positions: torch.Tensor, head_dim: int, n_rope_heads: int, eps2: float,
+                                   out_dtype=torch.bfloat16, out=None) -> torch.Tensor:
+    """flashnorm_linear_postnorm, then RoPE on the first n_rope_heads heads of every row.
+
+    rope_cs: fp32 [max_pos, head_dim/2, 2] from flashnorm_rope_table; positions: int32 [M] on the GPU.
+    """
+    _need(x, "x", dim=2)
+    _need(Wstar, "Wstar", dim=2)
+    _need(g2, "g2", dim=1)
+    _need(rope_cs, "rope_cs", torch.float32, dim=3)
+    _need(positions, "positions", torch.int32, dim=1)
+    M, d = x.shape
+    N = Wstar.shape[0]
+    if Wstar.shape[1] != d:
+        raise ValueError("Wstar must be [N, d] with the d of x")
+    if g2.shape[0] != head_dim:
+        raise ValueError("g2 must have head_dim elements")
+    if positions.shape[0] != M:
+        raise ValueError("positions must have one entry per row of x")
+    if rope_cs.shape[1:] != (head_dim // 2, 2):
+        raise ValueError("rope_cs must be [max_pos, head_dim / 2, 2]")
+    y = _output(out, (M, N), out_dtype, x)
+    lib = load_library()
+    _check("flashnorm_linear_postnorm_rope",
+           lib.flashnorm_linear_postnorm_rope(_ptr(x), _ptr(Wstar), _ptr(g2), _ptr(rope_cs), _ptr(positions), _ptr(y),
+                                              M, d, N, int(head_dim), int(n_rope_heads), int(rope_cs.shape[0]),
+                                              float(eps2), _out_code(out_dtype), _stream_ptr(x)))
     return y
 
 

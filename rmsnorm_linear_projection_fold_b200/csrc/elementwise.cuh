@@ -71,6 +71,22 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // One warp per row, 8 rows per block. Pass 1 sums squares, pass 2 (L1/L2 hits) scales and stores.
+// RoPE (cos, sin) table, fp32 [max_pos][head_dim/2][2]: pair i of position p is rotated by the angle
+// p * base^(-2i/head_dim) (RoFormer's rotary embedding). The angle and its cosine and sine are taken in
+// double precision (the CUDA math library's pow and sincos), then rounded once to fp32.
+__global__ void __launch_bounds__(256) k_rope_table(float* __restrict__ cs, int max_pos, int head_dim, double base) {
+  grid_dep_wait();
+  const int half = head_dim / 2;
+  const long long n = static_cast<long long>(max_pos) * half;
+  for (long long e = blockIdx.x * 256ll + threadIdx.x; e < n; e += static_cast<long long>(gridDim.x) * 256) {
+    const int p = static_cast<int>(e / half), i = static_cast<int>(e % half);
+    const double ang = static_cast<double>(p) * pow(base, -2.0 * i / head_dim);
+    double s, c;
+    sincos(ang, &s, &c);
+    reinterpret_cast<float2*>(cs)[e] = make_float2(static_cast<float>(c), static_cast<float>(s));
+  }
+}
+
 // Failure-detection self-test: one thread waits on an mbarrier that nothing will ever arrive at. The
 // bounded wait runs out after limit_ns (and as many SM cycles), records the timeout in the device
 // status word and the kernel returns normally.

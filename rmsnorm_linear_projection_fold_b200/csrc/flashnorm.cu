@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -236,10 +237,18 @@ fn_status run_pair_path(const void* x, const void* w, void* y, int64_t M, int64_
 #undef FN_PAIR
 }
 
+// RoPE applied by the post-norm epilogue (see flashnorm_linear_postnorm_rope).
+struct RopeArgs {
+  const float* cs;
+  const int* positions;
+  int n_rope_heads;
+  int max_pos;
+};
+
 // epi: fn::EpiKind; scale: apply the deferred 1/rms (sum of squares warpgroup on).
 fn_status run_tensor_path(const void* x, const void* w, void* y, const void* g2, int64_t M, int64_t d,
                           int64_t n_rows, int64_t n_out, int64_t head_dim, float eps, int out_dtype, int epi,
-                          bool scale, cudaStream_t stream) {
+                          bool scale, cudaStream_t stream, const RopeArgs* rope = nullptr) {
   int dev = 0;
   const int sms = device_sm_count(&dev);
   if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
@@ -268,6 +277,12 @@ fn_status run_tensor_path(const void* x, const void* w, void* y, const void* g2,
   p.num_m_tiles = static_cast<int>((M + fn::kBM - 1) / fn::kBM);
   p.num_n_tiles = static_cast<int>((n_rows + bn - 1) / bn);
   p.eps = eps;
+  if (rope != nullptr) {
+    p.rope_cs = rope->cs;
+    p.positions = rope->positions;
+    p.n_rope_heads = rope->n_rope_heads;
+    p.max_pos = rope->max_pos;
+  }
   const bool f32 = out_dtype == FN_F32;
 
 #define FN_LAUNCH(MAXBN, ST, EPI, SC)                                                        \
@@ -550,6 +565,49 @@ fn_status flashnorm_linear_postnorm(const void* x, const void* Wstar, const void
                          static_cast<cudaStream_t>(stream));
 }
 
+fn_status flashnorm_linear_postnorm_rope(const void* x, const void* Wstar, const void* g2, const void* rope_cs,
+                                         const void* positions, void* y, int64_t M, int64_t d, int64_t N,
+                                         int64_t head_dim, int64_t n_rope_heads, int64_t max_pos, float eps2,
+                                         int out_dtype, void* stream) {
+  g_last_error[0] = '\0';
+  fn_status st = check_common(x, Wstar, y, M, d, eps2, out_dtype);
+  if (st != FN_OK) return st;
+  if (head_dim < 16 || head_dim % 16 != 0) return fail(FN_ERR_INVALID_ARG, "head_dim = %lld must be a positive multiple of 16", (long long)head_dim);
+  if (head_dim > 512 || (head_dim > 256 && head_dim % fn::kPnCols == 0))
+    return fail(FN_ERR_UNSUPPORTED, "RoPE is fused for heads of at most 256 (and 320) features, not %lld", (long long)head_dim);
+  if (head_dim > 256 && head_dim % 32 != 0) return fail(FN_ERR_UNSUPPORTED, "head_dim in (256, 512] must be a multiple of 32");
+  if (N < head_dim || N > kMaxDim || N % head_dim != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a multiple of head_dim", (long long)N);
+  if (n_rope_heads < 0 || n_rope_heads > N / head_dim)
+    return fail(FN_ERR_INVALID_ARG, "n_rope_heads = %lld must be in [0, N / head_dim]", (long long)n_rope_heads);
+  if (max_pos < 1 || max_pos > kMaxDim) return fail(FN_ERR_INVALID_ARG, "max_pos = %lld must be positive", (long long)max_pos);
+  if ((st = check_ptr(g2, "g2")) != FN_OK) return st;
+  if ((st = check_ptr(rope_cs, "rope_cs")) != FN_OK) return st;
+  if (M == 0) return FN_OK;
+  if (positions == nullptr) return fail(FN_ERR_INVALID_ARG, "positions is NULL");
+  if ((reinterpret_cast<uintptr_t>(positions) & 3u) != 0) return fail(FN_ERR_ALIGN, "positions is not 4-byte aligned");
+  const RopeArgs rope = {static_cast<const float*>(rope_cs), static_cast<const int*>(positions),
+                         static_cast<int>(n_rope_heads), static_cast<int>(max_pos)};
+  return run_tensor_path(x, Wstar, y, g2, M, d, N, N, head_dim, eps2, out_dtype, fn::EPI_POSTNORM, false,
+                         static_cast<cudaStream_t>(stream), &rope);
+}
+
+fn_status flashnorm_rope_table(void* rope_cs, int64_t max_pos, int64_t head_dim, double base, void* stream) {
+  g_last_error[0] = '\0';
+  if (max_pos < 1 || max_pos > kMaxDim) return fail(FN_ERR_INVALID_ARG, "max_pos = %lld must be positive", (long long)max_pos);
+  if (head_dim < 2 || head_dim % 2 != 0 || head_dim > 65536)
+    return fail(FN_ERR_INVALID_ARG, "head_dim = %lld must be even", (long long)head_dim);
+  if (!(base > 1.0) || !std::isfinite(base)) return fail(FN_ERR_INVALID_ARG, "base must be finite and > 1");
+  fn_status st;
+  if ((st = check_ptr(rope_cs, "rope_cs")) != FN_OK) return st;
+  const long long n = static_cast<long long>(max_pos) * (head_dim / 2);
+  const long long blocks = std::min<long long>((n + 255) / 256, 148LL * 16);
+  cudaError_t e = launch_kernel(fn::k_rope_table, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                                static_cast<cudaStream_t>(stream), 1, static_cast<float*>(rope_cs),
+                                static_cast<int>(max_pos), static_cast<int>(head_dim), base);
+  if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+  return FN_OK;
+}
+
 fn_status flashnorm_rmsnorm(const void* x, const void* g, void* xn, int64_t M, int64_t d, float eps, void* stream) {
   g_last_error[0] = '\0';
   if (M < 0 || M > kMaxDim) return fail(FN_ERR_INVALID_ARG, "M out of range");
@@ -663,6 +721,8 @@ fn_status flashnorm_check_device_error(void* stream) {
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
     if (h & fn::kStatusTimeout) return fail(FN_ERR_TIMEOUT, "a kernel gave up on a bounded wait");
+    if (h & fn::kStatusBadPosition)
+      return fail(FN_ERR_INVALID_ARG, "a RoPE position was outside [0, max_pos); those rows were written as NaN");
   }
   return FN_OK;
 }

@@ -56,6 +56,11 @@ struct GemmParams {
   int num_m_tiles;
   int num_n_tiles;
   float eps;              // eps of the deferred norm (LINEAR/GLU) or eps2 (POSTNORM)
+  // POSTNORM with RoPE on the first n_rope_heads heads of a row (rope_cs == nullptr: none)
+  const float* rope_cs = nullptr;  // (cos, sin) fp32 [max_pos][head_dim / 2][2]
+  const int* positions = nullptr;  // int32 [M], position of each row
+  int n_rope_heads = 0;
+  int max_pos = 0;
 };
 
 template <int MAX_BN>
@@ -390,7 +395,31 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
       } else {  // EPI_POSTNORM
         const int hd = p.head_dim;
         const int col0 = nt * bn;
+        // This row's RoPE position: >= 0 valid, -1 no RoPE, -2 outside the table (recorded in the device
+        // status word; the row's rotated heads are written as NaN rather than read out of bounds).
+        int rope_pos = -1;
+        if (p.rope_cs != nullptr && row_ok) {
+          const int ps = p.positions[row];
+          if (ps >= 0 && ps < p.max_pos) {
+            rope_pos = ps;
+          } else {
+            rope_pos = -2;
+            atomicOr(&g_device_status, kStatusBadPosition);
+          }
+        }
         for (int h0 = 0; h0 < bn; h0 += hd) {
+          // RoPE on a query/key head: rotate pairs (2i, 2i+1) by this row's (cos, sin) of pair i. The table
+          // reads run one 16-column chunk ahead of their use (the first ones during the sum of squares),
+          // so the epilogue does not wait on each of them.
+          const bool rope_head = rope_pos >= 0 && (col0 + h0) / hd < p.n_rope_heads;
+          const bool rope_bad = rope_pos == -2 && (col0 + h0) / hd < p.n_rope_heads;
+          const float4* cs_row = reinterpret_cast<const float4*>(p.rope_cs) +
+                                 (rope_head ? static_cast<size_t>(rope_pos) * (hd / 4) : 0);
+          float4 wn[4];
+          if (rope_head) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) wn[k] = __ldg(cs_row + k);
+          }
           float ss = 0.0f;
           for (int c = 0; c < hd; c += 16) {
             uint32_t v[16];
@@ -405,6 +434,15 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
           }
           const float r2 = 1.0f / sqrtf(ss / static_cast<float>(hd) + p.eps);
           for (int c = 0; c < hd; c += 16) {
+            float4 w[4];
+            if (rope_head) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) w[k] = wn[k];
+              if (c + 16 < hd) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) wn[k] = __ldg(cs_row + (c + 16) / 4 + k);
+              }
+            }
             uint32_t v[16];
             tmem_ld16(t_row + h0 + c, v);
             tmem_ld_wait();
@@ -412,6 +450,19 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
             float o[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(v[j]) * r2 * g2s[c + j];
+            if (rope_head) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {  // w[k]: (cos, sin) of pairs c/2 + 2k and c/2 + 2k + 1
+                const float a0 = o[4 * k], b0 = o[4 * k + 1], a1 = o[4 * k + 2], b1 = o[4 * k + 3];
+                o[4 * k] = a0 * w[k].x - b0 * w[k].y;
+                o[4 * k + 1] = a0 * w[k].y + b0 * w[k].x;
+                o[4 * k + 2] = a1 * w[k].z - b1 * w[k].w;
+                o[4 * k + 3] = a1 * w[k].w + b1 * w[k].z;
+              }
+            } else if (rope_bad) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) o[j] = __int_as_float(0x7FC00000);
+            }
             if (row_ok) store16<OUT_F32>(p.y, p.ldy, row, col0 + h0 + c, p.n_out, o);
           }
         }

@@ -13,6 +13,7 @@ namespace fn {
 // bounded wait runs out; the host reads and clears it in flashnorm_check_device_error.
 __device__ unsigned int g_device_status;
 constexpr unsigned int kStatusTimeout = 1u;
+constexpr unsigned int kStatusBadPosition = 2u;  // a RoPE position outside its table (row written as NaN)
 
 // A wait that has not completed after this long is treated as a hang: the kernel records the
 // timeout and returns. Real waits in these kernels last microseconds. Expiry needs BOTH the global

@@ -99,3 +99,25 @@ def test_binding_rejects_cpu_tensors():
 @pytest.mark.parametrize("limit_us", [0, -5, 10_000_001])
 def test_selftest_timeout_rejects_bad_limits(lib, limit_us):
     assert lib.flashnorm_selftest_timeout(limit_us, NULL) == fn.FN_ERR_INVALID_ARG
+
+
+# flashnorm_linear_postnorm_rope(x, W*, g2, rope_cs, positions, y, M, d, N, head_dim, n_rope_heads, max_pos, eps2,
+#                                out_dtype, stream): rejected on the host
+@pytest.mark.parametrize("hd,n_rope,max_pos,pos_ptr,expected", [
+    (24, 1, 16, P, fn.FN_ERR_INVALID_ARG),    # head_dim % 16 != 0
+    (512, 1, 16, P, fn.FN_ERR_UNSUPPORTED),   # wide heads run on the cluster kernel, which has no RoPE
+    (64, -1, 16, P, fn.FN_ERR_INVALID_ARG),   # n_rope_heads < 0
+    (64, 5, 16, P, fn.FN_ERR_INVALID_ARG),    # more rotated heads than heads (N = 256)
+    (64, 1, 0, P, fn.FN_ERR_INVALID_ARG),     # empty table
+    (64, 1, 16, NULL, fn.FN_ERR_INVALID_ARG),  # no positions
+    (64, 1, 16, ctypes.c_void_p((1 << 20) + 2), fn.FN_ERR_ALIGN),  # positions not 4-byte aligned
+])
+def test_postnorm_rope_validation(lib, hd, n_rope, max_pos, pos_ptr, expected):
+    st = lib.flashnorm_linear_postnorm_rope(P, P, P, P, pos_ptr, P, 4, 128, 256 if hd != 512 else 512, hd, n_rope,
+                                            max_pos, 1e-6, 0, NULL)
+    assert st == expected
+
+
+@pytest.mark.parametrize("max_pos,hd,base", [(0, 64, 1e4), (8, 7, 1e4), (8, 64, 1.0), (8, 64, float("inf"))])
+def test_rope_table_validation(lib, max_pos, hd, base):
+    assert lib.flashnorm_rope_table(P, max_pos, hd, base, NULL) == fn.FN_ERR_INVALID_ARG

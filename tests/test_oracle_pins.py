@@ -26,6 +26,7 @@ import torch
 from oracle import flashnorm_oracle as O
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_worked.json")
+GOLDEN_ROPE = os.path.join(os.path.dirname(__file__), "golden", "rope_hand_worked.json")
 
 
 def _arr(v):
@@ -222,8 +223,55 @@ def check_brute_force(O):
     return fails
 
 
+def check_rope(O):
+    """RoPE on the normalised heads: hand-worked cases, the table against scalar math.cos / math.sin,
+    and the properties a rotation by position * frequency must have."""
+    import math
+
+    fails = []
+    with open(GOLDEN_ROPE) as f:
+        data = json.load(f)
+    for k, c in enumerate(data["cases"]):
+        pos = np.asarray(c["positions"])
+        table = O.rope_table(int(pos.max()) + 1, c["head_dim"], c["base"])
+        y = O.apply_rope(_arr(c["v"]), table, pos, c["head_dim"], c["n_rope_heads"])
+        if np.max(np.abs(y - _arr(c["y"]))) > 1e-14:
+            fails.append(f"rope golden case {k}")
+    # the table, entry by entry, against the scalar definition
+    hd, base = 16, 500.0
+    t = O.rope_table(40, hd, base)
+    for p in (0, 1, 7, 39):
+        for i in range(hd // 2):
+            a = p * base ** (-2.0 * i / hd)
+            if abs(t[p, i, 0] - math.cos(a)) > 1e-15 or abs(t[p, i, 1] - math.sin(a)) > 1e-15:
+                fails.append(f"rope table p={p} i={i}")
+    rng = np.random.default_rng(12)
+    hd, H = 8, 3
+    table = O.rope_table(64, hd, 10000.0)
+    v = rng.standard_normal((5, hd * H))
+    # position 0 is the identity; heads past n_rope_heads are untouched
+    if np.max(np.abs(O.apply_rope(v, table, np.zeros(5, dtype=int), hd, H) - v)) > 0:
+        fails.append("rope position 0 not identity")
+    pos = rng.integers(0, 64, 5)
+    y = O.apply_rope(v, table, pos, hd, 2)
+    if np.max(np.abs(y[:, 2 * hd:] - v[:, 2 * hd:])) > 0:
+        fails.append("rope touched a value head")
+    # every pair keeps its length (a rotation)
+    pl = lambda a: np.hypot(a[:, 0::2], a[:, 1::2])
+    if np.max(np.abs(pl(y[:, :2 * hd]) - pl(v[:, :2 * hd]))) > 1e-12:
+        fails.append("rope changed a pair's length")
+    # relative position: <R_p q, R_p' k> depends only on p' - p
+    q, k = rng.standard_normal((1, hd)), rng.standard_normal((1, hd))
+    def dot(p, pp):
+        return float(np.sum(O.apply_rope(q, table, [p], hd, 1) * O.apply_rope(k, table, [pp], hd, 1)))
+    for p, pp, s in ((3, 10, 5), (0, 20, 11), (30, 2, 7)):
+        if abs(dot(p, pp) - dot(p + s, pp + s)) > 1e-12:
+            fails.append(f"rope relative position {p},{pp},{s}")
+    return fails
+
+
 ALL_CHECKS = [check_golden, check_torch_rmsnorm, check_torch_silu, check_torch_bf16,
-              check_closed_forms, check_invariants, check_brute_force]
+              check_closed_forms, check_invariants, check_brute_force, check_rope]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
@@ -319,6 +367,38 @@ def _mut_postnorm_whole_row(v, g2, eps2, head_dim):
     return O.rmsnorm(v, np.tile(g2, N // head_dim), eps2)
 
 
+def _mut_rope_half_pairs(v, cs, positions, head_dim, n_rope_heads):
+    v = np.array(v, dtype=np.float64, copy=True)
+    M, N = v.shape
+    cs = np.asarray(cs, dtype=np.float64)[np.asarray(positions, dtype=np.int64)]
+    c, s = cs[..., 0], cs[..., 1]
+    vh = v.reshape(M, N // head_dim, head_dim)
+    h2 = head_dim // 2
+    for h in range(min(n_rope_heads, N // head_dim)):
+        a, b = vh[:, h, :h2].copy(), vh[:, h, h2:].copy()
+        vh[:, h, :h2] = a * c - b * s
+        vh[:, h, h2:] = a * s + b * c
+    return vh.reshape(M, N)
+
+
+def _mut_rope_sin_sign(v, cs, positions, head_dim, n_rope_heads):
+    cs = np.array(cs, dtype=np.float64, copy=True)
+    cs[..., 1] = -cs[..., 1]
+    return _ORIG_APPLY_ROPE(v, cs, positions, head_dim, n_rope_heads)
+
+
+def _mut_rope_freq(max_pos, head_dim, base):
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    ang = np.arange(max_pos, dtype=np.float64)[:, None] * np.power(float(base), -i / head_dim)[None, :]
+    return np.stack([np.cos(ang), np.sin(ang)], axis=-1)
+
+
+def _mut_rope_all_heads(v, cs, positions, head_dim, n_rope_heads):
+    return _ORIG_APPLY_ROPE(v, cs, positions, head_dim, np.asarray(v).shape[1] // head_dim)
+
+
+_ORIG_APPLY_ROPE = O.apply_rope
+
 MUTANTS = {
     "mean over d-1": ("inv_rms", _mut_mean_d_minus_1),
     "eps outside sqrt": ("inv_rms", _mut_eps_outside),
@@ -332,6 +412,10 @@ MUTANTS = {
     "bf16 ties away": ("f64_to_bf16", _mut_rne_ties_away),
     "W transposed": ("norm_then_project", _mut_transpose_product),
     "post-norm over whole row": ("_per_head_rmsnorm", _mut_postnorm_whole_row),
+    "rope pairs (i, i + hd/2)": ("apply_rope", _mut_rope_half_pairs),
+    "rope rotates the wrong way": ("apply_rope", _mut_rope_sin_sign),
+    "rope frequency base^(-i/hd)": ("rope_table", _mut_rope_freq),
+    "rope on the value heads too": ("apply_rope", _mut_rope_all_heads),
 }
 
 
