@@ -61,6 +61,7 @@ BENCH_WORKLOADS = {
     "gemma_qkvnorm_hd256_m2048": ["gemma_qkvnorm_hd256_m2048"],
     "gemma_qkvnorm_hd128_m2048": ["gemma_qkvnorm_hd128_m2048"],
     "gemma_qkvnorm_rope_hd256_m2048": ["gemma_qkvnorm_rope_hd256_m2048"],
+    "layernorm_qkv_m8192": ["layernorm_qkv_m8192"],
 }
 DEFAULT_WORKLOAD = "smollm2_prefill_m8192"
 
@@ -221,7 +222,10 @@ class Projection:
         x0 = _to_dev(b["x"], torch)
         self.g = _to_dev(b["g"], torch)
         W = _to_dev(b["w"], torch)
-        ws0 = fn.flashnorm_fold_weights(W, self.g, glu=glu)
+        if wl.kind == "layernorm":  # gain folded; column sums and bias of the LayerNorm fold, shared by the copies
+            ws0, self.ln_colsum, self.ln_bias = fn.flashnorm_fold_layernorm(W, self.g, _to_dev(b["beta"], torch))
+        else:
+            ws0 = fn.flashnorm_fold_weights(W, self.g, glu=glu)
         self.x = [x0] + [x0.clone() for _ in range(copies - 1)]
         self.ws = [ws0] + [ws0.clone() for _ in range(copies - 1)]
         self.y = [torch.empty(wl.M, wl.N, dtype=torch.bfloat16, device="cuda") for _ in range(copies)]
@@ -245,6 +249,8 @@ class Projection:
             fn.flashnorm_linear(x, self.ws[r], wl.eps, out=self.y[r])
         elif wl.kind == "glu":
             fn.flashnorm_glu(x, self.ws[r], wl.eps, out=self.y[r])
+        elif wl.kind == "layernorm":
+            fn.flashnorm_layernorm_linear(x, self.ws[r], self.ln_colsum, self.ln_bias, wl.eps, out=self.y[r])
         elif wl.kind == "postnorm_rope":
             fn.flashnorm_linear_postnorm_rope(x, self.ws[r], self.g2, self.rope_cs, self.positions, wl.head_dim,
                                               wl.n_rope_heads, wl.eps2, out=self.y[r])
@@ -441,6 +447,8 @@ def time_oracle(workload: str, budget_s: float):
     rows = [np.arange(min(w.M, 1024)) for w in wls]
 
     def oracle(w, b, r):
+        if w.kind == "layernorm":
+            return O.reference_layernorm(b, w.eps, rows=r)
         if w.kind == "postnorm_rope":
             return O.reference_postnorm_rope(b, w.eps, w.eps2, w.head_dim, w.positions(), w.n_rope_heads,
                                              w.rope_base, rows=r)

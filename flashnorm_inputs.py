@@ -28,7 +28,7 @@ import numpy as np
 
 BASE_SEED = 24070957
 
-_TAGS = {"x": 1, "g": 2, "w": 3, "g2": 4, "w2": 5}
+_TAGS = {"x": 1, "g": 2, "w": 3, "g2": 4, "w2": 5, "beta": 6}
 
 
 def _rng(seed: int, tag: str) -> np.random.Generator:
@@ -57,6 +57,23 @@ def activations(M: int, d: int, seed: int) -> np.ndarray:
     return f32_to_bf16_bits(x)
 
 
+def activations_offset(M: int, d: int, seed: int) -> np.ndarray:
+    """x[M, d] as bf16 bits for the LayerNorm cases: per row, (N(0,1) + a mean offset drawn from U(-1, 1))
+    times a log-uniform [0.1, 10] scale, so that the mean subtraction matters."""
+    rng = _rng(seed, "x")
+    row_scale = np.exp(rng.uniform(np.log(0.1), np.log(10.0), size=(M, 1))).astype(np.float32)
+    offset = rng.uniform(-1.0, 1.0, size=(M, 1)).astype(np.float32)
+    x = rng.standard_normal(size=(M, d), dtype=np.float32)
+    x = (x + offset) * row_scale
+    return f32_to_bf16_bits(x)
+
+
+def bias(d: int, seed: int) -> np.ndarray:
+    """beta[d] as bf16 bits: U(-0.5, 0.5)."""
+    rng = _rng(seed, "beta")
+    return f32_to_bf16_bits(rng.uniform(-0.5, 0.5, size=d).astype(np.float32))
+
+
 def gain(d: int, seed: int, tag: str = "g") -> np.ndarray:
     """g[d] as bf16 bits: U(0.5, 1.5)."""
     rng = _rng(seed, tag)
@@ -76,7 +93,7 @@ class Workload:
     """One synthetic problem: shapes, epsilon and the variant it exercises."""
 
     name: str
-    kind: str  # "linear" | "glu" | "postnorm" | "postnorm_rope"
+    kind: str  # "linear" | "glu" | "postnorm" | "postnorm_rope" | "layernorm"
     M: int
     d: int
     N: int  # linear: output columns; glu: F (W has 2F columns); postnorm: latent width
@@ -112,10 +129,12 @@ class Workload:
     def draw(self) -> dict:
         """All inputs of this workload as bf16 bit arrays."""
         out = {
-            "x": activations(self.M, self.d, self.seed),
+            "x": (activations_offset if self.kind == "layernorm" else activations)(self.M, self.d, self.seed),
             "g": gain(self.d, self.seed),
             "w": weight(self.d, self.w_cols, self.seed),
         }
+        if self.kind == "layernorm":
+            out["beta"] = bias(self.d, self.seed)
         if self.kind in ("postnorm", "postnorm_rope"):
             out["g2"] = gain(self.head_dim, self.seed, tag="g2")
         return out
@@ -140,6 +159,8 @@ WORKLOADS = {
                                           head_dim=256, eps2=1e-6, seed=BASE_SEED + 5),
     "gemma_qkvnorm_hd128_m2048": Workload("gemma_qkvnorm_hd128_m2048", "postnorm", 2048, 2560, 4096, 1e-6,
                                           head_dim=128, eps2=1e-6, seed=BASE_SEED + 6),
+    # LayerNorm (gain and bias) before the SmolLM2-sized QKV projection, 8192 tokens
+    "layernorm_qkv_m8192": Workload("layernorm_qkv_m8192", "layernorm", 8192, 576, 960, 1e-5, seed=BASE_SEED + 7),
     # The same with RoPE fused after the per-head norm on the query and key heads (8 q + 4 k heads of 256,
     # then 4 value heads), positions 0 .. 2047 of a prefill.
     "gemma_qkvnorm_rope_hd256_m2048": Workload("gemma_qkvnorm_rope_hd256_m2048", "postnorm_rope", 2048, 2560, 4096,

@@ -157,6 +157,28 @@ FN_API fn_status flashnorm_linear_postnorm_rope(const void* x, const void* Wstar
                                                 int out_dtype, void* stream);
 
 /*
+ * LayerNorm -> linear (FlashNorm Abstract: the same techniques extend to LayerNorm). With
+ *   LN(x) = (x - mu) / sqrt(var + eps) * gamma + beta,  mu = mean(x), var = mean((x - mu)^2) over the d features,
+ * y = LN(x) . W is computed as y = r (x . W*) - (r mu) colsum + bias with r = 1/sqrt(var + eps):
+ * gamma is folded into W* = diag(gamma) W as for RMSNorm, the mean subtraction becomes a rank-1 correction
+ * with the column sums of W*, and beta becomes a bias vector. mu and var are summed by the same warps
+ * that sum x^2 for RMSNorm, from the same staged x tiles, concurrently with the contraction; the correction
+ * and the bias are applied in the epilogue.
+ *
+ * flashnorm_fold_layernorm: W bf16 [d, N] row-major, gamma bf16 [d], beta bf16 [d] or NULL (no bias) ->
+ *   Wstar bf16 [N, d] (exactly flashnorm_fold_weights(W, gamma, glu = 0)), colsum fp32 [N] = sum over k of the
+ *   bf16 W*[n][k], bias fp32 [N] = sum over k of beta[k] W[k][n] (fp32). All caller-owned device memory.
+ * flashnorm_layernorm_linear: x bf16 [M, d] -> y [M, N] of out_dtype, on the CTA-pair tensor-core kernel
+ *   for every M. Constraints: d % 8 == 0, N % 8 == 0, eps >= 0. The variance is taken as
+ *   E[x^2] - mu^2 in fp32 (clamped at 0), accurate while |mu| is not large against the spread of x.
+ */
+FN_API fn_status flashnorm_fold_layernorm(const void* W, const void* gamma, const void* beta, void* Wstar,
+                                          void* colsum, void* bias, int64_t d, int64_t N, void* stream);
+FN_API fn_status flashnorm_layernorm_linear(const void* x, const void* Wstar, const void* colsum, const void* bias,
+                                            void* y, int64_t M, int64_t d, int64_t N, float eps, int out_dtype,
+                                            void* stream);
+
+/*
  * flashnorm_rope_table — fills rope_cs (fp32 [max_pos][head_dim / 2][2], caller-owned device memory,
  * 16-byte aligned) with cos and sin of p * base^(-2i/head_dim), computed in double precision and
  * rounded once to fp32. head_dim even, max_pos >= 1, base > 1 (RoFormer uses 10000). Asynchronous on

@@ -24,6 +24,9 @@ function below states the plainest reading of that prose:
 * Redundant-norm removal (with a linear layer between two RMSNorms, the abstract
   drops the first norm by the scale invariance of RMS): linear -> RMSNorm
   replaces RMSNorm -> linear -> RMSNorm.
+* LayerNorm (the abstract says the techniques extend to it): gamma folded,
+  1/sqrt(var + eps) deferred, the mean removed by a rank-1 term with the column
+  sums of W*, beta turned into a bias vector.
 * RoPE on the normalised query/key heads (the abstract names RoPE-based
   attention; the paper builds on RoFormer): pairs (2i, 2i+1) of a head rotated
   by pos * base^(-2i/head_dim), RoFormer's own pairing.
@@ -192,6 +195,49 @@ def postnorm_elided_exact_eps(x, Wstar1, g2, eps1, eps2, head_dim):
 
 
 # ---------------------------------------------------------------------------
+# LayerNorm -> linear. The abstract says the same techniques extend to
+# LayerNorm; the pages give no formula. Reading: the standard LayerNorm over the
+# d features of a row, biased variance, eps inside the root, gain gamma and bias
+# beta:  LN(x) = (x - mu) / sqrt(var + eps) * gamma + beta,
+#        mu = mean(x), var = mean((x - mu)^2).
+# Folded and deferred the way the abstract does it for RMSNorm: gamma goes into
+# W* = diag(gamma) W, the scalar 1/sqrt(var + eps) moves behind the product, and
+# the mean subtraction, being x - mu 1, becomes a rank-1 term with the column
+# sums c = 1^T W*; beta becomes the bias b = beta^T W:
+#        LN(x) . W = r (x . W* - mu c) + b,   r = 1 / sqrt(var + eps).
+# ---------------------------------------------------------------------------
+
+def layernorm(x, gamma, beta, eps):
+    """LayerNorm over the last axis (biased variance, two passes), float64."""
+    x = np.asarray(x, dtype=np.float64)
+    mu = np.mean(x, axis=-1, keepdims=True)
+    var = np.mean((x - mu) ** 2, axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * np.asarray(gamma, dtype=np.float64) + np.asarray(beta, dtype=np.float64)
+
+
+def layernorm_then_project(x, gamma, beta, W, eps):
+    """The definition: LN(x; gamma, beta) . W."""
+    return layernorm(x, gamma, beta, eps) @ np.asarray(W, dtype=np.float64)
+
+
+def layernorm_fold(W, gamma, beta):
+    """(W* = diag(gamma) W, c = 1^T W*, b = beta^T W), float64."""
+    Ws = fold(W, gamma)
+    return Ws, np.sum(Ws, axis=0), np.asarray(beta, dtype=np.float64) @ np.asarray(W, dtype=np.float64)
+
+
+def layernorm_deferred(x, Wstar, colsum, bias, eps):
+    """The folded, deferred form: r (x . W* - mu c) + b with r = 1/sqrt(var + eps)."""
+    x = np.asarray(x, dtype=np.float64)
+    mu = np.mean(x, axis=-1)
+    var = np.mean((x - mu[:, None]) ** 2, axis=-1)
+    r = 1.0 / np.sqrt(var + eps)
+    acc = x @ np.asarray(Wstar, dtype=np.float64)
+    return r[:, None] * (acc - mu[:, None] * np.asarray(colsum, dtype=np.float64)[None, :]) + \
+        np.asarray(bias, dtype=np.float64)[None, :]
+
+
+# ---------------------------------------------------------------------------
 # Rotary position embedding on the normalised heads. The abstract lists RoPE-based
 # attention among the cases the techniques extend to, and the paper builds on
 # "RoFormer: Enhanced Transformer with Rotary Position Embedding" (mlsanity page,
@@ -314,6 +360,24 @@ def exact_operand_postnorm_rope(bits: dict, wstar_bits, eps2: float, head_dim: i
         x, pos = x[rows], pos[rows]
     u = postnorm_elided(x, bf16_to_f64(wstar_bits), bf16_to_f64(bits["g2"]), eps2, head_dim)
     return apply_rope(u, table, pos, head_dim, n_rope_heads)
+
+
+def reference_layernorm(bits: dict, eps: float, rows=None) -> np.ndarray:
+    """Oracle of LN(x; gamma = bits["g"], beta = bits["beta"]) . W from bf16 bits (the definition)."""
+    x = bf16_to_f64(bits["x"])
+    if rows is not None:
+        x = x[rows]
+    return layernorm_then_project(x, bf16_to_f64(bits["g"]), bf16_to_f64(bits["beta"]), bf16_to_f64(bits["w"]), eps)
+
+
+def exact_operand_layernorm(bits: dict, wstar_bits, eps: float, rows=None) -> np.ndarray:
+    """The folded, deferred form on the bf16 W* (colsum from its bf16 values, bias from W and beta)."""
+    x = bf16_to_f64(bits["x"])
+    if rows is not None:
+        x = x[rows]
+    Ws = bf16_to_f64(wstar_bits)
+    bias = bf16_to_f64(bits["beta"]) @ bf16_to_f64(bits["w"])
+    return layernorm_deferred(x, Ws, np.sum(Ws, axis=0), bias, eps)
 
 
 def rel_err(y, y_ref) -> float:

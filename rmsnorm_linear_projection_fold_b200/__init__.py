@@ -30,6 +30,8 @@ __all__ = [
     "flashnorm_linear_postnorm",
     "flashnorm_linear_postnorm_rope",
     "flashnorm_rope_table",
+    "flashnorm_fold_layernorm",
+    "flashnorm_layernorm_linear",
     "flashnorm_rmsnorm",
     "flashnorm_linear_unfused",
     "flashnorm_glu_unfused",
@@ -64,6 +66,8 @@ _SIGNATURES = {
     "flashnorm_linear_postnorm": [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_linear_postnorm_rope": [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_rope_table": [_P, _I64, _I64, ctypes.c_double, _P],
+    "flashnorm_fold_layernorm": [_P, _P, _P, _P, _P, _P, _I64, _I64, _P],
+    "flashnorm_layernorm_linear": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_rmsnorm": [_P, _P, _P, _I64, _I64, _F, _P],
     "flashnorm_linear_unfused": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_glu_unfused": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
@@ -216,6 +220,46 @@ def flashnorm_linear_postnorm(x: torch.Tensor, Wstar: torch.Tensor, g2: torch.Te
     _check("flashnorm_linear_postnorm",
            lib.flashnorm_linear_postnorm(_ptr(x), _ptr(Wstar), _ptr(g2), _ptr(y), M, d, N, int(head_dim),
                                          float(eps2), _out_code(out_dtype), _stream_ptr(x)))
+    return y
+
+
+def flashnorm_fold_layernorm(W: torch.Tensor, gamma: torch.Tensor, beta=None):
+    """LayerNorm fold: (W* [N, d] bf16, colsum [N] fp32, bias [N] fp32) from W [d, N], gamma [d], beta [d] or None."""
+    _need(W, "W", dim=2)
+    _need(gamma, "gamma", dim=1)
+    d, N = W.shape
+    if gamma.shape[0] != d:
+        raise ValueError("gamma must have d elements")
+    if beta is not None:
+        _need(beta, "beta", dim=1)
+        if beta.shape[0] != d:
+            raise ValueError("beta must have d elements")
+    Ws = torch.empty(N, d, dtype=torch.bfloat16, device=W.device)
+    colsum = torch.empty(N, dtype=torch.float32, device=W.device)
+    bias = torch.empty(N, dtype=torch.float32, device=W.device)
+    lib = load_library()
+    _check("flashnorm_fold_layernorm",
+           lib.flashnorm_fold_layernorm(_ptr(W), _ptr(gamma), _ptr(beta), _ptr(Ws), _ptr(colsum), _ptr(bias), d, N,
+                                        _stream_ptr(W)))
+    return Ws, colsum, bias
+
+
+def flashnorm_layernorm_linear(x: torch.Tensor, Wstar: torch.Tensor, colsum: torch.Tensor, bias: torch.Tensor,
+                               eps: float, out_dtype=torch.bfloat16, out=None) -> torch.Tensor:
+    """y = LayerNorm(x; gamma, beta) . W from the folded (W*, colsum, bias) of flashnorm_fold_layernorm."""
+    _need(x, "x", dim=2)
+    _need(Wstar, "Wstar", dim=2)
+    _need(colsum, "colsum", torch.float32, dim=1)
+    _need(bias, "bias", torch.float32, dim=1)
+    M, d = x.shape
+    N = Wstar.shape[0]
+    if Wstar.shape[1] != d or colsum.shape[0] != N or bias.shape[0] != N:
+        raise ValueError("Wstar [N, d], colsum [N] and bias [N] must match x [M, d]")
+    y = _output(out, (M, N), out_dtype, x)
+    lib = load_library()
+    _check("flashnorm_layernorm_linear",
+           lib.flashnorm_layernorm_linear(_ptr(x), _ptr(Wstar), _ptr(colsum), _ptr(bias), _ptr(y), M, d, N, float(eps),
+                                          _out_code(out_dtype), _stream_ptr(x)))
     return y
 
 

@@ -71,6 +71,36 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // One warp per row, 8 rows per block. Pass 1 sums squares, pass 2 (L1/L2 hits) scales and stores.
+// LayerNorm fold, part 2: colsum[n] = sum_k W*[n][k] over the bf16 values of the folded weight (the
+// operand the MMA multiplies), one warp per output column n (a contiguous K-major row of W*).
+__global__ void __launch_bounds__(256) k_ln_colsum(const uint16_t* __restrict__ Wstar, float* __restrict__ colsum,
+                                                   int d, int N) {
+  grid_dep_wait();
+  const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (n >= N) return;
+  const uint16_t* row = Wstar + static_cast<size_t>(n) * d;
+  float s = 0.0f;
+  for (int k = lane; k < d; k += 32) s += __uint_as_float(static_cast<uint32_t>(row[k]) << 16);
+  s = warp_sum(s);
+  if (lane == 0) colsum[n] = s;
+}
+
+// LayerNorm fold, part 3: bias[n] = sum_k beta[k] W[k][n] (W row-major [d, N]; beta == nullptr gives 0),
+// one thread per column, fp32 products of the exact bf16 values.
+__global__ void __launch_bounds__(256) k_ln_bias(const uint16_t* __restrict__ W, const uint16_t* __restrict__ beta,
+                                                 float* __restrict__ bias, int d, int N) {
+  grid_dep_wait();
+  const int n = blockIdx.x * 256 + threadIdx.x;
+  if (n >= N) return;
+  float s = 0.0f;
+  if (beta != nullptr)
+    for (int k = 0; k < d; ++k)
+      s = fmaf(__uint_as_float(static_cast<uint32_t>(beta[k]) << 16),
+               __uint_as_float(static_cast<uint32_t>(W[static_cast<size_t>(k) * N + n]) << 16), s);
+  bias[n] = s;
+}
+
 // RoPE (cos, sin) table, fp32 [max_pos][head_dim/2][2]: pair i of position p is rotated by the angle
 // p * base^(-2i/head_dim) (RoFormer's rotary embedding). The angle and its cosine and sine are taken in
 // double precision (the CUDA math library's pow and sincos), then rounded once to fp32.

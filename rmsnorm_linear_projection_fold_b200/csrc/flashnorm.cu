@@ -203,7 +203,8 @@ fn_status launch_gemm_pair_t(const CUtensorMap& tx, const CUtensorMap& tw, const
 }
 
 fn_status run_pair_path(const void* x, const void* w, void* y, int64_t M, int64_t d, int64_t n_rows, int64_t n_out,
-                        float eps, int out_dtype, int epi, bool scale, cudaStream_t stream) {
+                        float eps, int out_dtype, int epi, bool scale, cudaStream_t stream,
+                        const float* ln_colsum = nullptr, const float* ln_bias = nullptr) {
   int dev = 0;
   const int sms = device_sm_count(&dev);
   if (sms <= 1) return fail(FN_ERR_CUDA, "cannot query the current device");
@@ -228,11 +229,14 @@ fn_status run_pair_path(const void* x, const void* w, void* y, int64_t M, int64_
   p.num_m_tiles = static_cast<int>((M + 2 * fn::kBM - 1) / (2 * fn::kBM));
   p.num_n_tiles = static_cast<int>((n_rows + bn - 1) / bn);
   p.eps = eps;
+  p.ln_colsum = ln_colsum;
+  p.ln_bias = ln_bias;
   const bool f32 = out_dtype == FN_F32;
 #define FN_PAIR(EPI, SC)                                                                                        \
   (f32 ? launch_gemm_pair_t<fn::kPairStages, EPI, SC, true>(tx, tw, p, sms, dev, stream)                       \
        : launch_gemm_pair_t<fn::kPairStages, EPI, SC, false>(tx, tw, p, sms, dev, stream))
   if (epi == fn::EPI_LINEAR) return scale ? FN_PAIR(fn::EPI_LINEAR, true) : FN_PAIR(fn::EPI_LINEAR, false);
+  if (epi == fn::EPI_LN) return FN_PAIR(fn::EPI_LN, true);
   return scale ? FN_PAIR(fn::EPI_GLU, true) : FN_PAIR(fn::EPI_GLU, false);
 #undef FN_PAIR
 }
@@ -589,6 +593,41 @@ fn_status flashnorm_linear_postnorm_rope(const void* x, const void* Wstar, const
                          static_cast<int>(n_rope_heads), static_cast<int>(max_pos)};
   return run_tensor_path(x, Wstar, y, g2, M, d, N, N, head_dim, eps2, out_dtype, fn::EPI_POSTNORM, false,
                          static_cast<cudaStream_t>(stream), &rope);
+}
+
+fn_status flashnorm_fold_layernorm(const void* W, const void* gamma, const void* beta, void* Wstar, void* colsum,
+                                   void* bias, int64_t d, int64_t N, void* stream) {
+  g_last_error[0] = '\0';
+  fn_status st;
+  // everything is validated before the first launch
+  if ((st = check_ptr(colsum, "colsum")) != FN_OK) return st;
+  if ((st = check_ptr(bias, "bias")) != FN_OK) return st;
+  if (beta != nullptr && (st = check_ptr(beta, "beta")) != FN_OK) return st;
+  st = flashnorm_fold_weights(W, gamma, Wstar, d, N, 0, stream);  // validates W, gamma, Wstar, d, N, then folds
+  if (st != FN_OK) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_kernel(fn::k_ln_colsum, dim3(static_cast<unsigned>((N + 7) / 8)), dim3(256), 0, s, 1,
+                                static_cast<const uint16_t*>(Wstar), static_cast<float*>(colsum), static_cast<int>(d),
+                                static_cast<int>(N));
+  if (e == cudaSuccess)
+    e = launch_kernel(fn::k_ln_bias, dim3(static_cast<unsigned>((N + 255) / 256)), dim3(256), 0, s, 1,
+                      static_cast<const uint16_t*>(W), static_cast<const uint16_t*>(beta), static_cast<float*>(bias),
+                      static_cast<int>(d), static_cast<int>(N));
+  if (e != cudaSuccess) return cuda_fail(e, "LayerNorm fold launch");
+  return FN_OK;
+}
+
+fn_status flashnorm_layernorm_linear(const void* x, const void* Wstar, const void* colsum, const void* bias, void* y,
+                                     int64_t M, int64_t d, int64_t N, float eps, int out_dtype, void* stream) {
+  g_last_error[0] = '\0';
+  fn_status st = check_common(x, Wstar, y, M, d, eps, out_dtype);
+  if (st != FN_OK) return st;
+  if (N < 8 || N > kMaxDim || N % 8 != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a positive multiple of 8", (long long)N);
+  if ((st = check_ptr(colsum, "colsum")) != FN_OK) return st;
+  if ((st = check_ptr(bias, "bias")) != FN_OK) return st;
+  if (M == 0) return FN_OK;
+  return run_pair_path(x, Wstar, y, M, d, N, N, eps, out_dtype, fn::EPI_LN, true, static_cast<cudaStream_t>(stream),
+                       static_cast<const float*>(colsum), static_cast<const float*>(bias));
 }
 
 fn_status flashnorm_rope_table(void* rope_cs, int64_t max_pos, int64_t head_dim, double base, void* stream) {

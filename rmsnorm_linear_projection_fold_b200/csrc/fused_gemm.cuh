@@ -42,7 +42,8 @@ constexpr int kAStageBytes = kBM * kBK * 2;  // 16 KB
 constexpr int kMmaK = 16;                    // k of one kind::f16 MMA
 constexpr uint32_t kTmemCols = 512;          // whole tensor memory of the SM (one CTA per SM)
 
-enum EpiKind { EPI_LINEAR = 0, EPI_GLU = 1, EPI_POSTNORM = 2 };
+// EPI_LN: LayerNorm -> linear (CTA-pair kernel only): y = r (x . W*) - (r mu) colsum(W*) + beta^T W.
+enum EpiKind { EPI_LINEAR = 0, EPI_GLU = 1, EPI_POSTNORM = 2, EPI_LN = 3 };
 
 struct GemmParams {
   void* y;                // output [M, ldy] (bf16 or fp32)
@@ -61,6 +62,9 @@ struct GemmParams {
   const int* positions = nullptr;  // int32 [M], position of each row
   int n_rope_heads = 0;
   int max_pos = 0;
+  // EPI_LN: fp32 [n_out] column sums of the folded W* and folded bias beta^T W
+  const float* ln_colsum = nullptr;
+  const float* ln_bias = nullptr;
 };
 
 template <int MAX_BN>

@@ -41,6 +41,8 @@ template <int STAGES, int EPI, bool SCALE, bool OUT_F32>
 __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
     k_fused_gemm_pair(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                       GemmParams p) {
+  constexpr bool LN = EPI == EPI_LN;
+  static_assert(!LN || SCALE, "the LayerNorm epilogue needs the mean and variance warps");
   constexpr int kSsWarps = SCALE ? 4 : 0;
   constexpr int kEpiWarps = gemm_epi_warps(EPI);
   constexpr int kEpiFirst = 2, kSsFirst = 2 + kEpiWarps;
@@ -62,7 +64,8 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
   uint64_t* ss_empty = ss_full + 2;                     // [2]
   uint64_t* drain = ss_empty + 2;                       // [1]
   float* rinv = reinterpret_cast<float*>(drain + 1);    // [2][128]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rinv + 2 * kBM);
+  float* kmu = rinv + 2 * kBM;                          // [2][128], LayerNorm: r * mean(x)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(kmu + 2 * kBM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x) >> 5, 0);
@@ -232,10 +235,11 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
       const int nt = t % p.num_n_tiles;
       if (!mbar_wait_cluster(&acc_full[acc], acc_ph, abort_flag)) break;
       tc_fence_after_sync();
-      float r = 1.0f;
+      float r = 1.0f, km = 0.0f;
       if (SCALE) {
         if (!mbar_wait(&ss_full[sb], sb_ph, abort_flag)) break;
         r = rinv[sb * kBM + row_in_tile];
+        if (LN) km = kmu[sb * kBM + row_in_tile];
         mbar_arrive(&ss_empty[sb]);
         sb ^= 1;
         if (sb == 0) sb_ph ^= 1u;
@@ -257,36 +261,45 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
       // The two warps of a lane quarter take alternate chunks; which one starts alternates from tile to
       // tile, so an odd chunk count does not always land on the same warp.
       for (int ch = (hh + t - t_begin) & 1; ch * CC < ocols && ocol0 + ch * CC < p.n_out; ch += 2) {
-        if (EPI == EPI_LINEAR) {
-          if (OUT_F32) {  // 16 columns -> 4 pieces
-            uint32_t v0[16];
-            tmem_ld16(t_row + ch * CC, v0);
-            tmem_ld_wait();
-            reg_fence16(v0);
+        if (EPI == EPI_LINEAR || LN) {
+          // CC accumulator columns -> CC outputs (4 pieces of 16 bytes): the deferred scale r, and for
+          // LayerNorm also the rank-1 mean correction and the folded bias, y = r acc - (r mu) colsum + bias
+          const int col = ocol0 + ch * CC;
+          float cq[CC], bq[CC];
+          if (LN) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              put16(j, make_uint4(__float_as_uint(__uint_as_float(v0[4 * j]) * r),
-                                  __float_as_uint(__uint_as_float(v0[4 * j + 1]) * r),
-                                  __float_as_uint(__uint_as_float(v0[4 * j + 2]) * r),
-                                  __float_as_uint(__uint_as_float(v0[4 * j + 3]) * r)));
-          } else {  // 32 columns -> 4 pieces
-            uint32_t v0[16], v1[16];
-            tmem_ld16(t_row + ch * CC, v0);
-            tmem_ld16(t_row + ch * CC + 16, v1);
-            tmem_ld_wait();
-            reg_fence16(v0);
-            reg_fence16(v1);
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              put16(j, make_uint4(pack_bf16x2(__uint_as_float(v0[8 * j]) * r, __uint_as_float(v0[8 * j + 1]) * r),
-                                  pack_bf16x2(__uint_as_float(v0[8 * j + 2]) * r, __uint_as_float(v0[8 * j + 3]) * r),
-                                  pack_bf16x2(__uint_as_float(v0[8 * j + 4]) * r, __uint_as_float(v0[8 * j + 5]) * r),
-                                  pack_bf16x2(__uint_as_float(v0[8 * j + 6]) * r, __uint_as_float(v0[8 * j + 7]) * r)));
-              put16(2 + j, make_uint4(pack_bf16x2(__uint_as_float(v1[8 * j]) * r, __uint_as_float(v1[8 * j + 1]) * r),
-                                      pack_bf16x2(__uint_as_float(v1[8 * j + 2]) * r, __uint_as_float(v1[8 * j + 3]) * r),
-                                      pack_bf16x2(__uint_as_float(v1[8 * j + 4]) * r, __uint_as_float(v1[8 * j + 5]) * r),
-                                      pack_bf16x2(__uint_as_float(v1[8 * j + 6]) * r, __uint_as_float(v1[8 * j + 7]) * r)));
+            for (int k = 0; k < CC / 4; ++k) {
+              float4 c4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = c4;
+              if (col + 4 * k < p.n_out) {  // n_out % 8 == 0: a group of 4 columns is wholly in or out
+                c4 = __ldg(reinterpret_cast<const float4*>(p.ln_colsum + col) + k);
+                b4 = __ldg(reinterpret_cast<const float4*>(p.ln_bias + col) + k);
+              }
+              cq[4 * k] = c4.x, cq[4 * k + 1] = c4.y, cq[4 * k + 2] = c4.z, cq[4 * k + 3] = c4.w;
+              bq[4 * k] = b4.x, bq[4 * k + 1] = b4.y, bq[4 * k + 2] = b4.z, bq[4 * k + 3] = b4.w;
             }
+          }
+          uint32_t v0[16], v1[16];
+          tmem_ld16(t_row + ch * CC, v0);
+          if constexpr (CC == 32) tmem_ld16(t_row + ch * CC + 16, v1);
+          tmem_ld_wait();
+          reg_fence16(v0);
+          if constexpr (CC == 32) reg_fence16(v1);
+          float o[CC];
+#pragma unroll
+          for (int jj = 0; jj < CC; ++jj) {
+            const float a = __uint_as_float(jj < 16 ? v0[jj & 15] : v1[jj & 15]);
+            o[jj] = LN ? fmaf(a, r, fmaf(-km, cq[jj], bq[jj])) : a * r;
+          }
+          if (OUT_F32) {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+              put16(jj, make_uint4(__float_as_uint(o[4 * jj]), __float_as_uint(o[4 * jj + 1]),
+                                   __float_as_uint(o[4 * jj + 2]), __float_as_uint(o[4 * jj + 3])));
+          } else {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+              put16(jj, make_uint4(pack_bf16x2(o[8 * jj], o[8 * jj + 1]), pack_bf16x2(o[8 * jj + 2], o[8 * jj + 3]),
+                                   pack_bf16x2(o[8 * jj + 4], o[8 * jj + 5]), pack_bf16x2(o[8 * jj + 6], o[8 * jj + 7])));
           }
         } else {
           // CC output columns = CC/16 (gate 16, up 16) pairs of accumulator columns
@@ -351,12 +364,13 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
     int sb = 0;
     uint32_t sb_ph = 0;
     int last_m = -1;
-    float r_row = 0.0f;
+    float r_row = 0.0f, km_row = 0.0f;
     bool ok = true;
     for (int t = t_begin; t < t_end && ok; ++t) {
       const int mt = t / p.num_n_tiles;
       const bool fresh = mt != last_m;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      float s0 = 0.f, s1 = 0.f;  // LayerNorm: sum of x
       for (int kb = 0; kb < num_kb; ++kb) {
         // As in the 1-CTA kernel: with this row block's 1/rms already known, release each stage use as
         // soon as its previous use has completed, without reading it (off the refill's critical path).
@@ -371,14 +385,14 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
           if (!fresh) break;
           const uint4 w = *reinterpret_cast<const uint4*>(line + (((c ^ lane) & 7) << 4));
           float f;
-          f = bf16lo_to_f32(w.x); a0 = fmaf(f, f, a0);
-          f = bf16hi_to_f32(w.x); a1 = fmaf(f, f, a1);
-          f = bf16lo_to_f32(w.y); a2 = fmaf(f, f, a2);
-          f = bf16hi_to_f32(w.y); a3 = fmaf(f, f, a3);
-          f = bf16lo_to_f32(w.z); a0 = fmaf(f, f, a0);
-          f = bf16hi_to_f32(w.z); a1 = fmaf(f, f, a1);
-          f = bf16lo_to_f32(w.w); a2 = fmaf(f, f, a2);
-          f = bf16hi_to_f32(w.w); a3 = fmaf(f, f, a3);
+          f = bf16lo_to_f32(w.x); a0 = fmaf(f, f, a0); if (LN) s0 += f;
+          f = bf16hi_to_f32(w.x); a1 = fmaf(f, f, a1); if (LN) s1 += f;
+          f = bf16lo_to_f32(w.y); a2 = fmaf(f, f, a2); if (LN) s0 += f;
+          f = bf16hi_to_f32(w.y); a3 = fmaf(f, f, a3); if (LN) s1 += f;
+          f = bf16lo_to_f32(w.z); a0 = fmaf(f, f, a0); if (LN) s0 += f;
+          f = bf16hi_to_f32(w.z); a1 = fmaf(f, f, a1); if (LN) s1 += f;
+          f = bf16lo_to_f32(w.w); a2 = fmaf(f, f, a2); if (LN) s0 += f;
+          f = bf16hi_to_f32(w.w); a3 = fmaf(f, f, a3); if (LN) s1 += f;
         }
         fence_proxy_async_smem();  // reads above before the TMA refill our arrival permits
         __syncwarp();
@@ -391,11 +405,20 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
       if (!ok) break;
       if (fresh) {
         const float ss = (a0 + a1) + (a2 + a3);
-        r_row = 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps);
+        if (LN) {
+          // LayerNorm: biased variance E[x^2] - mean^2 (clamped at 0 against rounding), eps inside the root
+          const float mu = (s0 + s1) / static_cast<float>(p.K);
+          const float var = fmaxf(ss / static_cast<float>(p.K) - mu * mu, 0.0f);
+          r_row = 1.0f / sqrtf(var + p.eps);
+          km_row = r_row * mu;
+        } else {
+          r_row = 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps);
+        }
         last_m = mt;
       }
       if (!mbar_wait(&ss_empty[sb], sb_ph ^ 1u, abort_flag)) break;
       rinv[sb * kBM + row_in_tile] = r_row;
+      if (LN) kmu[sb * kBM + row_in_tile] = km_row;
       mbar_arrive(&ss_full[sb]);
       sb ^= 1;
       if (sb == 0) sb_ph ^= 1u;

@@ -121,3 +121,12 @@ def test_postnorm_rope_validation(lib, hd, n_rope, max_pos, pos_ptr, expected):
 @pytest.mark.parametrize("max_pos,hd,base", [(0, 64, 1e4), (8, 7, 1e4), (8, 64, 1.0), (8, 64, float("inf"))])
 def test_rope_table_validation(lib, max_pos, hd, base):
     assert lib.flashnorm_rope_table(P, max_pos, hd, base, NULL) == fn.FN_ERR_INVALID_ARG
+
+
+def test_layernorm_validation(lib):
+    # d % 8, N % 8, eps < 0, misaligned colsum: all rejected on the host
+    assert lib.flashnorm_layernorm_linear(P, P, P, P, P, 4, 12, 64, 1e-5, 0, NULL) == fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_layernorm_linear(P, P, P, P, P, 4, 64, 60, 1e-5, 0, NULL) == fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_layernorm_linear(P, P, P, P, P, 4, 64, 64, -1.0, 0, NULL) == fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_layernorm_linear(P, P, P_MISALIGNED, P, P, 4, 64, 64, 1e-5, 0, NULL) == fn.FN_ERR_ALIGN
+    assert lib.flashnorm_fold_layernorm(P, P, P, P, P, NULL, 64, 64, NULL) == fn.FN_ERR_INVALID_ARG

@@ -27,6 +27,7 @@ from oracle import flashnorm_oracle as O
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_worked.json")
 GOLDEN_ROPE = os.path.join(os.path.dirname(__file__), "golden", "rope_hand_worked.json")
+GOLDEN_LN = os.path.join(os.path.dirname(__file__), "golden", "layernorm_hand_worked.json")
 
 
 def _arr(v):
@@ -270,8 +271,38 @@ def check_rope(O):
     return fails
 
 
+def check_layernorm(O):
+    """LayerNorm -> linear: hand-worked cases, torch's CPU layer_norm, the closed form of a constant row,
+    shift invariance, and folded + deferred == the definition."""
+    fails = []
+    with open(GOLDEN_LN) as f:
+        data = json.load(f)
+    for k, c in enumerate(data["cases"]):
+        y = O.layernorm_then_project(_arr(c["x"]), _arr(c["gamma"]), _arr(c["beta"]), _arr(c["W"]), c["eps"])
+        if np.max(np.abs(y - _arr(c["y"]))) > 1e-14:
+            fails.append(f"layernorm golden case {k}")
+    rng = np.random.default_rng(21)
+    for d, eps in ((7, 1e-5), (64, 0.0), (300, 0.1)):
+        x = rng.standard_normal((6, d)) * 3 + rng.uniform(-2, 2, (6, 1))
+        g, b = rng.uniform(0.5, 1.5, d), rng.uniform(-0.5, 0.5, d)
+        ref = torch.nn.functional.layer_norm(torch.from_numpy(x), (d,), torch.from_numpy(g), torch.from_numpy(b),
+                                             eps).numpy()
+        if np.max(np.abs(O.layernorm(x, g, b, eps) - ref)) > 1e-12:
+            fails.append(f"layernorm vs torch d={d}")
+        if np.max(np.abs(O.layernorm(x + 5.0, g, b, eps) - O.layernorm(x, g, b, eps))) > 1e-11:
+            fails.append(f"layernorm not shift invariant d={d}")
+        W = rng.standard_normal((d, 5))
+        Ws, cs, bb = O.layernorm_fold(W, g, b)
+        if np.max(np.abs(O.layernorm_deferred(x, Ws, cs, bb, eps) - O.layernorm_then_project(x, g, b, W, eps))) > 1e-10:
+            fails.append(f"layernorm folded != definition d={d}")
+        const = np.full((1, d), 1.75)  # dyadic: the mean is exact and x - mu is exactly 0
+        if np.max(np.abs(O.layernorm_then_project(const, g, b, W, max(eps, 1e-6)) - b @ W)) > 1e-12:
+            fails.append(f"layernorm constant row d={d}")
+    return fails
+
+
 ALL_CHECKS = [check_golden, check_torch_rmsnorm, check_torch_silu, check_torch_bf16,
-              check_closed_forms, check_invariants, check_brute_force, check_rope]
+              check_closed_forms, check_invariants, check_brute_force, check_rope, check_layernorm]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
@@ -399,6 +430,32 @@ def _mut_rope_all_heads(v, cs, positions, head_dim, n_rope_heads):
 
 _ORIG_APPLY_ROPE = O.apply_rope
 
+
+def _mut_ln_unbiased(x, gamma, beta, eps):
+    x = np.asarray(x, dtype=np.float64)
+    mu = np.mean(x, axis=-1, keepdims=True)
+    var = np.sum((x - mu) ** 2, axis=-1, keepdims=True) / max(x.shape[-1] - 1, 1)
+    return (x - mu) / np.sqrt(var + eps) * gamma + beta
+
+
+def _mut_ln_no_centering(x, gamma, beta, eps):
+    x = np.asarray(x, dtype=np.float64)
+    mu = np.mean(x, axis=-1, keepdims=True)
+    var = np.mean((x - mu) ** 2, axis=-1, keepdims=True)
+    return x / np.sqrt(var + eps) * gamma + beta
+
+
+def _mut_ln_beta_inside(x, gamma, beta, eps):
+    x = np.asarray(x, dtype=np.float64)
+    mu = np.mean(x, axis=-1, keepdims=True)
+    var = np.mean((x - mu) ** 2, axis=-1, keepdims=True)
+    return ((x - mu) / np.sqrt(var + eps) + beta) * gamma
+
+
+def _mut_ln_fold_colsum_unfolded(W, gamma, beta):
+    Ws = O.fold(W, gamma)
+    return Ws, np.sum(np.asarray(W, dtype=np.float64), axis=0), np.asarray(beta) @ np.asarray(W, dtype=np.float64)
+
 MUTANTS = {
     "mean over d-1": ("inv_rms", _mut_mean_d_minus_1),
     "eps outside sqrt": ("inv_rms", _mut_eps_outside),
@@ -416,6 +473,10 @@ MUTANTS = {
     "rope rotates the wrong way": ("apply_rope", _mut_rope_sin_sign),
     "rope frequency base^(-i/hd)": ("rope_table", _mut_rope_freq),
     "rope on the value heads too": ("apply_rope", _mut_rope_all_heads),
+    "layernorm unbiased variance": ("layernorm", _mut_ln_unbiased),
+    "layernorm without centering": ("layernorm", _mut_ln_no_centering),
+    "layernorm bias before gain": ("layernorm", _mut_ln_beta_inside),
+    "layernorm colsum of unfolded W": ("layernorm_fold", _mut_ln_fold_colsum_unfolded),
 }
 
 
