@@ -62,6 +62,8 @@ BENCH_WORKLOADS = {
     "gemma_qkvnorm_hd128_m2048": ["gemma_qkvnorm_hd128_m2048"],
     "gemma_qkvnorm_rope_hd256_m2048": ["gemma_qkvnorm_rope_hd256_m2048"],
     "layernorm_qkv_m8192": ["layernorm_qkv_m8192"],
+    "llama7b_qkv_fp8_m1": ["llama7b_qkv_fp8_m1"],
+    "llama7b_qkv_fp8_m4": ["llama7b_qkv_fp8_m4"],
 }
 DEFAULT_WORKLOAD = "smollm2_prefill_m8192"
 
@@ -121,6 +123,11 @@ def _is_decode(wls) -> bool:
     return all(w.M <= 16 for w in wls)
 
 
+def _weight_bytes(w) -> int:
+    """Bytes of the folded weight a decode step streams: bf16 W*, or FP8 codes plus fp32 channel scales."""
+    return w.d * w.w_cols + 4 * w.w_cols if w.kind == "linear_fp8" else 2 * w.d * w.w_cols
+
+
 def _metric(wls):
     if _is_decode(wls):
         return "fused RMSNorm+linear weight GB/s (decode)", "GB/s"
@@ -130,7 +137,7 @@ def _metric(wls):
 def _units(wls) -> float:
     """Work per step in the metric's numerator: FLOPs (prefill) or weight bytes (decode)."""
     if _is_decode(wls):
-        return float(sum(2 * w.d * w.w_cols for w in wls))
+        return float(sum(_weight_bytes(w) for w in wls))
     return float(sum(w.flops for w in wls))
 
 
@@ -209,7 +216,7 @@ def _to_dev(bits, torch):
 
 def _set_bytes(wl) -> int:
     """HBM bytes of one copy of a projection's buffers (x, W*, y)."""
-    return 2 * (wl.M * wl.d + wl.w_cols * wl.d + wl.M * wl.N)
+    return 2 * (wl.M * wl.d + wl.M * wl.N) + _weight_bytes(wl)
 
 
 class Projection:
@@ -224,6 +231,9 @@ class Projection:
         W = _to_dev(b["w"], torch)
         if wl.kind == "layernorm":  # gain folded; column sums and bias of the LayerNorm fold, shared by the copies
             ws0, self.ln_colsum, self.ln_bias = fn.flashnorm_fold_layernorm(W, self.g, _to_dev(b["beta"], torch))
+        elif wl.kind == "linear_fp8":  # FP8 codes; the channel scales are copied with them
+            ws0, s0 = fn.flashnorm_fold_weights_fp8(W, self.g)
+            self.fp8_scales = [s0] + [s0.clone() for _ in range(copies - 1)]
         else:
             ws0 = fn.flashnorm_fold_weights(W, self.g, glu=glu)
         self.x = [x0] + [x0.clone() for _ in range(copies - 1)]
@@ -249,6 +259,8 @@ class Projection:
             fn.flashnorm_linear(x, self.ws[r], wl.eps, out=self.y[r])
         elif wl.kind == "glu":
             fn.flashnorm_glu(x, self.ws[r], wl.eps, out=self.y[r])
+        elif wl.kind == "linear_fp8":
+            fn.flashnorm_linear_fp8(x, self.ws[r], self.fp8_scales[r], wl.eps, out=self.y[r])
         elif wl.kind == "layernorm":
             fn.flashnorm_layernorm_linear(x, self.ws[r], self.ln_colsum, self.ln_bias, wl.eps, out=self.y[r])
         elif wl.kind == "postnorm_rope":
@@ -449,6 +461,8 @@ def time_oracle(workload: str, budget_s: float):
     def oracle(w, b, r):
         if w.kind == "layernorm":
             return O.reference_layernorm(b, w.eps, rows=r)
+        if w.kind == "linear_fp8":
+            return O.exact_operand_fp8(b, w.eps, rows=r)
         if w.kind == "postnorm_rope":
             return O.reference_postnorm_rope(b, w.eps, w.eps2, w.head_dim, w.positions(), w.n_rope_heads,
                                              w.rope_base, rows=r)
@@ -461,7 +475,7 @@ def time_oracle(workload: str, budget_s: float):
         for w, b, r in zip(wls, draws, rows):
             oracle(w, b, r)
             if _is_decode(wls):
-                done_units += 2 * w.d * w.w_cols
+                done_units += _weight_bytes(w)
             else:
                 done_units += 2.0 * len(r) * w.d * w.w_cols
         passes += 1

@@ -93,7 +93,7 @@ class Workload:
     """One synthetic problem: shapes, epsilon and the variant it exercises."""
 
     name: str
-    kind: str  # "linear" | "glu" | "postnorm" | "postnorm_rope" | "layernorm"
+    kind: str  # "linear" | "glu" | "postnorm" | "postnorm_rope" | "layernorm" | "linear_fp8"
     M: int
     d: int
     N: int  # linear: output columns; glu: F (W has 2F columns); postnorm: latent width
@@ -120,6 +120,8 @@ class Workload:
         b = 2 * (self.M * self.d + self.d * self.w_cols + self.M * self.N)
         if self.kind == "postnorm_rope":
             b += 4 * self.M + 4 * self.M * self.head_dim
+        if self.kind == "linear_fp8":  # one byte per weight plus a fp32 scale per output channel
+            b = 2 * (self.M * self.d + self.M * self.N) + self.d * self.N + 4 * self.N
         return b
 
     def positions(self) -> np.ndarray:
@@ -159,6 +161,9 @@ WORKLOADS = {
                                           head_dim=256, eps2=1e-6, seed=BASE_SEED + 5),
     "gemma_qkvnorm_hd128_m2048": Workload("gemma_qkvnorm_hd128_m2048", "postnorm", 2048, 2560, 4096, 1e-6,
                                           head_dim=128, eps2=1e-6, seed=BASE_SEED + 6),
+    # Llama-7B QKV decode with the folded weight quantized to FP8 E4M3 per output channel
+    "llama7b_qkv_fp8_m1": Workload("llama7b_qkv_fp8_m1", "linear_fp8", 1, 4096, 12288, 1e-6, seed=BASE_SEED + 2),
+    "llama7b_qkv_fp8_m4": Workload("llama7b_qkv_fp8_m4", "linear_fp8", 4, 4096, 12288, 1e-6, seed=BASE_SEED + 2),
     # LayerNorm (gain and bias) before the SmolLM2-sized QKV projection, 8192 tokens
     "layernorm_qkv_m8192": Workload("layernorm_qkv_m8192", "layernorm", 8192, 576, 960, 1e-5, seed=BASE_SEED + 7),
     # The same with RoPE fused after the per-head norm on the query and key heads (8 q + 4 k heads of 256,

@@ -179,6 +179,24 @@ FN_API fn_status flashnorm_layernorm_linear(const void* x, const void* Wstar, co
                                             void* stream);
 
 /*
+ * Quantized W* (FlashNorm Abstract: folded checkpoints stay compatible with quantized models). The gain
+ * is folded first, then each output channel is quantized to FP8 E4M3 with its own scale; the deferred
+ * 1/rms and the channel scale multiply the output together:
+ *     W*[n][k] = g[k] W[k][n] (exact in fp32),   s[n] = max_k |W*[n][k]| / 448 (1 for a zero channel),
+ *     Q[n][k] = E4M3(W*[n][k] / s[n]) (fp32 division, round to nearest even, saturating),
+ *     y[m][n] = (sum_k x[m][k] Q[n][k]) * s[n] / sqrt(mean_k x[m][k]^2 + eps).
+ * flashnorm_fold_weights_fp8: W bf16 [d, N] row-major, g bf16 [d] -> Q uint8 [N, d] (K-major E4M3 codes)
+ *   and scales fp32 [N]; caller-owned device memory. d % 16 == 0, N % 8 == 0.
+ * flashnorm_linear_fp8: the decode path (M <= FN_DECODE_MAX_M): a GEMV that streams Q, one byte per
+ *   weight, half the bytes of bf16 W*, with x staged in shared memory. x bf16 [M, d]; y [M, N] of
+ *   out_dtype. Larger M returns FN_ERR_UNSUPPORTED.
+ */
+FN_API fn_status flashnorm_fold_weights_fp8(const void* W, const void* g, void* Q, void* scales, int64_t d, int64_t N,
+                                            void* stream);
+FN_API fn_status flashnorm_linear_fp8(const void* x, const void* Q, const void* scales, void* y, int64_t M, int64_t d,
+                                      int64_t N, float eps, int out_dtype, void* stream);
+
+/*
  * flashnorm_rope_table — fills rope_cs (fp32 [max_pos][head_dim / 2][2], caller-owned device memory,
  * 16-byte aligned) with cos and sin of p * base^(-2i/head_dim), computed in double precision and
  * rounded once to fp32. head_dim even, max_pos >= 1, base > 1 (RoFormer uses 10000). Asynchronous on

@@ -195,6 +195,76 @@ def postnorm_elided_exact_eps(x, Wstar1, g2, eps1, eps2, head_dim):
 
 
 # ---------------------------------------------------------------------------
+# Quantized W* (the abstract: the folded checkpoints stay compatible with
+# quantized models; survey row NEXT-4). Reading: weight-only fp8 E4M3 with one
+# scale per output channel, quantized AFTER the fold, so the gain is folded into
+# the quantized weight and the deferred 1/rms is applied with the channel scale:
+#   W*[n, k] = g[k] W[k, n] (exact: a bf16 x bf16 product fits fp32),
+#   s[n] = max_k |W*[n, k]| / 448 (fp32; 1 if the channel is all zero),
+#   Q[n, k] = E4M3_rne(W*[n, k] / s[n]) (fp32 division),
+#   y[m, n] = (sum_k x[m, k] dec(Q[n, k])) * s[n] * 1/sqrt(mean(x^2) + eps).
+# The scale and the codes are integer decisions taken in fp32, the kernel's
+# precision, so the oracle takes them in np.float32 too and the codes match bit
+# for bit. E4M3 ("fn" variant): 1 sign bit, 4 exponent bits with bias 7, 3
+# mantissa bits; normals 2^-6 .. 448, subnormals in steps of 2^-9, no infinity.
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def f64_to_e4m3(v) -> np.ndarray:
+    """Round to E4M3 with round-to-nearest, ties to even, saturating at +-448; return the codes (uint8).
+
+    Written from the format: a value in [2^e, 2^(e+1)) with e >= -6 is a multiple of 2^(e-3) (4
+    significant bits); below 2^-6 the quantum is 2^-9. np.rint rounds halfway cases to the even integer.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    a = np.minimum(np.abs(v), E4M3_MAX)
+    _, e = np.frexp(a)                       # a = f * 2^e, f in [0.5, 1): a in [2^(e-1), 2^e)
+    q = np.ldexp(1.0, np.maximum(e - 1, -6) - 3)
+    r = np.minimum(np.rint(a / q) * q, E4M3_MAX)
+    # encode r (now exactly representable)
+    _, er = np.frexp(r)
+    ex = er - 1                              # r in [2^ex, 2^(ex+1))
+    normal = r >= 2.0 ** -6
+    mant_n = np.where(normal, np.rint((np.ldexp(r, -np.where(normal, ex, 0)) - 1.0) * 8.0), 0)
+    code_n = ((np.where(normal, ex, 0) + 7) << 3) + mant_n.astype(np.int64)
+    code_s = np.rint(r / 2.0 ** -9).astype(np.int64)     # subnormals (and zero): m * 2^-9
+    code = np.where(normal, code_n, code_s).astype(np.int64)
+    code = code | np.where(np.signbit(v), 0x80, 0)  # the sign is kept, also on values that round to zero
+    return code.astype(np.uint8)
+
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Decode E4M3 codes exactly (0x7F / 0xFF, the NaN codes, never produced by f64_to_e4m3, decode as NaN)."""
+    c = np.asarray(codes, dtype=np.int64)
+    s = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.ldexp(1.0, e - 7))
+    val = np.where((c & 0x7F) == 0x7F, np.nan, val)
+    return s * val
+
+
+def fold_fp8(w_bits, g_bits):
+    """(codes uint8 [N, d], scales float32 [N]): the fold, then per-channel E4M3 quantization, in fp32."""
+    W = (np.asarray(w_bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+    g = (np.asarray(g_bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+    Ws = (g[:, None] * W).T.astype(np.float32)            # [N, d], exact products
+    amax = np.max(np.abs(Ws), axis=1)
+    scales = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    v = (Ws / scales[:, None]).astype(np.float32)          # IEEE fp32 division
+    return f64_to_e4m3(v.astype(np.float64)), scales
+
+
+def deferred_fp8(x, codes, scales, eps):
+    """y = (x . dec(Q)^T) * s * 1/sqrt(mean(x^2) + eps), in fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    Wq = e4m3_to_f64(codes) * np.asarray(scales, dtype=np.float64)[:, None]   # [N, d]
+    return (x @ Wq.T) * inv_rms(x, eps)[:, None]
+
+
+# ---------------------------------------------------------------------------
 # LayerNorm -> linear. The abstract says the same techniques extend to
 # LayerNorm; the pages give no formula. Reading: the standard LayerNorm over the
 # d features of a row, biased variance, eps inside the root, gain gamma and bias
@@ -360,6 +430,16 @@ def exact_operand_postnorm_rope(bits: dict, wstar_bits, eps2: float, head_dim: i
         x, pos = x[rows], pos[rows]
     u = postnorm_elided(x, bf16_to_f64(wstar_bits), bf16_to_f64(bits["g2"]), eps2, head_dim)
     return apply_rope(u, table, pos, head_dim, n_rope_heads)
+
+
+def exact_operand_fp8(bits: dict, eps: float, rows=None) -> np.ndarray:
+    """The quantized path on its own operands: the oracle's fold_fp8 codes and scales (the library's fold
+    matches them bit for bit), then y = (x . dec(Q)^T) * s * 1/rms in fp64."""
+    x = bf16_to_f64(bits["x"])
+    if rows is not None:
+        x = x[rows]
+    codes, scales = fold_fp8(bits["w"], bits["g"])
+    return deferred_fp8(x, codes, scales, eps)
 
 
 def reference_layernorm(bits: dict, eps: float, rows=None) -> np.ndarray:

@@ -31,6 +31,8 @@ __all__ = [
     "flashnorm_linear_postnorm_rope",
     "flashnorm_rope_table",
     "flashnorm_fold_layernorm",
+    "flashnorm_fold_weights_fp8",
+    "flashnorm_linear_fp8",
     "flashnorm_layernorm_linear",
     "flashnorm_rmsnorm",
     "flashnorm_linear_unfused",
@@ -67,6 +69,8 @@ _SIGNATURES = {
     "flashnorm_linear_postnorm_rope": [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_rope_table": [_P, _I64, _I64, ctypes.c_double, _P],
     "flashnorm_fold_layernorm": [_P, _P, _P, _P, _P, _P, _I64, _I64, _P],
+    "flashnorm_fold_weights_fp8": [_P, _P, _P, _P, _I64, _I64, _P],
+    "flashnorm_linear_fp8": [_P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_layernorm_linear": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_rmsnorm": [_P, _P, _P, _I64, _I64, _F, _P],
     "flashnorm_linear_unfused": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
@@ -220,6 +224,38 @@ def flashnorm_linear_postnorm(x: torch.Tensor, Wstar: torch.Tensor, g2: torch.Te
     _check("flashnorm_linear_postnorm",
            lib.flashnorm_linear_postnorm(_ptr(x), _ptr(Wstar), _ptr(g2), _ptr(y), M, d, N, int(head_dim),
                                          float(eps2), _out_code(out_dtype), _stream_ptr(x)))
+    return y
+
+
+def flashnorm_fold_weights_fp8(W: torch.Tensor, g: torch.Tensor):
+    """(Q uint8 [N, d] E4M3 codes, scales fp32 [N]): the gain fold, then per-channel FP8 quantization."""
+    _need(W, "W", dim=2)
+    _need(g, "g", dim=1)
+    d, N = W.shape
+    if g.shape[0] != d:
+        raise ValueError("g must have d elements")
+    Q = torch.empty(N, d, dtype=torch.uint8, device=W.device)
+    scales = torch.empty(N, dtype=torch.float32, device=W.device)
+    lib = load_library()
+    _check("flashnorm_fold_weights_fp8",
+           lib.flashnorm_fold_weights_fp8(_ptr(W), _ptr(g), _ptr(Q), _ptr(scales), d, N, _stream_ptr(W)))
+    return Q, scales
+
+
+def flashnorm_linear_fp8(x: torch.Tensor, Q: torch.Tensor, scales: torch.Tensor, eps: float,
+                         out_dtype=torch.bfloat16, out=None) -> torch.Tensor:
+    """Decode (M <= 16) with FP8 weights: y = (x . dec(Q)^T) * scales * 1/sqrt(mean(x^2) + eps)."""
+    _need(x, "x", dim=2)
+    _need(Q, "Q", torch.uint8, dim=2)
+    _need(scales, "scales", torch.float32, dim=1)
+    M, d = x.shape
+    N = Q.shape[0]
+    if Q.shape[1] != d or scales.shape[0] != N:
+        raise ValueError("Q [N, d] and scales [N] must match x [M, d]")
+    y = _output(out, (M, N), out_dtype, x)
+    lib = load_library()
+    _check("flashnorm_linear_fp8", lib.flashnorm_linear_fp8(_ptr(x), _ptr(Q), _ptr(scales), _ptr(y), M, d, N,
+                                                            float(eps), _out_code(out_dtype), _stream_ptr(x)))
     return y
 
 

@@ -16,6 +16,7 @@
 #include "decode_tc.cuh"
 #include "elementwise.cuh"
 #include "fused_gemm.cuh"
+#include "fp8.cuh"
 #include "fused_gemm_pair.cuh"
 #include "gemv.cuh"
 #include "postnorm_cluster.cuh"
@@ -413,6 +414,33 @@ fn_status run_gemv(const void* x, const void* w, void* y, int64_t M, int64_t d, 
 #undef FN_GEMV
 }
 
+// FP8 E4M3 weights (decode GEMV)
+template <int MT, int R, bool OUT_F32>
+fn_status launch_gemv_fp8_t(const void* x, const void* q, const void* scales, void* y, int64_t M, int64_t d,
+                            int64_t N, float eps, int sms, int dev, cudaStream_t stream) {
+  auto kern = fn::k_gemv_fp8<MT, R, OUT_F32>;
+  const int smem = fn::gemv_smem_bytes<MT>(static_cast<int>(d));
+  static int configured[kMaxDevices] = {0};
+  if (smem > 48 * 1024 && configured[dev] < smem) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (fp8 gemv)");
+    configured[dev] = smem;
+  }
+  const int64_t groups = (N + R - 1) / R;
+  const int64_t blocks_needed = (groups + 7) / 8;
+  int per_sm = (228 * 1024) / (smem + 1024);
+  if (per_sm > 8) per_sm = 8;
+  if (per_sm < 1) per_sm = 1;
+  int64_t grid = static_cast<int64_t>(sms) * per_sm;
+  if (blocks_needed < grid) grid = blocks_needed;
+  cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(fn::kGemvThreads),
+                                static_cast<size_t>(smem), stream, 1, static_cast<const uint16_t*>(x),
+                                static_cast<const uint8_t*>(q), static_cast<const float*>(scales), y,
+                                static_cast<int>(M), static_cast<int>(d), static_cast<int>(N), eps);
+  if (e != cudaSuccess) return cuda_fail(e, "fp8 GEMV launch");
+  return FN_OK;
+}
+
 // ------------------------------------------------------------------------------------------------
 // Tensor-core decode path
 // ------------------------------------------------------------------------------------------------
@@ -628,6 +656,60 @@ fn_status flashnorm_layernorm_linear(const void* x, const void* Wstar, const voi
   if (M == 0) return FN_OK;
   return run_pair_path(x, Wstar, y, M, d, N, N, eps, out_dtype, fn::EPI_LN, true, static_cast<cudaStream_t>(stream),
                        static_cast<const float*>(colsum), static_cast<const float*>(bias));
+}
+
+fn_status flashnorm_fold_weights_fp8(const void* W, const void* g, void* Q, void* scales, int64_t d, int64_t N,
+                                     void* stream) {
+  g_last_error[0] = '\0';
+  if (d < 16 || d > kMaxDim || d % 16 != 0) return fail(FN_ERR_INVALID_ARG, "d = %lld must be a positive multiple of 16", (long long)d);
+  if (N < 8 || N > kMaxDim || N % 8 != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a positive multiple of 8", (long long)N);
+  fn_status st;
+  if ((st = check_ptr(W, "W")) != FN_OK) return st;
+  if ((st = check_ptr(g, "g")) != FN_OK) return st;
+  if ((st = check_ptr(Q, "Q")) != FN_OK) return st;
+  if ((st = check_ptr(scales, "scales")) != FN_OK) return st;
+  dim3 grid(static_cast<unsigned>((N + fn::kFoldTile - 1) / fn::kFoldTile),
+            static_cast<unsigned>((d + fn::kFoldTile - 1) / fn::kFoldTile));
+  if (grid.y > 65535) return fail(FN_ERR_UNSUPPORTED, "d too large for the fold grid");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_kernel(fn::k_fp8_scales, dim3(static_cast<unsigned>((N + 255) / 256)), dim3(256), 0, s, 1,
+                                static_cast<const uint16_t*>(W), static_cast<const uint16_t*>(g),
+                                static_cast<float*>(scales), static_cast<int>(d), static_cast<int>(N));
+  if (e == cudaSuccess)
+    e = launch_kernel(fn::k_fold_fp8, grid, dim3(256), 0, s, 1, static_cast<const uint16_t*>(W),
+                      static_cast<const uint16_t*>(g), static_cast<const float*>(scales), static_cast<uint8_t*>(Q),
+                      static_cast<int>(d), static_cast<int>(N));
+  if (e != cudaSuccess) return cuda_fail(e, "fp8 fold launch");
+  return FN_OK;
+}
+
+fn_status flashnorm_linear_fp8(const void* x, const void* Q, const void* scales, void* y, int64_t M, int64_t d,
+                               int64_t N, float eps, int out_dtype, void* stream) {
+  g_last_error[0] = '\0';
+  fn_status st = check_common(x, Q, y, M, d, eps, out_dtype);
+  if (st != FN_OK) return st;
+  if (d % 16 != 0) return fail(FN_ERR_INVALID_ARG, "d = %lld must be a multiple of 16", (long long)d);
+  if (N < 8 || N > kMaxDim || N % 8 != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a positive multiple of 8", (long long)N);
+  if (M > FN_DECODE_MAX_M) return fail(FN_ERR_UNSUPPORTED, "the fp8 path is the decode GEMV: M <= %d", FN_DECODE_MAX_M);
+  if ((st = check_ptr(scales, "scales")) != FN_OK) return st;
+  if (M == 0) return FN_OK;
+  if (!gemv_fits(M, d)) return fail(FN_ERR_UNSUPPORTED, "x [%lld, %lld] does not fit in shared memory", (long long)M, (long long)d);
+  int dev = 0;
+  const int sms = device_sm_count(&dev);
+  if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool f32 = out_dtype == FN_F32;
+#define FN_G8(MT, R)                                                                          \
+  (f32 ? launch_gemv_fp8_t<MT, R, true>(x, Q, scales, y, M, d, N, eps, sms, dev, s)          \
+       : launch_gemv_fp8_t<MT, R, false>(x, Q, scales, y, M, d, N, eps, sms, dev, s))
+  switch (gemv_mt(M)) {
+    case 1: return FN_G8(1, 4);
+    case 2: return FN_G8(2, 4);
+    case 4: return FN_G8(4, 2);
+    case 8: return FN_G8(8, 2);
+    default: return FN_G8(16, 1);
+  }
+#undef FN_G8
 }
 
 fn_status flashnorm_rope_table(void* rope_cs, int64_t max_pos, int64_t head_dim, double base, void* stream) {

@@ -130,3 +130,10 @@ def test_layernorm_validation(lib):
     assert lib.flashnorm_layernorm_linear(P, P, P, P, P, 4, 64, 64, -1.0, 0, NULL) == fn.FN_ERR_INVALID_ARG
     assert lib.flashnorm_layernorm_linear(P, P, P_MISALIGNED, P, P, 4, 64, 64, 1e-5, 0, NULL) == fn.FN_ERR_ALIGN
     assert lib.flashnorm_fold_layernorm(P, P, P, P, P, NULL, 64, 64, NULL) == fn.FN_ERR_INVALID_ARG
+
+
+def test_fp8_validation(lib):
+    assert lib.flashnorm_fold_weights_fp8(P, P, P, P, 24, 64, NULL) == fn.FN_ERR_INVALID_ARG   # d % 16
+    assert lib.flashnorm_fold_weights_fp8(P, P, P, P, 64, 60, NULL) == fn.FN_ERR_INVALID_ARG   # N % 8
+    assert lib.flashnorm_linear_fp8(P, P, P, P, 17, 64, 64, 1e-6, 0, NULL) == fn.FN_ERR_UNSUPPORTED  # M > 16
+    assert lib.flashnorm_linear_fp8(P, P, P, P, 4, 72, 64, 1e-6, 0, NULL) == fn.FN_ERR_INVALID_ARG  # d % 16

@@ -301,8 +301,45 @@ def check_layernorm(O):
     return fails
 
 
+def check_fp8(O):
+    """E4M3 weight quantization: torch's own float8_e4m3fn conversion (encode on values within +-448,
+    decode of all 256 codes), hand-worked codes, and the properties of the per-channel fold."""
+    fails = []
+    rng = np.random.default_rng(31)
+    v = np.concatenate([rng.standard_normal(4000) * 60, rng.standard_normal(4000) * 0.02,
+                        np.arange(-600, 601) * 2.0 ** -11, [448.0, -448.0, 0.0, -0.0]])
+    v = np.clip(v, -448, 448).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    if np.any(O.f64_to_e4m3(v.astype(np.float64)) != ref):
+        fails.append("e4m3 encode vs torch")
+    codes = np.arange(256, dtype=np.uint8)
+    dec = O.e4m3_to_f64(codes)
+    tdec = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    if not np.all((dec == tdec) | (np.isnan(dec) & np.isnan(tdec))):
+        fails.append("e4m3 decode vs torch")
+    # hand-worked: 1 = 2^0 -> exponent field 7, mantissa 0; 448 = 1.75 * 2^8 -> 15, 6; 2^-9 is the smallest
+    # subnormal; 0.1 -> 1.625 * 2^-4 = 0.1015625 (3, 5); -0.3 -> -(1.25 * 2^-2) (sign, 5, 2)
+    for val, code in ((1.0, 0x38), (448.0, 0x7E), (2.0 ** -9, 0x01), (0.1, 0x1D), (-0.3, 0xAA), (0.0, 0x00)):
+        if int(O.f64_to_e4m3(np.array([val]))[0]) != code:
+            fails.append(f"e4m3 code of {val}")
+    # the fold: every channel's largest weight maps to +-448 and every weight is within half a step
+    d, N = 96, 24
+    wb = O.f64_to_bf16(rng.standard_normal((d, N)) / np.sqrt(d))
+    gb = O.f64_to_bf16(rng.uniform(0.5, 1.5, d))
+    Q, s = O.fold_fp8(wb, gb)
+    Ws = O.fold(O.bf16_to_f64(wb), O.bf16_to_f64(gb)).T  # [N, d]
+    deq = O.e4m3_to_f64(Q) / 1.0
+    if np.any(np.max(np.abs(deq), axis=1) != 448.0):
+        fails.append("fp8 fold: channel maximum not at 448")
+    err = np.abs(deq * s[:, None] - Ws)
+    step = np.maximum(np.abs(Ws) * 2.0 ** -4, 2.0 ** -10 * s[:, None])  # half a step: 2^-4 relative, 2^-10 s below 2^-6 s
+    if np.any(err > step * (1 + 1e-6)):
+        fails.append("fp8 fold: weight off by more than half a step")
+    return fails
+
+
 ALL_CHECKS = [check_golden, check_torch_rmsnorm, check_torch_silu, check_torch_bf16,
-              check_closed_forms, check_invariants, check_brute_force, check_rope, check_layernorm]
+              check_closed_forms, check_invariants, check_brute_force, check_rope, check_layernorm, check_fp8]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
@@ -431,6 +468,33 @@ def _mut_rope_all_heads(v, cs, positions, head_dim, n_rope_heads):
 _ORIG_APPLY_ROPE = O.apply_rope
 
 
+def _mut_fp8_truncate(v):
+    v = np.asarray(v, dtype=np.float64)
+    a = np.minimum(np.abs(v), 448.0)
+    _, e = np.frexp(a)
+    q = np.ldexp(1.0, np.maximum(e - 1, -6) - 3)
+    return _ORIG_F64_TO_E4M3(np.sign(v) * np.floor(a / q) * q)
+
+
+def _mut_fp8_bias8(codes):
+    c = np.asarray(codes, dtype=np.int64)
+    return _ORIG_E4M3_TO_F64(codes) * np.where(((c >> 3) & 0xF) == 0, 1.0, 0.5)
+
+
+def _mut_fp8_scale_rows(w_bits, g_bits):
+    W = O.bf16_to_f64(w_bits).astype(np.float32)
+    g = O.bf16_to_f64(g_bits).astype(np.float32)
+    Ws = (g[:, None] * W).T.astype(np.float32)
+    amax = np.max(np.abs(Ws), axis=0)  # per input feature instead of per output channel
+    s = np.float32(np.max(amax) / 448.0)
+    scales = np.full(Ws.shape[0], s, dtype=np.float32)
+    return _ORIG_F64_TO_E4M3((Ws / scales[:, None]).astype(np.float64)), scales
+
+
+_ORIG_F64_TO_E4M3 = O.f64_to_e4m3
+_ORIG_E4M3_TO_F64 = O.e4m3_to_f64
+
+
 def _mut_ln_unbiased(x, gamma, beta, eps):
     x = np.asarray(x, dtype=np.float64)
     mu = np.mean(x, axis=-1, keepdims=True)
@@ -477,6 +541,9 @@ MUTANTS = {
     "layernorm without centering": ("layernorm", _mut_ln_no_centering),
     "layernorm bias before gain": ("layernorm", _mut_ln_beta_inside),
     "layernorm colsum of unfolded W": ("layernorm_fold", _mut_ln_fold_colsum_unfolded),
+    "fp8 truncation": ("f64_to_e4m3", _mut_fp8_truncate),
+    "fp8 exponent bias 8": ("e4m3_to_f64", _mut_fp8_bias8),
+    "fp8 one scale for the whole matrix": ("fold_fp8", _mut_fp8_scale_rows),
 }
 
 
