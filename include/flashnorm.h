@@ -49,7 +49,7 @@ extern "C" {
 typedef enum {
   FN_OK = 0,
   FN_ERR_INVALID_ARG = 1, /* a size, pointer or flag is out of range */
-  FN_ERR_UNSUPPORTED = 2, /* a legal request this build has no kernel for (e.g. head_dim > 512) */
+  FN_ERR_UNSUPPORTED = 2, /* a legal request the library has no kernel for (e.g. head_dim > 512) */
   FN_ERR_ALIGN = 3,       /* a pointer or a leading dimension is not 16-byte aligned */
   FN_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (message has the CUDA error) */
   FN_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out (see flashnorm_check_device_error) */

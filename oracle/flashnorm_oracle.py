@@ -196,7 +196,7 @@ def postnorm_elided_exact_eps(x, Wstar1, g2, eps1, eps2, head_dim):
 
 # ---------------------------------------------------------------------------
 # Quantized W* (the abstract: the folded checkpoints stay compatible with
-# quantized models; survey row NEXT-4). Reading: weight-only fp8 E4M3 with one
+# quantized models). Reading: weight-only fp8 E4M3 with one
 # scale per output channel, quantized AFTER the fold, so the gain is folded into
 # the quantized weight and the deferred 1/rms is applied with the channel scale:
 #   W*[n, k] = g[k] W[k, n] (exact: a bf16 x bf16 product fits fp32),
