@@ -72,8 +72,9 @@ DEFAULT_WORKLOAD = "smollm2_prefill_m8192"
 # if the CUDA sources hash differently now, traffic is reported as null.
 NCU_TRAFFIC = {
     # workload: (bytes per launch, sha256[:16] of the csrc/*.cu* sources at capture time, profile file)
-    "smollm2_prefill_m8192": (13016832, "3bf9884b111041cf", "profiles/fused_gemm_pair_smollm2_ffn_m8192.md"),
-    "smollm2_ffn_m8192": (13016832, "3bf9884b111041cf", "profiles/fused_gemm_pair_smollm2_ffn_m8192.md"),
+    "smollm2_prefill_m8192": (13019904, "8aabada61cdaf1c6", "profiles/fused_gemm_pair_smollm2_ffn_m8192.md"),
+    "smollm2_ffn_m8192": (13019904, "8aabada61cdaf1c6", "profiles/fused_gemm_pair_smollm2_ffn_m8192.md"),
+    "llama7b_qkv_m4": (104848384, "8aabada61cdaf1c6", "profiles/decode_tc_llama7b_qkv_m4.md"),
 }
 
 L2_BYTES = 126 * 1000 * 1000
