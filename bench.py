@@ -20,7 +20,8 @@ against MEASURED_PEAKS.json, its duration taken with CUDA events around a separa
 kernel alone, back to back over the same rotation (events inside the step loop would end the overlap
 of one kernel's tail with the next kernel's prologue); `e2e` is the same metric through the same C-ABI calls with host
 buffers (pinned H2D copy of x and D2H copy of the outputs inside the timed region); `cpu_baseline`
-is the fp64 oracle timed on this host's cores on a bounded sample of the workload.
+is the fp64 oracle timed on this host's cores on a bounded sample of the workload; `graph` (one GPU) is the
+same steps captured once in a CUDA graph and replayed, the launch mode of a serving loop.
 
 --impl reference times the oracle itself (the only reference implementation there is: the pages
 ship no code) on the host cores, on the same workload, metric and unit.
@@ -352,6 +353,36 @@ def run_ours(args, rank, world, device_index):
         torch.distributed.barrier()
     ms_per_step = total_ms / args.steps
 
+    # The same steps captured once in a CUDA graph (R steps, one per input copy) and replayed: what a
+    # serving loop that replays graphs sees, with the host's per-call launch work gone. One GPU only
+    # (a capture failing on one rank would leave the others waiting in a collective).
+    graph = None
+    if world == 1:
+        try:
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                for i in range(copies):
+                    step(i)
+            torch.cuda.current_stream().wait_stream(side)
+            with torch.cuda.graph(g):
+                for i in range(copies):
+                    step(i)
+            torch.cuda.synchronize()
+            for _ in range(2):
+                g.replay()
+            torch.cuda.synchronize()
+            reps = max(1, args.steps // copies)
+            g_ms, _ = _time_back_to_back(torch, reps, lambda i: g.replay())
+            g_step = g_ms / (reps * copies)
+            graph = {"ms_per_step": g_step, "steps": reps * copies,
+                     "launch": f"one CUDA graph of {copies} steps, replayed {reps} times"}
+            fn.flashnorm_check_device_error()
+            del g
+        except Exception as e:  # reported, not fatal: the eager number above is the headline
+            graph = {"unavailable": f"{type(e).__name__}: {str(e)[:160]}"}
+
     # unfused two-kernel baseline (same workload, same timing), for what folding + deferral buy
     unfused = None
     if do_unfused:
@@ -441,6 +472,10 @@ def run_ours(args, rank, world, device_index):
     }
     if unfused is not None:
         out["unfused"] = unfused
+    if graph is not None:
+        if "ms_per_step" in graph:
+            graph["value"] = weak_scaling_value(units, world, graph["ms_per_step"], scale)
+        out["graph"] = graph
     return out
 
 
