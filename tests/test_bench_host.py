@@ -1,0 +1,56 @@
+"""Host-side pieces of bench.py that need no GPU: the units of the metric, the bytes a step moves, and the
+reference arm's bounded oracle sample."""
+
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import flashnorm_inputs as I  # noqa: E402
+
+
+def test_metric_units_prefill_and_decode():
+    pre = [I.WORKLOADS[n] for n in bench.BENCH_WORKLOADS["smollm2_prefill_m8192"]]
+    assert not bench._is_decode(pre)
+    assert bench._units(pre) == sum(w.flops for w in pre)
+    dec = [I.WORKLOADS["llama7b_qkv_m4"]]
+    assert bench._is_decode(dec) and bench._units(dec) == 2 * 4096 * 12288
+    fp8 = [I.WORKLOADS["llama7b_qkv_fp8_m4"]]
+    assert bench._units(fp8) == 4096 * 12288 + 4 * 12288  # one byte per weight plus the channel scales
+
+
+def test_step_bytes_follow_the_weight_format():
+    w16, w8 = I.WORKLOADS["llama7b_qkv_m4"], I.WORKLOADS["llama7b_qkv_fp8_m4"]
+    assert bench._set_bytes(w16) - bench._set_bytes(w8) == 4096 * 12288 - 4 * 12288
+    assert w8.bytes == 2 * (4 * 4096 + 4 * 12288) + 4096 * 12288 + 4 * 12288
+
+
+def test_reference_sample_shrinks_and_still_runs_the_oracle():
+    wl = "smollm2_qkv_m64"
+    bench._ORACLE_CACHE.pop(wl, None)
+    _, _, projs = bench._oracle_setup(wl)
+    assert len(projs[0]["rows"]) == 64
+    rate, cores, desc, el = bench.time_oracle(wl, 0.0)  # one pass
+    assert rate > 0 and cores >= 1 and "64 of 64 rows" in desc
+    bench._shrink_sample(wl, 0.25)
+    assert len(projs[0]["rows"]) == 16
+    rate2, _, desc2, _ = bench.time_oracle(wl, 0.0)
+    assert rate2 > 0 and "16 of 64 rows" in desc2
+    # the sampled rows are the oracle's own output for those rows
+    y = projs[0]["call"](projs[0]["rows"], projs[0]["chans"])
+    assert y.shape == (16, 960) and np.isfinite(y).all()
+    bench._ORACLE_CACHE.pop(wl, None)
+
+
+def test_decode_sample_shrinks_channels():
+    wl = "llama7b_qkv_fp8_m1"
+    bench._ORACLE_CACHE.pop(wl, None)
+    _, decode, projs = bench._oracle_setup(wl)
+    assert decode and projs[0]["chans"] == 1024
+    bench._shrink_sample(wl, 0.1)
+    assert projs[0]["chans"] == 96 and bench._pass_units(projs[0], True) == 96 * (4096 + 4)
+    bench._ORACLE_CACHE.pop(wl, None)
