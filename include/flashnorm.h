@@ -10,7 +10,9 @@
  *        on different warps, joined by shared-memory barriers).
  * It extends to GLU feed-forward layers (the deferred scale goes onto the gate and the up outputs
  * before SiLU) and to RMSNorm -> linear -> RMSNorm, where the first norm is dropped by the scale
- * invariance of RMS (same abstract).
+ * invariance of RMS (same abstract). The abstract also names LayerNorm, RoPE-based attention and
+ * quantized models among the cases the technique carries over to; this library covers LayerNorm ->
+ * linear, RoPE on the normalised heads of the post-norm path, and FP8 E4M3 weights for decode.
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are caller-owned DEVICE memory on the current device; the library never
@@ -25,8 +27,9 @@
  *     returns FN_ERR_INVALID_ARG / FN_ERR_ALIGN / FN_ERR_UNSUPPORTED with a message available from
  *     flashnorm_last_error(). A failed launch returns FN_ERR_CUDA.
  *   - M == 0 is a valid empty call: nothing is launched and FN_OK is returned.
- *   - Outputs must not overlap inputs. Results are deterministic (no atomics, no split reductions),
- *     so identical calls give bitwise identical outputs.
+ *   - Outputs must not overlap inputs. Results are deterministic (no atomics on results; the decode
+ *     kernel's split-K partial sums are combined in a fixed order), so identical calls give bitwise
+ *     identical outputs.
  *   - Every wait inside a kernel is bounded in time; a wait that runs out records FN_ERR_TIMEOUT in a
  *     device-side status word (read and cleared by flashnorm_check_device_error) and the kernel
  *     returns early instead of hanging.
@@ -98,7 +101,8 @@ FN_API fn_status flashnorm_fold_weights(const void* W, const void* g, void* Wsta
  *   x      bf16 [M, d]; Wstar bf16 [N, d] from flashnorm_fold_weights(glu = 0); y [M, N] of out_dtype.
  *   For M > 16 one persistent tcgen05 kernel computes x . W* into tensor memory while a separate
  *   warpgroup sums x^2 per row from the same shared-memory x tiles; the epilogue waits for both and
- *   scales each row. For M <= 16 a bandwidth-bound GEMV kernel streams W* once.
+ *   scales each row (CTA pairs sharing 2-SM MMAs for M > 128). For M <= 16 the tensor-core decode
+ *   kernel streams W* once, with W* rows on the MMA's M side and the tokens on its N side.
  * Constraints: M >= 0, d % 8 == 0, N % 8 == 0, eps >= 0 and finite.
  */
 FN_API fn_status flashnorm_linear(const void* x, const void* Wstar, void* y, int64_t M, int64_t d, int64_t N,
