@@ -250,7 +250,8 @@ FN_API fn_status flashnorm_linear_unfused_noalloc(const void* x, const void* g, 
 /*
  * flashnorm_check_device_error — synchronises `stream`, then reads and clears the device-side status
  * word of the current device. Returns FN_ERR_TIMEOUT if any kernel of this library gave up on a bounded
- * wait since the last check, FN_ERR_CUDA if the synchronisation itself failed, FN_OK otherwise.
+ * wait since the last check, FN_ERR_INVALID_ARG if a RoPE position fell outside its table (see
+ * flashnorm_linear_postnorm_rope), FN_ERR_CUDA if the synchronisation itself failed, FN_OK otherwise.
  */
 FN_API fn_status flashnorm_check_device_error(void* stream);
 
