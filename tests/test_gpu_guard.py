@@ -1,0 +1,106 @@
+"""Guard bands: every kernel family writes exactly its output and nothing past it.
+
+Each output is a contiguous slice at the start of a larger buffer whose remainder holds a sentinel
+pattern; after the call the sentinel must be intact, and the output must match the oracle. Shapes are
+ragged (M not a multiple of any tile, N not a multiple of the tile width) so that the partial tiles and
+the row and column guards in the epilogues are exercised."""
+
+import numpy as np
+import pytest
+import torch
+
+import flashnorm_inputs as I
+import rmsnorm_linear_projection_fold_b200 as fn
+from oracle import flashnorm_oracle as O
+from tests.gpu_util import to_dev, to_host_f64
+
+pytestmark = pytest.mark.gpu
+
+PAD = 4096          # elements of sentinel after the output
+SENTINEL = 0x7BAD   # a bf16 / fp32-half pattern no kernel writes by accident
+
+
+def _guarded(shape, dtype):
+    n = int(np.prod(shape))
+    flat = torch.empty(n + PAD, dtype=torch.int16 if dtype == torch.bfloat16 else torch.int32, device="cuda")
+    flat.fill_(SENTINEL if dtype == torch.bfloat16 else (SENTINEL << 16) | SENTINEL)
+    out = flat[:n].view(dtype).view(*shape)
+    return flat, out, n
+
+
+def _intact(flat, n):
+    tail = flat[n:].cpu().numpy()
+    ref = SENTINEL if flat.dtype == torch.int16 else (SENTINEL << 16) | SENTINEL
+    return bool(np.all(tail == ref))
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("kind,M,d,N,path", [
+    ("linear", 333, 576, 968, "pair"), ("linear", 333, 576, 968, "tensor"), ("linear", 7, 576, 968, "decode"),
+    ("linear", 5, 576, 968, "gemv"), ("glu", 301, 576, 272, "pair"), ("glu", 301, 576, 272, "tensor"),
+    ("glu", 9, 576, 272, "decode"),
+])
+def test_projection_writes_stay_in_bounds(kind, M, d, N, path, out_dtype):
+    bits = I.Workload("t", kind, M, d, N, 1e-5, seed=M + N).draw()
+    glu = kind == "glu"
+    ws = fn.flashnorm_fold_weights(to_dev(bits["w"]), to_dev(bits["g"]), glu=glu)
+    flat, y, n = _guarded((M, N), out_dtype)
+    f = fn.flashnorm_glu if glu else fn.flashnorm_linear
+    f(to_dev(bits["x"]), ws, 1e-5, out_dtype=out_dtype, out=y, path=path)
+    torch.cuda.synchronize()
+    assert _intact(flat, n)
+    ex = O.exact_operand_output(kind, bits, O.fold_bf16(bits["w"], bits["g"]), 1e-5)
+    tol = 1e-5 if out_dtype == torch.float32 else 5e-3
+    assert O.rel_err(to_host_f64(y), ex) <= tol
+
+
+@pytest.mark.parametrize("M,d,N,hd", [(130, 256, 640, 64), (70, 320, 512, 512), (40, 128, 640, 320)])
+def test_postnorm_writes_stay_in_bounds(M, d, N, hd):
+    bits = I.Workload("t", "postnorm", M, d, N, 1e-6, head_dim=hd, eps2=1e-6, seed=M).draw()
+    ws = fn.flashnorm_fold_weights(to_dev(bits["w"]), to_dev(bits["g"]))
+    flat, y, n = _guarded((M, N), torch.float32)
+    fn.flashnorm_linear_postnorm(to_dev(bits["x"]), ws, to_dev(bits["g2"]), hd, 1e-6, out_dtype=torch.float32, out=y)
+    torch.cuda.synchronize()
+    assert _intact(flat, n)
+    ex = O.exact_operand_output("postnorm", bits, O.fold_bf16(bits["w"], bits["g"]), 1e-6, eps2=1e-6, head_dim=hd)
+    assert O.rel_err(to_host_f64(y), ex) <= 1e-5
+
+
+def test_rope_layernorm_fp8_unfused_writes_stay_in_bounds():
+    # RoPE on the post-norm path
+    M, d, hd, H = 77, 256, 64, 3
+    wl = I.Workload("t", "postnorm_rope", M, d, H * hd, 1e-6, head_dim=hd, eps2=1e-6, seed=3, n_rope_heads=2)
+    bits = wl.draw()
+    cs = fn.flashnorm_rope_table(M, hd)
+    pos = torch.from_numpy(wl.positions()).cuda()
+    flat, y, n = _guarded((M, H * hd), torch.bfloat16)
+    fn.flashnorm_linear_postnorm_rope(to_dev(bits["x"]), fn.flashnorm_fold_weights(to_dev(bits["w"]), to_dev(bits["g"])),
+                                      to_dev(bits["g2"]), cs, pos, hd, 2, 1e-6, out=y)
+    torch.cuda.synchronize()
+    assert _intact(flat, n)
+    # LayerNorm
+    bits = I.Workload("t", "layernorm", 145, 576, 200, 1e-5, seed=4).draw()
+    Ws, csum, bias = fn.flashnorm_fold_layernorm(to_dev(bits["w"]), to_dev(bits["g"]), to_dev(bits["beta"]))
+    flat, y, n = _guarded((145, 200), torch.bfloat16)
+    fn.flashnorm_layernorm_linear(to_dev(bits["x"]), Ws, csum, bias, 1e-5, out=y)
+    torch.cuda.synchronize()
+    assert _intact(flat, n)
+    assert O.rel_err(to_host_f64(y), O.reference_layernorm(bits, 1e-5)) <= 5e-3
+    # FP8 decode
+    bits = I.Workload("t", "linear_fp8", 3, 576, 136, 1e-6, seed=5).draw()
+    Q, s = fn.flashnorm_fold_weights_fp8(to_dev(bits["w"]), to_dev(bits["g"]))
+    flat, y, n = _guarded((3, 136), torch.float32)
+    fn.flashnorm_linear_fp8(to_dev(bits["x"]), Q, s, 1e-6, out_dtype=torch.float32, out=y)
+    torch.cuda.synchronize()
+    assert _intact(flat, n)
+    assert O.rel_err(to_host_f64(y), O.exact_operand_fp8(bits, 1e-6)) <= 1e-5
+    # unfused baseline: both its intermediate and its output
+    bits = I.Workload("t", "linear", 150, 576, 520, 1e-5, seed=6).draw()
+    ones = to_dev(np.full(576, 0x3F80, dtype=np.uint16))
+    wk = fn.flashnorm_fold_weights(to_dev(bits["w"]), ones)
+    flat_xn, xn, n_xn = _guarded((150, 576), torch.bfloat16)
+    flat, y, n = _guarded((150, 520), torch.bfloat16)
+    fn.flashnorm_linear_unfused(to_dev(bits["x"]), to_dev(bits["g"]), wk, 1e-5, xn_ws=xn, out=y)
+    torch.cuda.synchronize()
+    assert _intact(flat_xn, n_xn) and _intact(flat, n)
+    fn.flashnorm_check_device_error()

@@ -268,12 +268,12 @@ def test_full_size_sampled_rows(name):
 
 
 # ------------------------------------------------------------------------------------------ join / lag / determinism
-@pytest.mark.parametrize("path,M", [("tensor", 300), ("gemv", 4)])
-def test_no_stale_output_back_to_back(path, M):
+@pytest.mark.parametrize("path,M,T", [("pair", 300, 400), ("tensor", 300, 200), ("decode", 4, 200), ("gemv", 4, 100)])
+def test_no_stale_output_back_to_back(path, M, T):
     """Many calls back to back on one stream into ONE output buffer, each followed by an async copy
     out; no host sync in between. Every copy must match its own input and not the previous one
-    (the failure the talk pages describe: outputs one step behind)."""
-    d, N, T = 576, 960, 24
+    (the failure the talk pages describe: outputs one step behind, seen only over long runs)."""
+    d, N = 576, 960
     wl = _wl("linear", M, d, N, seed=5)
     bits = wl.draw()
     ws = _fold(bits, False)
@@ -286,14 +286,15 @@ def test_no_stale_output_back_to_back(path, M):
         fn.flashnorm_linear(xs[t], ws, 1e-5, out=y, path=path)
         outs.append(y.clone())
     torch.cuda.synchronize()
+    prev = None
     for t in range(T):
         b = dict(bits, x=xs_bits[t])
         ref = O.reference_output("linear", b, 1e-5)
         got = to_host_f64(outs[t])
         check_bf16(got, ref, _exact("linear", b, 1e-5))
-        if t > 0:
-            prev = O.reference_output("linear", dict(bits, x=xs_bits[t - 1]), 1e-5)
+        if prev is not None:
             assert O.rel_err(got, prev) > 0.1
+        prev = ref
 
 
 def test_two_streams_and_determinism():
