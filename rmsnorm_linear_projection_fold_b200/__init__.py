@@ -123,6 +123,26 @@ def _check(name: str, status: int) -> None:
         raise FlashNormError(name, status, detail)
 
 
+def _same_device(lead: torch.Tensor, **others) -> None:
+    """Every tensor of a call must live on the device of `lead` (the C ABI takes bare pointers)."""
+    for name, t in others.items():
+        if t is not None and t.device != lead.device:
+            raise ValueError(f"{name} is on {t.device}, expected {lead.device}")
+
+
+def _invoke(entry: str, lead: torch.Tensor, *args, report: str | None = None) -> None:
+    """Call the library's `entry` with `lead`'s device current: the library launches on, and looks up
+    its per-device state for, the current device."""
+    lib = load_library()
+    dev = lead.device.index
+    if dev == torch.cuda.current_device():
+        status = getattr(lib, entry)(*args)
+    else:
+        with torch.cuda.device(dev):
+            status = getattr(lib, entry)(*args)
+    _check(report or entry, status)
+
+
 def _stream_ptr(t: torch.Tensor):
     return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
 
@@ -158,6 +178,7 @@ def _output(out, shape, dtype, like):
     _need(out, "out", dtype)
     if tuple(out.shape) != tuple(shape):
         raise ValueError(f"out must have shape {tuple(shape)}, got {tuple(out.shape)}")
+    _same_device(like, out=out)
     return out
 
 
@@ -168,10 +189,9 @@ def flashnorm_fold_weights(W: torch.Tensor, g: torch.Tensor, glu: bool = False, 
     d, N = W.shape
     if g.shape[0] != d:
         raise ValueError("g must have d elements")
+    _same_device(W, g=g)
     out = _output(out, (N, d), torch.bfloat16, W)
-    lib = load_library()
-    _check("flashnorm_fold_weights",
-           lib.flashnorm_fold_weights(_ptr(W), _ptr(g), _ptr(out), d, N, int(bool(glu)), _stream_ptr(W)))
+    _invoke("flashnorm_fold_weights", W, _ptr(W), _ptr(g), _ptr(out), d, N, int(bool(glu)), _stream_ptr(W))
     return out
 
 
@@ -184,10 +204,10 @@ def flashnorm_linear(x: torch.Tensor, Wstar: torch.Tensor, eps: float, out_dtype
     N = Wstar.shape[0]
     if Wstar.shape[1] != d:
         raise ValueError("Wstar must be [N, d] with the d of x")
+    _same_device(x, Wstar=Wstar)
     y = _output(out, (M, N), out_dtype, x)
-    lib = load_library()
-    _check("flashnorm_linear", lib.flashnorm_linear_ex(_ptr(x), _ptr(Wstar), _ptr(y), M, d, N, float(eps),
-                                                       _out_code(out_dtype), PATHS[path], _stream_ptr(x)))
+    _invoke("flashnorm_linear_ex", x, _ptr(x), _ptr(Wstar), _ptr(y), M, d, N, float(eps), _out_code(out_dtype),
+            PATHS[path], _stream_ptr(x), report="flashnorm_linear")
     return y
 
 
@@ -200,10 +220,10 @@ def flashnorm_glu(x: torch.Tensor, Wstar_gu: torch.Tensor, eps: float, out_dtype
     if Wstar_gu.shape[1] != d or Wstar_gu.shape[0] % 2:
         raise ValueError("Wstar_gu must be [2F, d] with the d of x")
     F = Wstar_gu.shape[0] // 2
+    _same_device(x, Wstar_gu=Wstar_gu)
     y = _output(out, (M, F), out_dtype, x)
-    lib = load_library()
-    _check("flashnorm_glu", lib.flashnorm_glu_ex(_ptr(x), _ptr(Wstar_gu), _ptr(y), M, d, F, float(eps),
-                                                 _out_code(out_dtype), PATHS[path], _stream_ptr(x)))
+    _invoke("flashnorm_glu_ex", x, _ptr(x), _ptr(Wstar_gu), _ptr(y), M, d, F, float(eps), _out_code(out_dtype),
+            PATHS[path], _stream_ptr(x), report="flashnorm_glu")
     return y
 
 
@@ -219,11 +239,10 @@ def flashnorm_linear_postnorm(x: torch.Tensor, Wstar: torch.Tensor, g2: torch.Te
         raise ValueError("Wstar must be [N, d] with the d of x")
     if g2.shape[0] != head_dim:
         raise ValueError("g2 must have head_dim elements")
+    _same_device(x, Wstar=Wstar, g2=g2)
     y = _output(out, (M, N), out_dtype, x)
-    lib = load_library()
-    _check("flashnorm_linear_postnorm",
-           lib.flashnorm_linear_postnorm(_ptr(x), _ptr(Wstar), _ptr(g2), _ptr(y), M, d, N, int(head_dim),
-                                         float(eps2), _out_code(out_dtype), _stream_ptr(x)))
+    _invoke("flashnorm_linear_postnorm", x, _ptr(x), _ptr(Wstar), _ptr(g2), _ptr(y), M, d, N, int(head_dim),
+            float(eps2), _out_code(out_dtype), _stream_ptr(x))
     return y
 
 
@@ -234,11 +253,10 @@ def flashnorm_fold_weights_fp8(W: torch.Tensor, g: torch.Tensor):
     d, N = W.shape
     if g.shape[0] != d:
         raise ValueError("g must have d elements")
+    _same_device(W, g=g)
     Q = torch.empty(N, d, dtype=torch.uint8, device=W.device)
     scales = torch.empty(N, dtype=torch.float32, device=W.device)
-    lib = load_library()
-    _check("flashnorm_fold_weights_fp8",
-           lib.flashnorm_fold_weights_fp8(_ptr(W), _ptr(g), _ptr(Q), _ptr(scales), d, N, _stream_ptr(W)))
+    _invoke("flashnorm_fold_weights_fp8", W, _ptr(W), _ptr(g), _ptr(Q), _ptr(scales), d, N, _stream_ptr(W))
     return Q, scales
 
 
@@ -252,10 +270,10 @@ def flashnorm_linear_fp8(x: torch.Tensor, Q: torch.Tensor, scales: torch.Tensor,
     N = Q.shape[0]
     if Q.shape[1] != d or scales.shape[0] != N:
         raise ValueError("Q [N, d] and scales [N] must match x [M, d]")
+    _same_device(x, Q=Q, scales=scales)
     y = _output(out, (M, N), out_dtype, x)
-    lib = load_library()
-    _check("flashnorm_linear_fp8", lib.flashnorm_linear_fp8(_ptr(x), _ptr(Q), _ptr(scales), _ptr(y), M, d, N,
-                                                            float(eps), _out_code(out_dtype), _stream_ptr(x)))
+    _invoke("flashnorm_linear_fp8", x, _ptr(x), _ptr(Q), _ptr(scales), _ptr(y), M, d, N, float(eps),
+            _out_code(out_dtype), _stream_ptr(x))
     return y
 
 
@@ -270,13 +288,12 @@ def flashnorm_fold_layernorm(W: torch.Tensor, gamma: torch.Tensor, beta=None):
         _need(beta, "beta", dim=1)
         if beta.shape[0] != d:
             raise ValueError("beta must have d elements")
+    _same_device(W, gamma=gamma, beta=beta)
     Ws = torch.empty(N, d, dtype=torch.bfloat16, device=W.device)
     colsum = torch.empty(N, dtype=torch.float32, device=W.device)
     bias = torch.empty(N, dtype=torch.float32, device=W.device)
-    lib = load_library()
-    _check("flashnorm_fold_layernorm",
-           lib.flashnorm_fold_layernorm(_ptr(W), _ptr(gamma), _ptr(beta), _ptr(Ws), _ptr(colsum), _ptr(bias), d, N,
-                                        _stream_ptr(W)))
+    _invoke("flashnorm_fold_layernorm", W, _ptr(W), _ptr(gamma), _ptr(beta), _ptr(Ws), _ptr(colsum), _ptr(bias), d,
+            N, _stream_ptr(W))
     return Ws, colsum, bias
 
 
@@ -291,11 +308,10 @@ def flashnorm_layernorm_linear(x: torch.Tensor, Wstar: torch.Tensor, colsum: tor
     N = Wstar.shape[0]
     if Wstar.shape[1] != d or colsum.shape[0] != N or bias.shape[0] != N:
         raise ValueError("Wstar [N, d], colsum [N] and bias [N] must match x [M, d]")
+    _same_device(x, Wstar=Wstar, colsum=colsum, bias=bias)
     y = _output(out, (M, N), out_dtype, x)
-    lib = load_library()
-    _check("flashnorm_layernorm_linear",
-           lib.flashnorm_layernorm_linear(_ptr(x), _ptr(Wstar), _ptr(colsum), _ptr(bias), _ptr(y), M, d, N, float(eps),
-                                          _out_code(out_dtype), _stream_ptr(x)))
+    _invoke("flashnorm_layernorm_linear", x, _ptr(x), _ptr(Wstar), _ptr(colsum), _ptr(bias), _ptr(y), M, d, N,
+            float(eps), _out_code(out_dtype), _stream_ptr(x))
     return y
 
 
@@ -308,9 +324,7 @@ def flashnorm_rope_table(max_pos: int, head_dim: int, base: float = 10000.0, dev
         _need(out, "out", torch.float32)
         if tuple(out.shape) != (max_pos, head_dim // 2, 2):
             raise ValueError("out must be [max_pos, head_dim / 2, 2]")
-    lib = load_library()
-    _check("flashnorm_rope_table",
-           lib.flashnorm_rope_table(_ptr(out), int(max_pos), int(head_dim), float(base), _stream_ptr(out)))
+    _invoke("flashnorm_rope_table", out, _ptr(out), int(max_pos), int(head_dim), float(base), _stream_ptr(out))
     return out
 
 
@@ -336,12 +350,11 @@ def flashnorm_linear_postnorm_rope(x: torch.Tensor, Wstar: torch.Tensor, g2: tor
         raise ValueError("positions must have one entry per row of x")
     if rope_cs.shape[1:] != (head_dim // 2, 2):
         raise ValueError("rope_cs must be [max_pos, head_dim / 2, 2]")
+    _same_device(x, Wstar=Wstar, g2=g2, rope_cs=rope_cs, positions=positions)
     y = _output(out, (M, N), out_dtype, x)
-    lib = load_library()
-    _check("flashnorm_linear_postnorm_rope",
-           lib.flashnorm_linear_postnorm_rope(_ptr(x), _ptr(Wstar), _ptr(g2), _ptr(rope_cs), _ptr(positions), _ptr(y),
-                                              M, d, N, int(head_dim), int(n_rope_heads), int(rope_cs.shape[0]),
-                                              float(eps2), _out_code(out_dtype), _stream_ptr(x)))
+    _invoke("flashnorm_linear_postnorm_rope", x, _ptr(x), _ptr(Wstar), _ptr(g2), _ptr(rope_cs), _ptr(positions),
+            _ptr(y), M, d, N, int(head_dim), int(n_rope_heads), int(rope_cs.shape[0]), float(eps2),
+            _out_code(out_dtype), _stream_ptr(x))
     return y
 
 
@@ -350,9 +363,9 @@ def flashnorm_rmsnorm(x: torch.Tensor, g: torch.Tensor, eps: float, out=None) ->
     _need(x, "x", dim=2)
     _need(g, "g", dim=1)
     M, d = x.shape
+    _same_device(x, g=g)
     xn = _output(out, (M, d), torch.bfloat16, x)
-    lib = load_library()
-    _check("flashnorm_rmsnorm", lib.flashnorm_rmsnorm(_ptr(x), _ptr(g), _ptr(xn), M, d, float(eps), _stream_ptr(x)))
+    _invoke("flashnorm_rmsnorm", x, _ptr(x), _ptr(g), _ptr(xn), M, d, float(eps), _stream_ptr(x))
     return xn
 
 
@@ -363,12 +376,11 @@ def flashnorm_linear_unfused(x, g, W_kmajor, eps, xn_ws=None, out_dtype=torch.bf
     _need(W_kmajor, "W_kmajor", dim=2)
     M, d = x.shape
     N = W_kmajor.shape[0]
+    _same_device(x, g=g, W_kmajor=W_kmajor)
     xn_ws = _output(xn_ws, (M, d), torch.bfloat16, x)
     y = _output(out, (M, N), out_dtype, x)
-    lib = load_library()
-    _check("flashnorm_linear_unfused",
-           lib.flashnorm_linear_unfused(_ptr(x), _ptr(g), _ptr(W_kmajor), _ptr(xn_ws), _ptr(y), M, d, N, float(eps),
-                                        _out_code(out_dtype), _stream_ptr(x)))
+    _invoke("flashnorm_linear_unfused", x, _ptr(x), _ptr(g), _ptr(W_kmajor), _ptr(xn_ws), _ptr(y), M, d, N,
+            float(eps), _out_code(out_dtype), _stream_ptr(x))
     return y
 
 
@@ -379,12 +391,11 @@ def flashnorm_glu_unfused(x, g, W_kmajor_gu, eps, xn_ws=None, out_dtype=torch.bf
     _need(W_kmajor_gu, "W_kmajor_gu", dim=2)
     M, d = x.shape
     F = W_kmajor_gu.shape[0] // 2
+    _same_device(x, g=g, W_kmajor_gu=W_kmajor_gu)
     xn_ws = _output(xn_ws, (M, d), torch.bfloat16, x)
     y = _output(out, (M, F), out_dtype, x)
-    lib = load_library()
-    _check("flashnorm_glu_unfused",
-           lib.flashnorm_glu_unfused(_ptr(x), _ptr(g), _ptr(W_kmajor_gu), _ptr(xn_ws), _ptr(y), M, d, F, float(eps),
-                                     _out_code(out_dtype), _stream_ptr(x)))
+    _invoke("flashnorm_glu_unfused", x, _ptr(x), _ptr(g), _ptr(W_kmajor_gu), _ptr(xn_ws), _ptr(y), M, d, F,
+            float(eps), _out_code(out_dtype), _stream_ptr(x))
     return y
 
 
@@ -401,11 +412,10 @@ def flashnorm_linear_unfused_noalloc(x, g, W_kmajor, eps, out_dtype=torch.bfloat
     _need(W_kmajor, "W_kmajor", dim=2)
     M, d = x.shape
     N = W_kmajor.shape[0]
+    _same_device(x, g=g, W_kmajor=W_kmajor)
     y = _output(out, (M, N), out_dtype, x)
-    lib = load_library()
-    _check("flashnorm_linear_unfused_noalloc",
-           lib.flashnorm_linear_unfused_noalloc(_ptr(x), _ptr(g), _ptr(W_kmajor), _ptr(y), M, d, N, float(eps),
-                                                _out_code(out_dtype), _stream_ptr(x)))
+    _invoke("flashnorm_linear_unfused_noalloc", x, _ptr(x), _ptr(g), _ptr(W_kmajor), _ptr(y), M, d, N, float(eps),
+            _out_code(out_dtype), _stream_ptr(x))
     return y
 
 
@@ -414,7 +424,9 @@ def flashnorm_check_device_error(device=None) -> None:
     dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
     lib = load_library()
     s = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
-    _check("flashnorm_check_device_error", lib.flashnorm_check_device_error(s))
+    with torch.cuda.device(dev):  # the status word read is the current device's
+        status = lib.flashnorm_check_device_error(s)
+    _check("flashnorm_check_device_error", status)
 
 
 def flashnorm_selftest_timeout(limit_us: int = 20000, device=None) -> int:
@@ -423,7 +435,8 @@ def flashnorm_selftest_timeout(limit_us: int = 20000, device=None) -> int:
     dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
     lib = load_library()
     s = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
-    return int(lib.flashnorm_selftest_timeout(int(limit_us), s))
+    with torch.cuda.device(dev):
+        return int(lib.flashnorm_selftest_timeout(int(limit_us), s))
 
 
 def flashnorm_version() -> int:

@@ -96,6 +96,16 @@ def test_binding_rejects_cpu_tensors():
         fn.flashnorm_linear(x, torch.zeros(16, 16, dtype=torch.bfloat16), 1e-5)
 
 
+def test_binding_rejects_mixed_devices():
+    # the C ABI takes bare pointers on one device, so the binding refuses tensors spread over several
+    import torch
+
+    a, b = torch.zeros(2), torch.zeros(2, device="meta")
+    fn._same_device(a, b=torch.zeros(3), c=None)
+    with pytest.raises(ValueError, match="b is on meta"):
+        fn._same_device(a, b=b)
+
+
 @pytest.mark.parametrize("limit_us", [0, -5, 10_000_001])
 def test_selftest_timeout_rejects_bad_limits(lib, limit_us):
     assert lib.flashnorm_selftest_timeout(limit_us, NULL) == fn.FN_ERR_INVALID_ARG
