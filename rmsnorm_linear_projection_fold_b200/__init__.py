@@ -1,8 +1,9 @@
 """FlashNorm RMSNorm -> linear on B200: a thin binding of the C ABI in include/flashnorm.h.
 
 Each function here has the name of the C entry point it calls and only marshals arguments: it
-checks that the torch tensors are CUDA bf16 / fp32 and contiguous, allocates outputs the caller did
-not pass, and hands raw pointers plus the current CUDA stream to libflashnorm.so. All arithmetic
+checks that the torch tensors are CUDA bf16 / fp32, contiguous and on one device, allocates outputs
+the caller did not pass, makes that device current, and hands raw pointers plus its current CUDA
+stream to libflashnorm.so. All arithmetic
 runs in the library's sm_100a kernels; there is no fallback of any kind. If the library is missing,
 importing works but every call raises.
 
