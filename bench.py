@@ -645,6 +645,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        ap.error(f"--gpus {args.gpus} needs {args.gpus} ranks, found WORLD_SIZE={world}: launch N > 1 with "
+                 f"python -m torch.distributed.run --nproc-per-node {args.gpus} bench.py --gpus {args.gpus}")
 
     if args.impl == "reference":
         out = run_reference(args, rank, world)

@@ -54,3 +54,13 @@ def test_decode_sample_shrinks_channels():
     bench._shrink_sample(wl, 0.1)
     assert projs[0]["chans"] == 96 and bench._pass_units(projs[0], True) == 96 * (4096 + 4)
     bench._ORACLE_CACHE.pop(wl, None)
+
+
+def test_gpu_count_must_match_the_ranks():
+    # --gpus N without N ranks would print a line for fewer GPUs than asked; bench.py refuses instead
+    import subprocess
+
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference"],
+                       capture_output=True, text=True, env=env, timeout=120)
+    assert r.returncode == 2 and "WORLD_SIZE=1" in r.stderr
