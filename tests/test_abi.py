@@ -147,3 +147,11 @@ def test_fp8_validation(lib):
     assert lib.flashnorm_fold_weights_fp8(P, P, P, P, 64, 60, NULL) == fn.FN_ERR_INVALID_ARG   # N % 8
     assert lib.flashnorm_linear_fp8(P, P, P, P, 17, 64, 64, 1e-6, 0, NULL) == fn.FN_ERR_UNSUPPORTED  # M > 16
     assert lib.flashnorm_linear_fp8(P, P, P, P, 4, 72, 64, 1e-6, 0, NULL) == fn.FN_ERR_INVALID_ARG  # d % 16
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    # no fallback: every entry point goes through load_library, which raises when the library is not built
+    monkeypatch.setattr(fn, "_LIB_PATH", str(tmp_path / "libflashnorm.so"))
+    monkeypatch.setattr(fn, "_lib", None)
+    with pytest.raises(fn.FlashNormError, match="is missing"):
+        fn.load_library()
