@@ -33,6 +33,10 @@
  *   - Every wait inside a kernel is bounded in time; a wait that runs out records FN_ERR_TIMEOUT in a
  *     device-side status word (read and cleared by flashnorm_check_device_error) and the kernel
  *     returns early instead of hanging.
+ *   - Host threads: entry points may be called from several threads. flashnorm_last_error is kept per
+ *     thread. The one-time per-device setup of the first calls on a device (kernel shared-memory
+ *     attributes, the SM count) sets the same values whoever performs it, so concurrent first calls
+ *     only repeat it.
  */
 #ifndef FLASHNORM_H
 #define FLASHNORM_H
