@@ -52,7 +52,10 @@ import numpy as np
 # ---------------------------------------------------------------------------
 
 def bf16_to_f64(bits) -> np.ndarray:
-    """Decode bf16 bit patterns exactly to float64."""
+    """Decode bf16 bit patterns exactly to float64.
+
+    Source: the bf16 format itself (the top 16 bits of an IEEE-754 binary32), not the pages.
+    """
     b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
     return b.view(np.float32).astype(np.float64)
 
@@ -91,20 +94,32 @@ def f64_to_bf16(v) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 def inv_rms(x: np.ndarray, eps: float) -> np.ndarray:
-    """Per-row 1 / sqrt(mean_i x_i^2 + eps), mean over the feature axis."""
+    """Per-row 1 / sqrt(mean_i x_i^2 + eps), mean over the feature axis.
+
+    Source: the RMSNorm definition ("Root Mean Square Layer Normalization", the paper it builds on); the
+    scalar the "FlashNorm: Fast Normalization for Transformers", Abstract item (ii) defers.
+    """
     x = np.asarray(x, dtype=np.float64)
     ms = np.mean(x * x, axis=-1)
     return 1.0 / np.sqrt(ms + eps)
 
 
 def rmsnorm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
-    """RMSNorm(x) = x / sqrt(mean(x^2) + eps) * g, row-wise."""
+    """RMSNorm(x) = x / sqrt(mean(x^2) + eps) * g, row-wise.
+
+    Source: "Root Mean Square Layer Normalization", the RMSNorm definition the FlashNorm paper builds
+    on.
+    """
     x = np.asarray(x, dtype=np.float64)
     return x * inv_rms(x, eps)[..., None] * np.asarray(g, dtype=np.float64)
 
 
 def norm_then_project(x, g, W, eps):
-    """The operation FlashNorm reformulates: RMSNorm(x) . W, W of shape [d, N]."""
+    """The operation FlashNorm reformulates: RMSNorm(x) . W, W of shape [d, N].
+
+    Source: "FlashNorm: Fast Normalization for Transformers", Abstract, the RMSNorm -> linear pair the
+    method starts from.
+    """
     return rmsnorm(x, g, eps) @ np.asarray(W, dtype=np.float64)
 
 
@@ -113,17 +128,28 @@ def norm_then_project(x, g, W, eps):
 # ---------------------------------------------------------------------------
 
 def fold(W, g) -> np.ndarray:
-    """W* = diag(g) . W in float64 (row i of W scaled by g_i)."""
+    """W* = diag(g) . W in float64 (row i of W scaled by g_i).
+
+    Source: "FlashNorm: Fast Normalization for Transformers", Abstract, item (i), weight folding.
+    """
     return np.asarray(g, dtype=np.float64)[:, None] * np.asarray(W, dtype=np.float64)
 
 
 def fold_bf16(w_bits, g_bits) -> np.ndarray:
-    """W* rounded once to bf16: bits of RNE(g_i * W_ij), same [d, N] shape as W."""
+    """W* rounded once to bf16: bits of RNE(g_i * W_ij), same [d, N] shape as W.
+
+    Source: "FlashNorm: Fast Normalization for Transformers", Abstract, item (i); the single RNE
+    rounding to bf16 is the reading that makes the fold exact to check.
+    """
     return f64_to_bf16(fold(bf16_to_f64(w_bits), bf16_to_f64(g_bits)))
 
 
 def deferred(x, Wstar, eps):
-    """(x . W*) scaled per row by 1/sqrt(mean(x^2) + eps): the reformulated form."""
+    """(x . W*) scaled per row by 1/sqrt(mean(x^2) + eps): the reformulated form.
+
+    Source: "FlashNorm: Fast Normalization for Transformers", Abstract, item (ii), deferred
+    normalization.
+    """
     x = np.asarray(x, dtype=np.float64)
     return (x @ np.asarray(Wstar, dtype=np.float64)) * inv_rms(x, eps)[:, None]
 
@@ -133,7 +159,11 @@ def deferred(x, Wstar, eps):
 # ---------------------------------------------------------------------------
 
 def silu(t):
-    """SiLU(t) = t / (1 + exp(-t))."""
+    """SiLU(t) = t / (1 + exp(-t)).
+
+    Source: the SiLU of the gated feed-forward layers that "FlashNorm: Fast Normalization for
+    Transformers", Abstract names among the extensions.
+    """
     t = np.asarray(t, dtype=np.float64)
     with np.errstate(over="ignore"):
         return t / (1.0 + np.exp(-t))
@@ -147,7 +177,11 @@ def glu_norm_then_project(x, g, W_gu, eps):
 
 
 def glu_deferred(x, Wstar_gu, eps):
-    """silu(r * (x . W*_gate)) * (r * (x . W*_up)), r = 1/rms(x): scale before SiLU."""
+    """silu(r * (x . W*_gate)) * (r * (x . W*_up)), r = 1/rms(x): scale before SiLU.
+
+    Source: "FlashNorm: Fast Normalization for Transformers", Abstract, the GLU variants: the deferred
+    scale goes on gate and up before SiLU.
+    """
     x = np.asarray(x, dtype=np.float64)
     r = inv_rms(x, eps)[:, None]
     z = x @ np.asarray(Wstar_gu, dtype=np.float64)
@@ -161,6 +195,12 @@ def glu_deferred(x, Wstar_gu, eps):
 # ---------------------------------------------------------------------------
 
 def _per_head_rmsnorm(v, g2, eps2, head_dim):
+    """RMSNorm over each head of head_dim consecutive features of a row, one gain g2 [head_dim] for all
+    heads.
+
+    Source: the per-head (query/key) norm of the redundant-norm case in "FlashNorm: Fast Normalization
+    for Transformers", Abstract; a head as the unit is the reading for QK-norm models.
+    """
     M, N = v.shape
     vh = v.reshape(M, N // head_dim, head_dim)
     return rmsnorm(vh, g2, eps2).reshape(M, N)
@@ -184,6 +224,9 @@ def postnorm_elided_exact_eps(x, Wstar1, g2, eps1, eps2, head_dim):
     With v = u * r1 and r1 = 1/sqrt(ms_x + eps1), mean(v^2) = r1^2 mean(u^2), so
     v / sqrt(mean(v^2) + eps2) = u / sqrt(mean(u^2) + eps2 (ms_x + eps1)).
     The elided form drops the eps2 (ms_x + eps1) correction; it is exact at eps = 0.
+
+    Source: "FlashNorm: Fast Normalization for Transformers", Abstract, redundant-norm removal by scale
+    invariance; this is that identity with eps kept.
     """
     x = np.asarray(x, dtype=np.float64)
     u = x @ np.asarray(Wstar1, dtype=np.float64)
@@ -258,7 +301,11 @@ def fold_fp8(w_bits, g_bits):
 
 
 def deferred_fp8(x, codes, scales, eps):
-    """y = (x . dec(Q)^T) * s * 1/sqrt(mean(x^2) + eps), in fp64."""
+    """y = (x . dec(Q)^T) * s * 1/sqrt(mean(x^2) + eps), in fp64.
+
+    Source: "FlashNorm: Fast Normalization for Transformers", Abstract, folded weights staying
+    compatible with quantized models; the E4M3 per-channel scheme is the reading stated at fold_fp8.
+    """
     x = np.asarray(x, dtype=np.float64)
     Wq = e4m3_to_f64(codes) * np.asarray(scales, dtype=np.float64)[:, None]   # [N, d]
     return (x @ Wq.T) * inv_rms(x, eps)[:, None]
@@ -278,7 +325,11 @@ def deferred_fp8(x, codes, scales, eps):
 # ---------------------------------------------------------------------------
 
 def layernorm(x, gamma, beta, eps):
-    """LayerNorm over the last axis (biased variance, two passes), float64."""
+    """LayerNorm over the last axis (biased variance, two passes), float64.
+
+    Source: the standard LayerNorm definition, which "FlashNorm: Fast Normalization for Transformers",
+    Abstract says the techniques extend to.
+    """
     x = np.asarray(x, dtype=np.float64)
     mu = np.mean(x, axis=-1, keepdims=True)
     var = np.mean((x - mu) ** 2, axis=-1, keepdims=True)
@@ -291,13 +342,20 @@ def layernorm_then_project(x, gamma, beta, W, eps):
 
 
 def layernorm_fold(W, gamma, beta):
-    """(W* = diag(gamma) W, c = 1^T W*, b = beta^T W), float64."""
+    """(W* = diag(gamma) W, c = 1^T W*, b = beta^T W), float64.
+
+    Source: "FlashNorm: Fast Normalization for Transformers", Abstract, item (i) applied to LayerNorm,
+    with the mean as a rank-1 term (the extension the abstract names).
+    """
     Ws = fold(W, gamma)
     return Ws, np.sum(Ws, axis=0), np.asarray(beta, dtype=np.float64) @ np.asarray(W, dtype=np.float64)
 
 
 def layernorm_deferred(x, Wstar, colsum, bias, eps):
-    """The folded, deferred form: r (x . W* - mu c) + b with r = 1/sqrt(var + eps)."""
+    """The folded, deferred form: r (x . W* - mu c) + b with r = 1/sqrt(var + eps).
+
+    Source: "FlashNorm: Fast Normalization for Transformers", Abstract, item (ii) applied to LayerNorm.
+    """
     x = np.asarray(x, dtype=np.float64)
     mu = np.mean(x, axis=-1)
     var = np.mean((x - mu[:, None]) ** 2, axis=-1)
@@ -320,7 +378,11 @@ def layernorm_deferred(x, Wstar, colsum, bias, eps):
 # ---------------------------------------------------------------------------
 
 def rope_table(max_pos: int, head_dim: int, base: float) -> np.ndarray:
-    """(cos, sin) of the rotation angles, float64 [max_pos, head_dim/2, 2]."""
+    """(cos, sin) of the rotation angles, float64 [max_pos, head_dim/2, 2].
+
+    Source: RoFormer's rotary embedding (the paper builds on it; "FlashNorm: Fast Normalization for
+    Transformers", Abstract names RoPE-based attention).
+    """
     i = np.arange(head_dim // 2, dtype=np.float64)
     inv_freq = np.power(float(base), -2.0 * i / head_dim)
     ang = np.arange(max_pos, dtype=np.float64)[:, None] * inv_freq[None, :]
@@ -332,6 +394,8 @@ def apply_rope(v, cs, positions, head_dim: int, n_rope_heads: int) -> np.ndarray
 
     cs is a (cos, sin) table [max_pos, head_dim/2, 2] (any float type; widened to
     float64) and positions [M] the position of each row.
+
+    Source: RoFormer's rotary embedding, adjacent-pair form.
     """
     v = np.array(v, dtype=np.float64, copy=True)
     M, N = v.shape
@@ -396,6 +460,9 @@ def exact_operand_output(kind: str, bits: dict, wstar_bits, eps: float, *, eps2:
 
     Used for fp32 outputs, where the fold's own bf16 rounding of W* would
     otherwise dominate the comparison.
+
+    Source: "FlashNorm: Fast Normalization for Transformers", Abstract, items (i) and (ii), evaluated on
+    the rounded operands.
     """
     x = bf16_to_f64(bits["x"])
     if rows is not None:
@@ -423,7 +490,11 @@ def reference_postnorm_rope(bits: dict, eps: float, eps2: float, head_dim: int, 
 
 def exact_operand_postnorm_rope(bits: dict, wstar_bits, eps2: float, head_dim: int, positions, n_rope_heads: int,
                                 table, rows=None) -> np.ndarray:
-    """The elided post-norm on the bf16 W*, rotated with the given (cos, sin) table: the fp32-output bar."""
+    """The elided post-norm on the bf16 W*, rotated with the given (cos, sin) table: the fp32-output bar.
+
+    Source: "FlashNorm: Fast Normalization for Transformers", Abstract, redundant-norm removal, then
+    RoFormer's rotation.
+    """
     x = bf16_to_f64(bits["x"])
     pos = np.asarray(positions)
     if rows is not None:
@@ -434,7 +505,10 @@ def exact_operand_postnorm_rope(bits: dict, wstar_bits, eps2: float, head_dim: i
 
 def exact_operand_fp8(bits: dict, eps: float, rows=None) -> np.ndarray:
     """The quantized path on its own operands: the oracle's fold_fp8 codes and scales (the library's fold
-    matches them bit for bit), then y = (x . dec(Q)^T) * s * 1/rms in fp64."""
+    matches them bit for bit), then y = (x . dec(Q)^T) * s * 1/rms in fp64.
+
+    Source: as deferred_fp8.
+    """
     x = bf16_to_f64(bits["x"])
     if rows is not None:
         x = x[rows]
@@ -451,7 +525,10 @@ def reference_layernorm(bits: dict, eps: float, rows=None) -> np.ndarray:
 
 
 def exact_operand_layernorm(bits: dict, wstar_bits, eps: float, rows=None) -> np.ndarray:
-    """The folded, deferred form on the bf16 W* (colsum from its bf16 values, bias from W and beta)."""
+    """The folded, deferred form on the bf16 W* (colsum from its bf16 values, bias from W and beta).
+
+    Source: as layernorm_deferred.
+    """
     x = bf16_to_f64(bits["x"])
     if rows is not None:
         x = x[rows]
@@ -461,7 +538,10 @@ def exact_operand_layernorm(bits: dict, wstar_bits, eps: float, rows=None) -> np
 
 
 def rel_err(y, y_ref) -> float:
-    """max |y - y_ref| / max |y_ref|, the parity metric."""
+    """max |y - y_ref| / max |y_ref|, the parity metric.
+
+    Source: not the pages; the parity metric the tests state.
+    """
     y = np.asarray(y, dtype=np.float64)
     y_ref = np.asarray(y_ref, dtype=np.float64)
     denom = np.max(np.abs(y_ref))
