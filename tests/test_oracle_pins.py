@@ -268,6 +268,13 @@ def check_rope(O):
     for p, pp, s in ((3, 10, 5), (0, 20, 11), (30, 2, 7)):
         if abs(dot(p, pp) - dot(p + s, pp + s)) > 1e-12:
             fails.append(f"rope relative position {p},{pp},{s}")
+    # RoFormer's complex form: pair (2i, 2i+1) as the number v_2i + j v_2i+1, multiplied by exp(j p theta_i)
+    theta = 10000.0 ** (-2.0 * np.arange(hd // 2) / hd)
+    z = v[:, :2 * hd].reshape(5, 2, hd // 2, 2)
+    zc = (z[..., 0] + 1j * z[..., 1]) * np.exp(1j * pos[:, None, None] * theta[None, None, :])
+    yc = np.stack([zc.real, zc.imag], axis=-1).reshape(5, 2 * hd)
+    if np.max(np.abs(yc - y[:, :2 * hd])) > 1e-12:
+        fails.append("rope vs the complex-exponential form")
     return fails
 
 
