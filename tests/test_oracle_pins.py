@@ -342,6 +342,17 @@ def check_fp8(O):
     step = np.maximum(np.abs(Ws) * 2.0 ** -4, 2.0 ** -10 * s[:, None])  # half a step: 2^-4 relative, 2^-10 s below 2^-6 s
     if np.any(err > step * (1 + 1e-6)):
         fails.append("fp8 fold: weight off by more than half a step")
+    # the quantized deferred output against the definition (RMSNorm, then the unquantized W): within the
+    # bound those half steps give, r_m * sum_k |x_mk| * step_nk, and well away from zero error
+    x = O.bf16_to_f64(O.f64_to_bf16(rng.standard_normal((6, d)) * np.exp(rng.uniform(-2, 2, (6, 1)))))
+    eps = 1e-6
+    y8 = O.deferred_fp8(x, Q, s, eps)
+    ydef = O.norm_then_project(x, O.bf16_to_f64(gb), O.bf16_to_f64(wb), eps)
+    bound = O.inv_rms(x, eps)[:, None] * (np.abs(x) @ step.T)
+    if np.any(np.abs(y8 - ydef) > bound * (1 + 1e-9) + 1e-15):
+        fails.append("fp8 deferred output outside the quantization bound")
+    if not (1e-4 < O.rel_err(y8, ydef) < 0.1):
+        fails.append("fp8 deferred output: error not of the size E4M3 gives")
     return fails
 
 
@@ -527,6 +538,17 @@ def _mut_ln_fold_colsum_unfolded(W, gamma, beta):
     Ws = O.fold(W, gamma)
     return Ws, np.sum(np.asarray(W, dtype=np.float64), axis=0), np.asarray(beta) @ np.asarray(W, dtype=np.float64)
 
+def _mut_fp8_deferred_no_scale(x, codes, scales, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return (x @ O.e4m3_to_f64(codes).T) * O.inv_rms(x, eps)[:, None]
+
+
+def _mut_fp8_deferred_scale_by_row(x, codes, scales, eps):
+    x = np.asarray(x, dtype=np.float64)
+    s = np.asarray(scales, dtype=np.float64)
+    return (x @ O.e4m3_to_f64(codes).T) * O.inv_rms(x, eps)[:, None] * s[: x.shape[0], None]
+
+
 MUTANTS = {
     "mean over d-1": ("inv_rms", _mut_mean_d_minus_1),
     "eps outside sqrt": ("inv_rms", _mut_eps_outside),
@@ -551,6 +573,8 @@ MUTANTS = {
     "fp8 truncation": ("f64_to_e4m3", _mut_fp8_truncate),
     "fp8 exponent bias 8": ("e4m3_to_f64", _mut_fp8_bias8),
     "fp8 one scale for the whole matrix": ("fold_fp8", _mut_fp8_scale_rows),
+    "fp8 channel scale dropped": ("deferred_fp8", _mut_fp8_deferred_no_scale),
+    "fp8 scale indexed by token": ("deferred_fp8", _mut_fp8_deferred_scale_by_row),
 }
 
 
