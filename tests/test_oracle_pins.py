@@ -8,7 +8,10 @@
   gate and up columns);
 * invariants the abstract states: folded == unfolded ("exact reformulation"),
   scale invariance of RMS, and the redundant-norm identity;
-* brute force in exact rational arithmetic (50-digit square roots) on tiny inputs.
+* brute force in exact rational arithmetic (50-digit square roots) on tiny inputs;
+* for the extensions: hand-worked RoPE and LayerNorm cases (tests/golden/), torch's CPU
+  layer_norm and float8_e4m3fn conversion, RoFormer's complex-exponential form of the
+  rotation, and the FP8 output within the bound its half-step quantization gives.
 
 The last test plants plausible mistakes in the oracle (on the CPU) and checks
 that every one of them is caught by at least one pin.
