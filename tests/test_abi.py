@@ -155,3 +155,32 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(fn, "_lib", None)
     with pytest.raises(fn.FlashNormError, match="is missing"):
         fn.load_library()
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    # a C99 program that includes the header, takes the address of every declared entry point and is
+    # linked against the library: the boundary needs nothing beyond C and the shared object
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    from rmsnorm_linear_projection_fold_b200 import build
+
+    lib_path = build.build()
+    names = _declared_symbols()
+    src = tmp_path / "consumer.c"
+    src.write_text("#include \"flashnorm.h\"\n#include <stdio.h>\n"
+                   "typedef void (*fn_ptr)(void);\n"
+                   "int main(void) {\n  fn_ptr fns[] = {\n"
+                   + "".join(f"    (fn_ptr)&{n},\n" for n in names)
+                   + "  };\n  printf(\"%d\\n\", (int)(sizeof(fns) / sizeof(fns[0])));\n  return 0;\n}\n")
+    exe = tmp_path / "consumer"
+    cmd = [gcc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"), str(src),
+           lib_path, "-Wl,--unresolved-symbols=ignore-in-shared-libs", "-o", str(exe)]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    env = dict(os.environ, LD_LIBRARY_PATH=os.path.dirname(lib_path) + ":" + os.environ.get("LD_LIBRARY_PATH", ""))
+    r = subprocess.run([str(exe)], capture_output=True, text=True, env=env, timeout=60)
+    assert r.returncode == 0 and int(r.stdout) == len(names), (r.stdout, r.stderr)
