@@ -11,7 +11,9 @@
 * brute force in exact rational arithmetic (50-digit square roots) on tiny inputs;
 * for the extensions: hand-worked RoPE and LayerNorm cases (tests/golden/), torch's CPU
   layer_norm and float8_e4m3fn conversion, RoFormer's complex-exponential form of the
-  rotation, and the FP8 output within the bound its half-step quantization gives.
+  rotation, and the FP8 output within the bound its half-step quantization gives;
+* the parity metric itself (rel_err, the comparator every GPU parity test uses) on
+  hand-worked cases where a sign, an absolute value or the denominator matters.
 
 The last test plants plausible mistakes in the oracle (on the CPU) and checks
 that every one of them is caught by at least one pin.
@@ -359,8 +361,27 @@ def check_fp8(O):
     return fails
 
 
+def check_rel_err(O):
+    """The parity metric max|y - y_ref| / max|y_ref| on hand-worked cases, chosen so that a sign, a
+    missing absolute value, the wrong denominator or swapped arguments each change the result."""
+    fails = []
+    cases = [
+        # y, y_ref, expected (worked by hand)
+        ([-5.0, 1.0], [-4.0, 1.0], 0.25),            # |dy| = (1, 0); max|y_ref| = 4 (not max y_ref = 1)
+        ([[0.0, 3.0], [1.0, 1.0]], [[0.5, 2.0], [1.0, -2.0]], 1.5),  # max|dy| = 3 at a negative reference
+        ([2.0, -3.0], [2.0, -3.0], 0.0),
+        ([1e-3, -2e-3], [0.0, 0.0], 2e-3),          # zero reference: the absolute difference
+    ]
+    for y, ref, want in cases:
+        got = O.rel_err(_arr(y), _arr(ref))
+        if not abs(got - want) <= 1e-15:
+            fails.append(f"rel_err({y}, {ref}) = {got}, expected {want}")
+    return fails
+
+
 ALL_CHECKS = [check_golden, check_torch_rmsnorm, check_torch_silu, check_torch_bf16,
-              check_closed_forms, check_invariants, check_brute_force, check_rope, check_layernorm, check_fp8]
+              check_closed_forms, check_invariants, check_brute_force, check_rope, check_layernorm, check_fp8,
+              check_rel_err]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
@@ -370,17 +391,59 @@ def test_oracle_pin(check):
 
 
 def test_reference_output_wrappers():
-    """The bit-array wrappers route to the pinned functions with the right operands."""
+    """The bit-array wrappers route to the pinned functions with the right operands, row subsets
+    included: linear, SwiGLU, post-norm, post-norm + RoPE, LayerNorm and FP8."""
     from flashnorm_inputs import Workload
 
+    rows = [1, 3]
+    # linear and SwiGLU (gate = the first F columns of W, up = the last F)
+    for kind in ("linear", "glu"):
+        bits = Workload("t", kind, 5, 24, 8, 1e-5, seed=3).draw()
+        x, g, W = (O.bf16_to_f64(bits[k]) for k in ("x", "g", "w"))
+        ws = O.fold_bf16(bits["w"], bits["g"])
+        Ws = O.bf16_to_f64(ws)
+        plain = O.norm_then_project if kind == "linear" else O.glu_norm_then_project
+        folded = O.deferred if kind == "linear" else O.glu_deferred
+        assert np.allclose(O.reference_output(kind, bits, 1e-5), plain(x, g, W, 1e-5), rtol=1e-15, atol=0)
+        assert np.allclose(O.reference_output(kind, bits, 1e-5, rows=rows), plain(x[rows], g, W, 1e-5),
+                           rtol=1e-15, atol=0)
+        assert np.allclose(O.exact_operand_output(kind, bits, ws, 1e-5, rows=rows), folded(x[rows], Ws, 1e-5),
+                           rtol=1e-15, atol=0)
+        assert O.reference_output(kind, bits, 1e-5).shape == (5, 8)
+    # post-norm: the full chain keeps the first norm, the exact-operand form drops it
     wl = Workload("t", "postnorm", 5, 24, 8, 1e-6, head_dim=4, eps2=1e-6, seed=7)
     bits = wl.draw()
     x, g, W, g2 = (O.bf16_to_f64(bits[k]) for k in ("x", "g", "w", "g2"))
     y = O.reference_output("postnorm", bits, 1e-6, eps2=1e-6, head_dim=4)
     assert np.allclose(y, O.postnorm_full(x, g, W, g2, 1e-6, 1e-6, 4), rtol=1e-15)
     ws = O.fold_bf16(bits["w"], bits["g"])
-    y2 = O.exact_operand_output("postnorm", bits, ws, 1e-6, eps2=1e-6, head_dim=4, rows=[1, 3])
-    assert np.allclose(y2, O.postnorm_elided(x[[1, 3]], O.bf16_to_f64(ws), g2, 1e-6, 4), rtol=1e-15)
+    y2 = O.exact_operand_output("postnorm", bits, ws, 1e-6, eps2=1e-6, head_dim=4, rows=rows)
+    assert np.allclose(y2, O.postnorm_elided(x[rows], O.bf16_to_f64(ws), g2, 1e-6, 4), rtol=1e-15)
+    # post-norm + RoPE: positions follow the selected rows
+    pos = np.array([4, 0, 2, 9, 1])
+    y = O.reference_postnorm_rope(bits, 1e-6, 1e-6, 4, pos, 1, 10000.0, rows=rows)
+    assert np.allclose(y, O.postnorm_rope_full(x[rows], g, W, g2, 1e-6, 1e-6, 4, pos[rows], 1, 10000.0),
+                       rtol=1e-15)
+    table = O.rope_table(10, 4, 10000.0)
+    y = O.exact_operand_postnorm_rope(bits, ws, 1e-6, 4, pos, 1, table, rows=rows)
+    u = O.postnorm_elided(x[rows], O.bf16_to_f64(ws), g2, 1e-6, 4)
+    assert np.allclose(y, O.apply_rope(u, table, pos[rows], 4, 1), rtol=1e-15)
+    assert not np.allclose(y, u)  # the rotation did something
+    # LayerNorm: gamma = bits["g"], beta = bits["beta"]; colsum of the bf16 W*, bias from the unfolded W
+    bits = Workload("t", "layernorm", 5, 24, 8, 1e-5, seed=4).draw()
+    x, g, W, beta = (O.bf16_to_f64(bits[k]) for k in ("x", "g", "w", "beta"))
+    assert np.allclose(O.reference_layernorm(bits, 1e-5, rows=rows),
+                       O.layernorm_then_project(x[rows], g, beta, W, 1e-5), rtol=1e-15)
+    ws = O.fold_bf16(bits["w"], bits["g"])
+    Ws = O.bf16_to_f64(ws)
+    assert np.allclose(O.exact_operand_layernorm(bits, ws, 1e-5, rows=rows),
+                       O.layernorm_deferred(x[rows], Ws, Ws.sum(axis=0), beta @ W, 1e-5), rtol=1e-13)
+    # FP8: the oracle's own fold, then the deferred form on the decoded codes
+    bits = Workload("t", "linear_fp8", 3, 32, 8, 1e-6, seed=5).draw()
+    x = O.bf16_to_f64(bits["x"])
+    codes, scales = O.fold_fp8(bits["w"], bits["g"])
+    assert np.allclose(O.exact_operand_fp8(bits, 1e-6, rows=[0, 2]), O.deferred_fp8(x[[0, 2]], codes, scales, 1e-6),
+                       rtol=1e-15)
 
 
 # ---------------------------------------------------------------------------
@@ -552,6 +615,22 @@ def _mut_fp8_deferred_scale_by_row(x, codes, scales, eps):
     return (x @ O.e4m3_to_f64(codes).T) * O.inv_rms(x, eps)[:, None] * s[: x.shape[0], None]
 
 
+def _mut_rel_err_signed(y, y_ref):
+    y, y_ref = np.asarray(y, dtype=np.float64), np.asarray(y_ref, dtype=np.float64)
+    return float(np.max(y - y_ref) / np.max(np.abs(y_ref)))
+
+
+def _mut_rel_err_denominator_of_y(y, y_ref):
+    y, y_ref = np.asarray(y, dtype=np.float64), np.asarray(y_ref, dtype=np.float64)
+    return float(np.max(np.abs(y - y_ref)) / np.max(np.abs(y)))
+
+
+def _mut_rel_err_max_not_abs(y, y_ref):
+    y, y_ref = np.asarray(y, dtype=np.float64), np.asarray(y_ref, dtype=np.float64)
+    d = np.max(y_ref)
+    return float(np.max(np.abs(y - y_ref)) / d) if d > 0 else float(np.max(np.abs(y - y_ref)))
+
+
 MUTANTS = {
     "mean over d-1": ("inv_rms", _mut_mean_d_minus_1),
     "eps outside sqrt": ("inv_rms", _mut_eps_outside),
@@ -578,6 +657,9 @@ MUTANTS = {
     "fp8 one scale for the whole matrix": ("fold_fp8", _mut_fp8_scale_rows),
     "fp8 channel scale dropped": ("deferred_fp8", _mut_fp8_deferred_no_scale),
     "fp8 scale indexed by token": ("deferred_fp8", _mut_fp8_deferred_scale_by_row),
+    "rel_err without the absolute value": ("rel_err", _mut_rel_err_signed),
+    "rel_err relative to the result": ("rel_err", _mut_rel_err_denominator_of_y),
+    "rel_err relative to max(y_ref)": ("rel_err", _mut_rel_err_max_not_abs),
 }
 
 
