@@ -2,10 +2,12 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-Default workload (one "step"): the SmolLM2-135M-shaped prefill of 8192 tokens, d = 576: the fused
-QKV projection (W [576, 960]) and the fused SwiGLU up-projection (W [576, 2 x 1536]), both with the
-RMSNorm gain folded into the weights and the 1/rms scale deferred into the kernels' epilogues.
-Weights are folded once, outside the timed region (folding is an offline step).
+Default workload (one "step"): the Llama-7B-shaped RMSNorm + SwiGLU up-projection of 2048 tokens,
+x [2048, 4096], gate/up W [4096, 2 x 11008] -> y [2048, 11008] (369 GFLOP), the largest single-GPU
+configuration, with the RMSNorm gain folded into the weights and the 1/rms scale deferred into the
+kernel's epilogue. --workload selects the others (the SmolLM2-135M-shaped prefill of 8192 tokens,
+Llama-7B QKV decode and prefill, the MLA latent post-norm, ...). Weights are folded once, outside the
+timed region (folding is an offline step).
 
 Timing: W untimed warm-up steps, then exactly K steps back to back between two CUDA events on the
 launching stream. The inputs are larger than L2: every buffer of a step (x, W*, y) exists in R
@@ -16,9 +18,11 @@ batch (weak scaling, no collective on the data path); the time is the max over r
 
 One JSON line is printed by rank 0. `value` is TFLOP/s of the contraction (2 M d N per projection)
 for prefill workloads and weight GB/s for decode workloads. `roofline` describes the dominant kernel
-against MEASURED_PEAKS.json, its duration taken with CUDA events around a separate run of that
-kernel alone, back to back over the same rotation (events inside the step loop would end the overlap
-of one kernel's tail with the next kernel's prologue); `e2e` is the same metric through the same C-ABI calls with host
+against MEASURED_PEAKS.json, its duration taken with CUDA events around a separate loop of that
+kernel alone (at least 200 launches and about a second, whatever K is), back to back over the same
+rotation (events inside the step loop would end the overlap of one kernel's tail with the next
+kernel's prologue). `unfused` times the two-kernel baseline against the fused step in alternating
+blocks and reports the median of the per-block ratios; `e2e` is the same metric through the same C-ABI calls with host
 buffers (pinned H2D copy of x and D2H copy of the outputs inside the timed region); `cpu_baseline`
 is the fp64 oracle timed on this host's cores on a bounded sample of the workload; `graph` (one GPU) is the
 same steps captured once in a CUDA graph and replayed, the launch mode of a serving loop.
@@ -65,18 +69,30 @@ BENCH_WORKLOADS = {
     "layernorm_qkv_m8192": ["layernorm_qkv_m8192"],
     "llama7b_qkv_fp8_m1": ["llama7b_qkv_fp8_m1"],
     "llama7b_qkv_fp8_m4": ["llama7b_qkv_fp8_m4"],
+    "llama7b_qkv_fp8_m16": ["llama7b_qkv_fp8_m16"],
+    "llama7b_qkv_fp8_gemv_m1": ["llama7b_qkv_fp8_m1"],
+    "llama7b_qkv_fp8_gemv_m4": ["llama7b_qkv_fp8_m4"],
+    # the same decode projection on the CUDA-core GEMV instead of the tensor-core decode kernel
+    "llama7b_qkv_gemv_m16": ["llama7b_qkv_m16"],
+    "llama7b_qkv_gemv_m1": ["llama7b_qkv_m1"],
 }
-DEFAULT_WORKLOAD = "smollm2_prefill_m8192"
+# Kernel family forced for a bench workload (default: the library's own choice, FN_PATH_AUTO).
+BENCH_PATHS = {"llama7b_qkv_gemv_m16": "gemv", "llama7b_qkv_gemv_m1": "gemv", "llama7b_qkv_fp8_gemv_m1": "gemv",
+               "llama7b_qkv_fp8_gemv_m4": "gemv"}
+DEFAULT_WORKLOAD = "llama7b_ffn_m2048"
 
-# DRAM traffic of the dominant kernel per launch, from the ncu capture summarised in profiles/
-# (dram__bytes_read.sum + dram__bytes_write.sum). Valid only for the kernel source it was taken on:
-# if the CUDA sources hash differently now, traffic is reported as null.
+# DRAM traffic of the dominant kernel per launch (dram__bytes_read.sum + dram__bytes_write.sum of one
+# ncu capture of that kernel). Valid only for the kernel source it was taken on: if the CUDA sources
+# hash differently now, traffic is reported as null.
 NCU_TRAFFIC = {
-    # workload: (bytes per launch, sha256[:16] of the csrc/*.cu* sources at capture time, profile file)
-    "smollm2_prefill_m8192": (13019904, "8aabada61cdaf1c6", "profiles/fused_gemm_pair_smollm2_ffn_m8192.md"),
-    "smollm2_ffn_m8192": (13019904, "8aabada61cdaf1c6", "profiles/fused_gemm_pair_smollm2_ffn_m8192.md"),
-    "llama7b_qkv_m4": (104848384, "8aabada61cdaf1c6", "profiles/decode_tc_llama7b_qkv_m4.md"),
+    # workload: (bytes per launch, sha256[:16] of the csrc/*.cu* sources at capture time)
 }
+
+# The dominant-kernel loop and each block of the fused/unfused comparison run at least this many
+# launches and this long, whatever --steps is, so that the clocks settle and samplers see the load.
+MIN_LAUNCHES = 200
+MIN_LOOP_S = 1.0
+UNFUSED_BLOCKS = 5
 
 L2_BYTES = 126 * 1000 * 1000
 MAX_COPIES = 8
@@ -224,8 +240,8 @@ def _set_bytes(wl) -> int:
 class Projection:
     """One workload's projection: R copies of its inputs resident in HBM, weights folded once each."""
 
-    def __init__(self, wl, fn, torch, copies, unfused):
-        self.wl, self.fn, self.torch = wl, fn, torch
+    def __init__(self, wl, fn, torch, copies, unfused, path="auto"):
+        self.wl, self.fn, self.torch, self.path = wl, fn, torch, path
         b = wl.draw()
         glu = wl.kind == "glu"
         x0 = _to_dev(b["x"], torch)
@@ -258,11 +274,11 @@ class Projection:
         wl, fn = self.wl, self.fn
         x = self.x[r] if x is None else x
         if wl.kind == "linear":
-            fn.flashnorm_linear(x, self.ws[r], wl.eps, out=self.y[r])
+            fn.flashnorm_linear(x, self.ws[r], wl.eps, out=self.y[r], path=self.path)
         elif wl.kind == "glu":
-            fn.flashnorm_glu(x, self.ws[r], wl.eps, out=self.y[r])
+            fn.flashnorm_glu(x, self.ws[r], wl.eps, out=self.y[r], path=self.path)
         elif wl.kind == "linear_fp8":
-            fn.flashnorm_linear_fp8(x, self.ws[r], self.fp8_scales[r], wl.eps, out=self.y[r])
+            fn.flashnorm_linear_fp8(x, self.ws[r], self.fp8_scales[r], wl.eps, out=self.y[r], path=self.path)
         elif wl.kind == "layernorm":
             fn.flashnorm_layernorm_linear(x, self.ws[r], self.ln_colsum, self.ln_bias, wl.eps, out=self.y[r])
         elif wl.kind == "postnorm_rope":
@@ -280,6 +296,13 @@ class Projection:
 
     def launches(self) -> int:
         return 1
+
+
+def loop_count(est_ms: float, min_s: float = MIN_LOOP_S, min_launches: int = MIN_LAUNCHES,
+               cap: int = 200000) -> int:
+    """Launches for a loop of calls that take est_ms each: at least min_launches and about min_s seconds."""
+    est_ms = max(float(est_ms), 1e-4)
+    return int(min(cap, max(min_launches, int(np.ceil(min_s * 1e3 / est_ms)))))
 
 
 def _time_back_to_back(torch, steps, body):
@@ -307,7 +330,8 @@ def run_ours(args, rank, world, device_index):
     per_set = sum(_set_bytes(w) for w in wls)
     copies = int(min(MAX_COPIES, max(2, -(-2 * L2_BYTES // per_set))))
     do_unfused = all(w.kind in ("linear", "glu") for w in wls) and not _is_decode(wls)
-    projs = [Projection(w, fn, torch, copies, do_unfused) for w in wls]
+    path = BENCH_PATHS.get(args.workload, "auto")
+    projs = [Projection(w, fn, torch, copies, do_unfused, path) for w in wls]
 
     # the dominant kernel: the projection with the most work
     dom = max(range(len(projs)), key=lambda i: wls[i].flops if not _is_decode(wls) else wls[i].bytes)
@@ -333,21 +357,19 @@ def run_ours(args, rank, world, device_index):
     fn.flashnorm_check_device_error()
     # The dominant kernel alone, back to back over the same rotation: events between the kernels of a
     # step would end the overlap of one kernel's tail with the next one's prologue (programmatic
-    # dependent launch), so the step loop above carries no per-kernel events. A workload of one
-    # projection has nothing else in its step: the step loop is that measurement already.
-    dom_sampler = sampler
-    if len(projs) == 1:
-        k_dom = args.steps
-        dom_ms = total_ms / args.steps
-        dom_timing = f"CUDA events around the {k_dom} timed steps (the step is this kernel alone)"
-    else:
-        k_dom = max(3, min(args.steps, 1000))
-        dom_sampler = ClockSampler(device_index)
-        with dom_sampler:
-            dom_total, _ = _time_back_to_back(torch, k_dom, lambda i: projs[dom].run(i % copies))
-        dom_ms = dom_total / k_dom
-        dom_timing = f"CUDA events around {k_dom} back-to-back launches of this kernel (same input rotation)"
-        fn.flashnorm_check_device_error()
+    # dependent launch), so the step loop above carries no per-kernel events. The loop runs at least
+    # MIN_LAUNCHES launches and MIN_LOOP_S seconds, sized from a short probe.
+    def dom_body(i):
+        projs[dom].run(i % copies)
+
+    probe_ms, _ = _time_back_to_back(torch, 20, dom_body)
+    k_dom = loop_count(probe_ms / 20)
+    dom_sampler = ClockSampler(device_index)
+    with dom_sampler:
+        dom_total, _ = _time_back_to_back(torch, k_dom, dom_body)
+    dom_ms = dom_total / k_dom
+    dom_timing = f"CUDA events around {k_dom} back-to-back launches of this kernel (same input rotation)"
+    fn.flashnorm_check_device_error()
     total_ms = max_over_ranks(total_ms, world, "cuda")
     if world > 1:
         torch.distributed.barrier()
@@ -383,16 +405,31 @@ def run_ours(args, rank, world, device_index):
         except Exception as e:  # reported, not fatal: the eager number above is the headline
             graph = {"unavailable": f"{type(e).__name__}: {str(e)[:160]}"}
 
-    # unfused two-kernel baseline (same workload, same timing), for what folding + deferral buy
+    # Unfused two-kernel baseline (same workload, same rotation), for what folding + deferral buy. The
+    # two arms alternate in UNFUSED_BLOCKS blocks of equal length, so that clock and power drift hit
+    # both; the reported ratio is the median of the per-block ratios.
     unfused = None
     if do_unfused:
+        def unf_body(i):
+            for p in projs:
+                p.run_unfused(i % copies)
+
         for i in range(args.warmup):
-            [p.run_unfused(i % copies) for p in projs]
+            unf_body(i)
         torch.cuda.synchronize()
-        k_unf = max(3, min(args.steps, 500))
-        unf_ms, _ = _time_back_to_back(torch, k_unf, lambda i: [p.run_unfused(i % copies) for p in projs])
-        unfused = {"ms_per_step": unf_ms / k_unf, "fused_speedup": (unf_ms / k_unf) / ms_per_step,
-                   "kernels_per_step": 2 * len(projs)}
+        n_blk = loop_count(ms_per_step, min_s=MIN_LOOP_S / 2)
+        fused_ms, unf_ms = [], []
+        for _ in range(UNFUSED_BLOCKS):
+            f_ms, _ = _time_back_to_back(torch, n_blk, step)
+            u_ms, _ = _time_back_to_back(torch, n_blk, unf_body)
+            fused_ms.append(f_ms / n_blk)
+            unf_ms.append(u_ms / n_blk)
+        fn.flashnorm_check_device_error()
+        ratios = [u / f for u, f in zip(unf_ms, fused_ms)]
+        unfused = {"ms_per_step": float(np.median(unf_ms)), "fused_ms_per_step": float(np.median(fused_ms)),
+                   "fused_speedup": float(np.median(ratios)), "speedup_min_max": [min(ratios), max(ratios)],
+                   "kernels_per_step": 2 * len(projs),
+                   "timing": f"{UNFUSED_BLOCKS} alternating blocks of {n_blk} fused and {n_blk} unfused steps"}
 
     # end to end through the same calls with host buffers: H2D of x, the kernels, D2H of the outputs
     k_e2e = max(3, min(args.steps, 100))
@@ -457,6 +494,7 @@ def run_ours(args, rank, world, device_index):
         "data": "synthetic (seeded; x ~ N(0,1) x log-uniform[0.1,10] row scale, g ~ U(0.5,1.5), W ~ N(0,1/d))",
         "config": {
             "workload": args.workload,
+            "kernel_path": path,
             "projections": [{"name": w.name, "kind": w.kind, "M": w.M, "d": w.d, "N": w.N, "eps": w.eps}
                             for w in wls],
             "tokens_per_rank": wls[0].M,

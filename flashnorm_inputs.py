@@ -164,6 +164,7 @@ WORKLOADS = {
     # Llama-7B QKV decode with the folded weight quantized to FP8 E4M3 per output channel
     "llama7b_qkv_fp8_m1": Workload("llama7b_qkv_fp8_m1", "linear_fp8", 1, 4096, 12288, 1e-6, seed=BASE_SEED + 2),
     "llama7b_qkv_fp8_m4": Workload("llama7b_qkv_fp8_m4", "linear_fp8", 4, 4096, 12288, 1e-6, seed=BASE_SEED + 2),
+    "llama7b_qkv_fp8_m16": Workload("llama7b_qkv_fp8_m16", "linear_fp8", 16, 4096, 12288, 1e-6, seed=BASE_SEED + 2),
     # LayerNorm (gain and bias) before the SmolLM2-sized QKV projection, 8192 tokens
     "layernorm_qkv_m8192": Workload("layernorm_qkv_m8192", "layernorm", 8192, 576, 960, 1e-5, seed=BASE_SEED + 7),
     # The same with RoPE fused after the per-head norm on the query and key heads (8 q + 4 k heads of 256,
