@@ -32,7 +32,10 @@
  *     identical outputs.
  *   - Every wait inside a kernel is bounded in time; a wait that runs out records FN_ERR_TIMEOUT in a
  *     device-side status word (read and cleared by flashnorm_check_device_error) and the kernel
- *     returns early instead of hanging.
+ *     returns early instead of hanging. The outputs of such a call are not valid; the tensor-core
+ *     decode kernel writes the outputs that a failed wait affects as NaN (its K-split partial sums
+ *     from the CTA that gave up are NaN), the prefill kernels leave the tiles they did not finish
+ *     unwritten.
  *   - Host threads: entry points may be called from several threads. flashnorm_last_error is kept per
  *     thread. The one-time per-device setup of the first calls on a device (kernel shared-memory
  *     attributes, the SM count) sets the same values whoever performs it, so concurrent first calls
@@ -195,14 +198,22 @@ FN_API fn_status flashnorm_layernorm_linear(const void* x, const void* Wstar, co
  *     y[m][n] = (sum_k x[m][k] Q[n][k]) * s[n] / sqrt(mean_k x[m][k]^2 + eps).
  * flashnorm_fold_weights_fp8: W bf16 [d, N] row-major, g bf16 [d] -> Q uint8 [N, d] (K-major E4M3 codes)
  *   and scales fp32 [N]; caller-owned device memory. d % 16 == 0, N % 8 == 0.
- * flashnorm_linear_fp8: the decode path (M <= FN_DECODE_MAX_M): a GEMV that streams Q, one byte per
- *   weight, half the bytes of bf16 W*, with x staged in shared memory. x bf16 [M, d]; y [M, N] of
- *   out_dtype. Larger M returns FN_ERR_UNSUPPORTED.
+ * flashnorm_linear_fp8: the decode path (M <= FN_DECODE_MAX_M), streaming Q, one byte per weight, half
+ *   the bytes of bf16 W*: y = (x . dec(Q)^T) * scales * 1/sqrt(mean(x^2) + eps). x bf16 [M, d];
+ *   y [M, N] of out_dtype. Larger M returns FN_ERR_UNSUPPORTED. Runs flashnorm_linear_fp8_ex with
+ *   FN_PATH_AUTO.
+ * flashnorm_linear_fp8_ex: the same with a kernel choice. FN_PATH_AUTO or FN_PATH_DECODE: the tensor-core
+ *   kernel (Q widened on chip, exactly, to f16; x given to the MMA as f16 after a per-token power-of-two
+ *   scale that makes every bf16 value of the token down to 2^-29 of its largest an exact f16, undone in
+ *   the epilogue; fp32 accumulation). FN_PATH_GEMV: the CUDA-core GEMV (x staged in shared memory, each
+ *   16-byte load carries 16 weights). Other paths return FN_ERR_INVALID_ARG.
  */
 FN_API fn_status flashnorm_fold_weights_fp8(const void* W, const void* g, void* Q, void* scales, int64_t d, int64_t N,
                                             void* stream);
 FN_API fn_status flashnorm_linear_fp8(const void* x, const void* Q, const void* scales, void* y, int64_t M, int64_t d,
                                       int64_t N, float eps, int out_dtype, void* stream);
+FN_API fn_status flashnorm_linear_fp8_ex(const void* x, const void* Q, const void* scales, void* y, int64_t M,
+                                         int64_t d, int64_t N, float eps, int out_dtype, int path, void* stream);
 
 /*
  * flashnorm_rope_table — fills rope_cs (fp32 [max_pos][head_dim / 2][2], caller-owned device memory,
@@ -241,7 +252,9 @@ FN_API fn_status flashnorm_glu_unfused(const void* x, const void* g, const void*
  *   Arguments and results as flashnorm_linear_unfused; M * d must not exceed FN_NOALLOC_MAX_ELEMS
  *   (larger requests return FN_ERR_UNSUPPORTED and launch nothing).
  *   The first call on a device looks up the scratch array's device address on that device (with
- *   that device current); make that first call before any stream capture.
+ *   that device current) and keeps it for the life of the process; make that first call before any
+ *   stream capture. A device reset (cudaDeviceReset, or the primary context torn down and created
+ *   again) invalidates the kept address: do not call this entry point on a device after resetting it.
  *   All calls share the one array and it keeps the previous call's contents (every call overwrites
  *   the rows it uses before reading them). Calls whose kernels overlap on the GPU -- on different
  *   streams, or from different host threads -- race on it; serialise them.

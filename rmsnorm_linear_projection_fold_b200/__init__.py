@@ -34,6 +34,7 @@ __all__ = [
     "flashnorm_fold_layernorm",
     "flashnorm_fold_weights_fp8",
     "flashnorm_linear_fp8",
+    "flashnorm_linear_fp8_ex",
     "flashnorm_layernorm_linear",
     "flashnorm_rmsnorm",
     "flashnorm_linear_unfused",
@@ -72,6 +73,7 @@ _SIGNATURES = {
     "flashnorm_fold_layernorm": [_P, _P, _P, _P, _P, _P, _I64, _I64, _P],
     "flashnorm_fold_weights_fp8": [_P, _P, _P, _P, _I64, _I64, _P],
     "flashnorm_linear_fp8": [_P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
+    "flashnorm_linear_fp8_ex": [_P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _INT, _P],
     "flashnorm_layernorm_linear": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_rmsnorm": [_P, _P, _P, _I64, _I64, _F, _P],
     "flashnorm_linear_unfused": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
@@ -262,8 +264,10 @@ def flashnorm_fold_weights_fp8(W: torch.Tensor, g: torch.Tensor):
 
 
 def flashnorm_linear_fp8(x: torch.Tensor, Q: torch.Tensor, scales: torch.Tensor, eps: float,
-                         out_dtype=torch.bfloat16, out=None) -> torch.Tensor:
-    """Decode (M <= 16) with FP8 weights: y = (x . dec(Q)^T) * scales * 1/sqrt(mean(x^2) + eps)."""
+                         out_dtype=torch.bfloat16, out=None, path: str = "auto") -> torch.Tensor:
+    """Decode (M <= 16) with FP8 weights: y = (x . dec(Q)^T) * scales * 1/sqrt(mean(x^2) + eps).
+
+    path "auto" / "decode": the tensor-core kernel; "gemv": the CUDA-core GEMV."""
     _need(x, "x", dim=2)
     _need(Q, "Q", torch.uint8, dim=2)
     _need(scales, "scales", torch.float32, dim=1)
@@ -273,8 +277,8 @@ def flashnorm_linear_fp8(x: torch.Tensor, Q: torch.Tensor, scales: torch.Tensor,
         raise ValueError("Q [N, d] and scales [N] must match x [M, d]")
     _same_device(x, Q=Q, scales=scales)
     y = _output(out, (M, N), out_dtype, x)
-    _invoke("flashnorm_linear_fp8", x, _ptr(x), _ptr(Q), _ptr(scales), _ptr(y), M, d, N, float(eps),
-            _out_code(out_dtype), _stream_ptr(x))
+    _invoke("flashnorm_linear_fp8_ex", x, _ptr(x), _ptr(Q), _ptr(scales), _ptr(y), M, d, N, float(eps),
+            _out_code(out_dtype), PATHS[path], _stream_ptr(x), report="flashnorm_linear_fp8")
     return y
 
 

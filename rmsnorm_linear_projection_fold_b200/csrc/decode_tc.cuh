@@ -11,7 +11,8 @@
 // When there are too few 128-row slabs to occupy the GPU, the contraction is split over K across a
 // thread-block cluster of `ksplit` CTAs: every CTA reduces one K range into its own accumulator and
 // sum of squares, the partial results are written into the leader CTA's shared memory through the
-// cluster's distributed shared memory, and the leader adds them, scales and stores.
+// cluster's distributed shared memory, and the leader adds them, scales and stores. A CTA whose bounded
+// wait gave up sends NaN partial sums, so the outputs they feed are NaN rather than plausible values.
 //
 // Warps: 0 = TMA producer, 1 = TMEM allocator + MMA issuer, 2..5 = sum of squares, then epilogue.
 #pragma once
@@ -206,6 +207,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         ph ^= 1u;
       }
     }
+    // A wait that gave up leaves this thread's part of the sum incomplete: it contributes NaN instead,
+    // so every output that depends on it is written as NaN (the status word reports the timeout).
+    const float kNaN = __int_as_float(0x7fc00000);
+    if (!ok) ss = kNaN;
     // the eight threads of a token are eight consecutive lanes
     ss += __shfl_xor_sync(0xffffffffu, ss, 4);
     ss += __shfl_xor_sync(0xffffffffu, ss, 2);
@@ -223,8 +228,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
       for (int j = 0; j < kDecTok; ++j) v[j] = __uint_as_float(r[j]);
     } else {
+      // an empty K range (more CTAs than k-blocks) contributes zero; a failed wait contributes NaN
 #pragma unroll
-      for (int j = 0; j < kDecTok; ++j) v[j] = 0.f;
+      for (int j = 0; j < kDecTok; ++j) v[j] = ok ? 0.f : kNaN;
     }
     const int row = q * 32 + lane;  // W* row within the slab held by this thread
     if (KSPLIT > 1) {
@@ -246,7 +252,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
       if (chunk == 0) rs[tok] = 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps);
       named_bar_sync(1, 128);
-      if (ok) {
+      {
         if (!GLU) {
           const int n = n0 + row;
 #pragma unroll

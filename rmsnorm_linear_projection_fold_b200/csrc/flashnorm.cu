@@ -13,6 +13,7 @@
 #include <utility>
 
 #include "../../include/flashnorm.h"
+#include "decode_fp8.cuh"
 #include "decode_tc.cuh"
 #include "elementwise.cuh"
 #include "fused_gemm.cuh"
@@ -20,6 +21,7 @@
 #include "fused_gemm_pair.cuh"
 #include "gemv.cuh"
 #include "postnorm_cluster.cuh"
+#include "postnorm_pair.cuh"
 
 namespace {
 
@@ -114,6 +116,21 @@ fn_status make_operand_map(CUtensorMap* map, const void* ptr, int64_t k, int64_t
   return FN_OK;
 }
 
+// 2-D one-byte operand [rows, k] (FP8 E4M3 codes) with a (128 x box_rows) box and 128-byte swizzle.
+fn_status make_u8_map(CUtensorMap* map, const void* ptr, int64_t k, int64_t rows, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k)};
+  cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  return FN_OK;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 fn_status check_ptr(const void* p, const char* name) {
@@ -185,8 +202,8 @@ fn_status launch_gemm_t(const CUtensorMap& tx, const CUtensorMap& tw, const fn::
 // ---- CTA-pair (2-SM MMA) variant ------------------------------------------------------------------
 
 template <int STAGES, int EPI, bool SCALE, bool OUT_F32>
-fn_status launch_gemm_pair_t(const CUtensorMap& tx, const CUtensorMap& tw, const fn::GemmParams& p, int sms, int dev,
-                             cudaStream_t stream) {
+fn_status launch_gemm_pair_t(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& tw2,
+                             const fn::GemmParams& p, int sms, int dev, cudaStream_t stream) {
   auto kern = fn::k_fused_gemm_pair<STAGES, EPI, SCALE, OUT_F32>;
   constexpr int smem = fn::gemm_pair_smem_bytes<STAGES>();
   static bool configured[kMaxDevices] = {false};
@@ -198,7 +215,7 @@ fn_status launch_gemm_pair_t(const CUtensorMap& tx, const CUtensorMap& tw, const
   const int tiles = p.num_m_tiles * p.num_n_tiles;
   const int pairs = tiles < sms / 2 ? tiles : sms / 2;
   cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(2 * pairs)), dim3(fn::gemm_threads(EPI, SCALE)),
-                                smem, stream, 2, tx, tw, p);
+                                smem, stream, 2, tx, tw, tw2, p);
   if (e != cudaSuccess) return cuda_fail(e, "pair GEMM launch");
   return FN_OK;
 }
@@ -211,12 +228,22 @@ fn_status run_pair_path(const void* x, const void* w, void* y, int64_t M, int64_
   if (sms <= 1) return fail(FN_ERR_CUDA, "cannot query the current device");
   // Pair tiles are 256 rows; the choice of width counts pairs of SMs. A tile's output columns are a
   // whole number of the epilogue's 64-byte chunks (32 bf16 outputs, i.e. 64 W* rows for the GLU).
-  const int bn = choose_bn((M + 1) / 2, n_rows, sms / 2,
-                           epi == fn::EPI_GLU ? 2 * fn::pair_chunk_cols(out_dtype == FN_F32) : 32);
-  CUtensorMap tx, tw;
+  const int step = epi == fn::EPI_GLU ? 2 * fn::pair_chunk_cols(out_dtype == FN_F32) : 32;
+  const int bn = choose_bn((M + 1) / 2, n_rows, sms / 2, step);
+  const int64_t num_m_tiles = (M + 2 * fn::kBM - 1) / (2 * fn::kBM);
+  const int64_t num_n_tiles = (n_rows + bn - 1) / bn;
+  const int64_t tiles = num_m_tiles * num_n_tiles;
+  const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
+  // A last wave that fills at most half of the pairs is run as half tiles, one per pair.
+  int64_t num_main = tiles;
+  const int64_t rem = tiles % pairs;
+  if (tiles > pairs && rem > 0 && 2 * rem <= pairs && (bn / 2) % step == 0) num_main = tiles - rem;
+  CUtensorMap tx, tw, tw2;
   fn_status st = make_operand_map(&tx, x, d, M, fn::kBM);
   if (st != FN_OK) return st;
   st = make_operand_map(&tw, w, d, n_rows, bn / 2);
+  if (st != FN_OK) return st;
+  st = make_operand_map(&tw2, w, d, n_rows, num_main < tiles ? bn / 4 : bn / 2);
   if (st != FN_OK) return st;
   fn::GemmParams p;
   p.y = y;
@@ -227,15 +254,16 @@ fn_status run_pair_path(const void* x, const void* w, void* y, int64_t M, int64_
   p.ldy = static_cast<int>(n_out);
   p.bn = bn;
   p.head_dim = 0;
-  p.num_m_tiles = static_cast<int>((M + 2 * fn::kBM - 1) / (2 * fn::kBM));
-  p.num_n_tiles = static_cast<int>((n_rows + bn - 1) / bn);
+  p.num_m_tiles = static_cast<int>(num_m_tiles);
+  p.num_n_tiles = static_cast<int>(num_n_tiles);
+  p.num_main = static_cast<int>(num_main);
   p.eps = eps;
   p.ln_colsum = ln_colsum;
   p.ln_bias = ln_bias;
   const bool f32 = out_dtype == FN_F32;
 #define FN_PAIR(EPI, SC)                                                                                        \
-  (f32 ? launch_gemm_pair_t<fn::kPairStages, EPI, SC, true>(tx, tw, p, sms, dev, stream)                       \
-       : launch_gemm_pair_t<fn::kPairStages, EPI, SC, false>(tx, tw, p, sms, dev, stream))
+  (f32 ? launch_gemm_pair_t<fn::kPairStages, EPI, SC, true>(tx, tw, tw2, p, sms, dev, stream)                  \
+       : launch_gemm_pair_t<fn::kPairStages, EPI, SC, false>(tx, tw, tw2, p, sms, dev, stream))
   if (epi == fn::EPI_LINEAR) return scale ? FN_PAIR(fn::EPI_LINEAR, true) : FN_PAIR(fn::EPI_LINEAR, false);
   if (epi == fn::EPI_LN) return FN_PAIR(fn::EPI_LN, true);
   return scale ? FN_PAIR(fn::EPI_GLU, true) : FN_PAIR(fn::EPI_GLU, false);
@@ -302,6 +330,7 @@ fn_status run_tensor_path(const void* x, const void* w, void* y, const void* g2,
 
 // ------------------------------------------------------------------------------------------------
 // Wide-head post-norm: one cluster of (head_dim / 128) x KS CTAs per 128-row tile and head
+// (replaced by the CTA-pair kernel below; kept until that one is measured)
 // ------------------------------------------------------------------------------------------------
 
 template <bool OUT_F32>
@@ -352,6 +381,101 @@ fn_status run_postnorm_cluster(const void* x, const void* w, const void* g2, voi
   if (st != FN_OK) return st;
   return out_dtype == FN_F32 ? launch_postnorm_cluster_t<true>(tx, tw, p, static_cast<int>(ctas), dev, stream)
                              : launch_postnorm_cluster_t<false>(tx, tw, p, static_cast<int>(ctas), dev, stream);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Wide-head post-norm on CTA pairs: one cluster of 2 x 2 x KS CTAs per 256-row tile and head
+// ------------------------------------------------------------------------------------------------
+
+// Clusters of `csize` CTAs of the wide-head kernel that can be resident at once on this device.
+template <bool OUT_F32>
+int postnorm_pair_max_clusters(int csize, int dev) {
+  static int cache[kMaxDevices][3] = {{0}};
+  const int slot = csize == 16 ? 2 : csize == 8 ? 1 : 0;
+  if (cache[dev][slot] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(csize));
+    cfg.blockDim = dim3(fn::kPpThreads);
+    cfg.dynamicSmemBytes = fn::postnorm_pair_smem_bytes();
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = static_cast<unsigned>(csize);
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn::k_postnorm_pair<OUT_F32>, &cfg) != cudaSuccess || n < 0) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    cache[dev][slot] = n > 0 ? n : -1;  // -1: this cluster size cannot run
+  }
+  return cache[dev][slot];
+}
+
+template <bool OUT_F32>
+fn_status run_postnorm_pair_t(const void* x, const void* w, const void* g2, void* y, int64_t M, int64_t d, int64_t N,
+                              int64_t head_dim, float eps2, cudaStream_t stream) {
+  int dev = 0;
+  const int sms = device_sm_count(&dev);
+  if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
+  auto kern = fn::k_postnorm_pair<OUT_F32>;
+  constexpr int smem = fn::postnorm_pair_smem_bytes();
+  static bool configured[kMaxDevices] = {false};
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (wide-head post-norm)");
+    configured[dev] = true;
+  }
+  fn::PostnormPairParams p;
+  p.y = y;
+  p.g2 = static_cast<const uint16_t*>(g2);
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(d);
+  p.N = static_cast<int>(N);
+  p.head_dim = static_cast<int>(head_dim);
+  p.num_m_tiles = static_cast<int>((M + 255) / 256);
+  p.eps2 = eps2;
+  const int64_t clusters = p.num_m_tiles * (N / head_dim);
+  const int64_t num_kb = (d + 63) / 64;
+  const int64_t nw = head_dim / 2;
+  // K ranges per cluster: the split with the fewest (waves x k-blocks per range + a fixed cost of about
+  // six k-blocks for the pipeline fill, the reduce-scatter and the stores), among those whose column
+  // slices are whole 16-column chunks and whose K ranges are not empty.
+  int best_ks = 0;
+  int64_t best_cost = INT64_MAX;
+  for (int ks = fn::kPpMaxKS; ks >= 1; ks /= 2) {
+    if ((nw / ks) % 16 != 0 || ks > num_kb) continue;
+    const int maxc = postnorm_pair_max_clusters<OUT_F32>(2 * fn::kPpNP * ks, dev);
+    if (maxc <= 0) continue;
+    const int64_t waves = (clusters + maxc - 1) / maxc;
+    const int64_t cost = waves * ((num_kb + ks - 1) / ks + 6);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best_ks = ks;
+    }
+  }
+  if (best_ks == 0) return fail(FN_ERR_UNSUPPORTED, "no cluster shape of the wide-head kernel can run on this device");
+  p.ks = best_ks;
+  const int64_t ctas = clusters * 2 * fn::kPpNP * best_ks;
+  if (ctas > INT32_MAX) return fail(FN_ERR_UNSUPPORTED, "too many tiles");
+  CUtensorMap tx, tw;
+  fn_status st = make_operand_map(&tx, x, d, M, 128);
+  if (st != FN_OK) return st;
+  st = make_operand_map(&tw, w, d, N, static_cast<int>(head_dim / 4));
+  if (st != FN_OK) return st;
+  cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(ctas)), dim3(fn::kPpThreads), smem, stream,
+                                static_cast<unsigned>(2 * fn::kPpNP * best_ks), tx, tw, p);
+  if (e != cudaSuccess) return cuda_fail(e, "wide-head post-norm launch");
+  return FN_OK;
+}
+
+fn_status run_postnorm_pair(const void* x, const void* w, const void* g2, void* y, int64_t M, int64_t d, int64_t N,
+                            int64_t head_dim, float eps2, int out_dtype, cudaStream_t stream) {
+  return out_dtype == FN_F32 ? run_postnorm_pair_t<true>(x, w, g2, y, M, d, N, head_dim, eps2, stream)
+                             : run_postnorm_pair_t<false>(x, w, g2, y, M, d, N, head_dim, eps2, stream);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -442,6 +566,76 @@ fn_status launch_gemv_fp8_t(const void* x, const void* q, const void* scales, vo
 }
 
 // ------------------------------------------------------------------------------------------------
+// FP8 decode on the tensor cores
+// ------------------------------------------------------------------------------------------------
+
+template <int KSPLIT, bool OUT_F32>
+fn_status launch_decode_fp8_t(const CUtensorMap& tq, const fn::DecodeFp8Params& p, int slabs, int smem, int dev,
+                              cudaStream_t stream) {
+  auto kern = fn::k_decode_fp8<KSPLIT, OUT_F32>;
+  static int configured[kMaxDevices] = {0};
+  if (configured[dev] < smem) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (fp8 decode)");
+    configured[dev] = smem;
+  }
+  cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(slabs * KSPLIT)), dim3(fn::kD8Threads),
+                                static_cast<size_t>(smem), stream, KSPLIT, tq, p);
+  if (e != cudaSuccess) return cuda_fail(e, "fp8 decode launch");
+  return FN_OK;
+}
+
+fn_status run_decode_fp8(const void* x, const void* q, const void* scales, void* y, int64_t M, int64_t d, int64_t N,
+                         float eps, int out_dtype, cudaStream_t stream) {
+  int dev = 0;
+  const int sms = device_sm_count(&dev);
+  if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
+  const int64_t slabs = (N + fn::kD8Rows - 1) / fn::kD8Rows;
+  const int64_t units = (d + fn::kD8KStage - 1) / fn::kD8KStage;
+  // K split: the one that leaves the least W* to the busiest SM (ceil(CTAs / SMs) CTAs of 1/ks slab each),
+  // among those whose CTA fits in shared memory; among equals the smaller split (fewer partial sums).
+  // Llama-7B QKV (96 slabs): in three, 288 CTAs of 112 KB, two on every SM.
+  int best = 0;
+  double best_load = 1e30;
+  for (int ks = 1; ks <= 4 && ks <= units; ++ks) {
+    if (fn::decode_fp8_smem_bytes(static_cast<int>((units + ks - 1) / ks), ks) > 227 * 1024) continue;
+    const double load = static_cast<double>((slabs * ks + sms - 1) / sms) / ks;
+    if (load < best_load - 1e-9) {
+      best_load = load;
+      best = ks;
+    }
+  }
+  if (best == 0) return fail(FN_ERR_UNSUPPORTED, "fp8 decode: d = %lld leaves no K split that fits in shared memory",
+                             (long long)d);
+  const int smem = fn::decode_fp8_smem_bytes(static_cast<int>((units + best - 1) / best), best);
+  CUtensorMap tq;
+  fn_status st = make_u8_map(&tq, q, d, N, fn::kD8Rows);
+  if (st != FN_OK) return st;
+  fn::DecodeFp8Params p;
+  p.y = y;
+  p.x = static_cast<const uint16_t*>(x);
+  p.scales = static_cast<const float*>(scales);
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(d);
+  p.N = static_cast<int>(N);
+  p.ldy = static_cast<int>(N);
+  p.ksplit = best;
+  p.eps = eps;
+  const int sl = static_cast<int>(slabs);
+  const bool f32 = out_dtype == FN_F32;
+#define FN_D8(KS)                                                                                              \
+  (f32 ? launch_decode_fp8_t<KS, true>(tq, p, sl, smem, dev, stream)                                           \
+       : launch_decode_fp8_t<KS, false>(tq, p, sl, smem, dev, stream))
+  switch (best) {
+    case 1: return FN_D8(1);
+    case 2: return FN_D8(2);
+    case 3: return FN_D8(3);
+    default: return FN_D8(4);
+  }
+#undef FN_D8
+}
+
+// ------------------------------------------------------------------------------------------------
 // Tensor-core decode path
 // ------------------------------------------------------------------------------------------------
 
@@ -472,6 +666,7 @@ fn_status run_decode_tc(const void* x, const void* w, void* y, int64_t M, int64_
   // Split K across a cluster so that more SMs stream W*: in two while there are at most as many slabs as
   // SMs (two 5-stage CTAs fit one SM), in four when there are few slabs. Llama-7B QKV (96 slabs): 22.7 ->
   // 19-21 us with the split in two; in four, 25.5 us.
+  // (A split in three, 288 four-stage CTAs two to an SM, measured 27.0 us against 20.6 us in two.)
   int ksplit = 1;
   if (slabs <= sms && num_kb >= 2) ksplit = 2;
   if (slabs * 4 <= sms && num_kb >= 4) ksplit = 4;
@@ -593,8 +788,8 @@ fn_status flashnorm_linear_postnorm(const void* x, const void* Wstar, const void
   if (N < head_dim || N > kMaxDim || N % head_dim != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a multiple of head_dim", (long long)N);
   if ((st = check_ptr(g2, "g2")) != FN_OK) return st;
   if (M == 0) return FN_OK;
-  if (head_dim > 256 && head_dim % fn::kPnCols == 0)
-    return run_postnorm_cluster(x, Wstar, g2, y, M, d, N, head_dim, eps2, out_dtype, static_cast<cudaStream_t>(stream));
+  if (head_dim > 256)
+    return run_postnorm_pair(x, Wstar, g2, y, M, d, N, head_dim, eps2, out_dtype, static_cast<cudaStream_t>(stream));
   return run_tensor_path(x, Wstar, y, g2, M, d, N, N, head_dim, eps2, out_dtype, fn::EPI_POSTNORM, false,
                          static_cast<cudaStream_t>(stream));
 }
@@ -685,9 +880,11 @@ fn_status flashnorm_fold_weights_fp8(const void* W, const void* g, void* Q, void
   return FN_OK;
 }
 
-fn_status flashnorm_linear_fp8(const void* x, const void* Q, const void* scales, void* y, int64_t M, int64_t d,
-                               int64_t N, float eps, int out_dtype, void* stream) {
+fn_status flashnorm_linear_fp8_ex(const void* x, const void* Q, const void* scales, void* y, int64_t M, int64_t d,
+                                  int64_t N, float eps, int out_dtype, int path, void* stream) {
   g_last_error[0] = '\0';
+  if (path != FN_PATH_AUTO && path != FN_PATH_DECODE && path != FN_PATH_GEMV)
+    return fail(FN_ERR_INVALID_ARG, "fp8 path %d: AUTO, DECODE or GEMV", path);
   fn_status st = check_common(x, Q, y, M, d, eps, out_dtype);
   if (st != FN_OK) return st;
   if (d % 16 != 0) return fail(FN_ERR_INVALID_ARG, "d = %lld must be a multiple of 16", (long long)d);
@@ -695,6 +892,8 @@ fn_status flashnorm_linear_fp8(const void* x, const void* Q, const void* scales,
   if (M > FN_DECODE_MAX_M) return fail(FN_ERR_UNSUPPORTED, "the fp8 path is the decode GEMV: M <= %d", FN_DECODE_MAX_M);
   if ((st = check_ptr(scales, "scales")) != FN_OK) return st;
   if (M == 0) return FN_OK;
+  if (path != FN_PATH_GEMV)
+    return run_decode_fp8(x, Q, scales, y, M, d, N, eps, out_dtype, static_cast<cudaStream_t>(stream));
   if (!gemv_fits(M, d)) return fail(FN_ERR_UNSUPPORTED, "x [%lld, %lld] does not fit in shared memory", (long long)M, (long long)d);
   int dev = 0;
   const int sms = device_sm_count(&dev);
@@ -712,6 +911,11 @@ fn_status flashnorm_linear_fp8(const void* x, const void* Q, const void* scales,
     default: return FN_G8(16, 1);
   }
 #undef FN_G8
+}
+
+fn_status flashnorm_linear_fp8(const void* x, const void* Q, const void* scales, void* y, int64_t M, int64_t d,
+                               int64_t N, float eps, int out_dtype, void* stream) {
+  return flashnorm_linear_fp8_ex(x, Q, scales, y, M, d, N, eps, out_dtype, FN_PATH_AUTO, stream);
 }
 
 fn_status flashnorm_rope_table(void* rope_cs, int64_t max_pos, int64_t head_dim, double base, void* stream) {

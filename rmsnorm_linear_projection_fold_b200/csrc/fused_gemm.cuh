@@ -65,6 +65,8 @@ struct GemmParams {
   // EPI_LN: fp32 [n_out] column sums of the folded W* and folded bias beta^T W
   const float* ln_colsum = nullptr;
   const float* ln_bias = nullptr;
+  // CTA-pair kernel: tiles 0 .. num_main-1 are full width, the rest are split in two halves
+  int num_main = 0;
 };
 
 template <int MAX_BN>
@@ -497,11 +499,16 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
       const bool fresh = mt != last_m;  // same for the whole CTA
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
       for (int kb = 0; kb < num_kb; ++kb) {
-        // Every stage use still gets this warp's release (the stage barriers count it). When the row
-        // block's sum of squares is already known, the warp does not read the stage and releases it as
-        // soon as the stage's previous use has completed, i.e. before it is even refilled, so that it
-        // never delays the refill; otherwise it waits for the data and reads it.
-        if (!(fresh ? mbar_wait(&full[s], ph, abort_flag) : mbar_wait(&empty[s], ph ^ 1u, abort_flag))) {
+        // Every stage use gets this warp's release (the stage barriers count it), and the warp waits
+        // for every use's data, reading it only when the row block's sum of squares is not known yet.
+        // The wait matters even when nothing is read: a parity wait tells its phase apart only from the
+        // phase just before it. A warp that skipped the data waits could run ahead, release a use the
+        // TMA had not filled yet, and then, on the next row block, find the full barrier's phase
+        // two uses back completed (same parity), take it as this use, read stale x and arrive a
+        // second time on the earlier phase of `empty`. That phase would then complete without the MMA's
+        // commit, the refill would overlap a load in flight, and a later full phase would never
+        // collect its bytes.
+        if (!mbar_wait(&full[s], ph, abort_flag)) {
           ok = false;
           break;
         }

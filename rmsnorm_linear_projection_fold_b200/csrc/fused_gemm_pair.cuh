@@ -10,9 +10,14 @@
 //     leader's stage barrier, and the leader's commits arrive on both CTAs' barriers (commit
 //     multicast; every TMA load is an ordinary single-CTA fetch);
 //   * each CTA's tensor memory holds the accumulator of its own 128 rows, read by its own epilogue;
-//   * each CTA's sum-of-squares warps read only their own x tile; the leader forwards "stage landed"
-//     to both CTAs once the whole pair stage is in, and each stage is released only after the MMA
-//     and the CTA's own reduction warps are done with it (the explicit join of the 1-SM kernel);
+//   * each CTA's sum-of-squares warps read only their own x tile, and only on a row block's first tile
+//     in this pair's tile range (later tiles of the row block reuse its 1/rms). On those stage uses the
+//     leader forwards "stage landed" (xfull) to both CTAs once the whole pair stage is in, and the
+//     stage is refilled only after the MMA's commit (empty) AND the CTA's own reduction warps
+//     (xempty) have released it, the explicit join of the 1-SM kernel. On every other use the MMA's
+//     commit alone releases the stage and the reduction warps take no part: no waits or arrivals on
+//     the MMA issuer's or the producer's path. Producer, MMA issuer and reduction warps all derive
+//     which uses are read from the same tile sequence, so their phase counts agree stage by stage;
 //   * the epilogue stages each warp's 32 rows x 64 bytes of output in swizzled shared memory and writes
 //     them back row-contiguously (8 rows x 64 bytes per warp store) instead of every lane storing its
 //     own row (32 cache lines per warp store, which made the epilogue as long as a short-K tile).
@@ -37,10 +42,15 @@ __host__ __device__ constexpr int gemm_pair_smem_bytes() {
 __host__ __device__ constexpr int pair_chunk_cols(bool out_f32) { return out_f32 ? 16 : 32; }
 
 // p.num_m_tiles counts 256-row pair tiles; p.bn is the pair tile width (W* rows), each CTA holding bn/2.
+// Tiles are handed to CTA pairs in contiguous ranges (row-block-major). When the tile count leaves a
+// short last wave, its tiles (the last num_tiles - p.num_main of them) are each split into two halves
+// of bn/2 columns, one half per pair: with 688 tiles on 74 pairs (Llama-7B SwiGLU, 2048 tokens) every
+// pair runs 9 full tiles and at most one half tile, 9.5 tile times instead of 10. tm_w loads the W*
+// rows of a full tile (bn/2 per CTA), tm_w2 those of a half tile (bn/4 per CTA).
 template <int STAGES, int EPI, bool SCALE, bool OUT_F32>
 __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
     k_fused_gemm_pair(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                      GemmParams p) {
+                      const __grid_constant__ CUtensorMap tm_w2, GemmParams p) {
   constexpr bool LN = EPI == EPI_LN;
   static_assert(!LN || SCALE, "the LayerNorm epilogue needs the mean and variance warps");
   constexpr int kSsWarps = SCALE ? 4 : 0;
@@ -58,7 +68,8 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(tail);  // used in the leader
   uint64_t* empty = full + STAGES;
   uint64_t* xfull = empty + STAGES;                     // "x tile of this stage has landed" (reduction)
-  uint64_t* acc_full = xfull + STAGES;                  // [2]
+  uint64_t* xempty = xfull + STAGES;                    // "reduction warps are done with this stage"
+  uint64_t* acc_full = xempty + STAGES;                 // [2]
   uint64_t* acc_empty = acc_full + 2;                   // [2], used in the leader
   uint64_t* ss_full = acc_empty + 2;                    // [2]
   uint64_t* ss_empty = ss_full + 2;                     // [2]
@@ -76,8 +87,9 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);  // the leader's expect-tx arrival covers both CTAs' bytes
-      mbar_init(&empty[s], 1 + kSsWarps);
+      mbar_init(&empty[s], 1);  // the MMA's commit (multicast to both CTAs)
       mbar_init(&xfull[s], 1);
+      mbar_init(&xempty[s], kSsWarps > 0 ? kSsWarps : 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -92,6 +104,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_w2);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, kTmemCols);
@@ -107,33 +120,64 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
   const int num_tiles = p.num_m_tiles * p.num_n_tiles;
   const int cl = static_cast<int>(blockIdx.x) >> 1;
   const int ncl = static_cast<int>(gridDim.x) >> 1;
-  const int t_begin = static_cast<int>(static_cast<long long>(cl) * num_tiles / ncl);
-  const int t_end = static_cast<int>(static_cast<long long>(cl + 1) * num_tiles / ncl);
+  const int t_begin = static_cast<int>(static_cast<long long>(cl) * p.num_main / ncl);
+  const int t_end = static_cast<int>(static_cast<long long>(cl + 1) * p.num_main / ncl);
+  const int num_halves = 2 * (num_tiles - p.num_main);
+  const int n_items = (t_end - t_begin) + (cl < num_halves ? 1 : 0);
   const int num_kb = (p.K + kBK - 1) / kBK;
   const int bn = p.bn;
-  const int half = bn / 2;
+  // Item i of this pair: its row block, first W* row and width (full tiles first, then a half tile).
+  auto tile_at = [&](int i, int& mt, int& n0, int& width) {
+    if (i < t_end - t_begin) {
+      const int t = t_begin + i;
+      mt = t / p.num_n_tiles;
+      n0 = (t % p.num_n_tiles) * bn;
+      width = bn;
+    } else {
+      const int t = p.num_main + (cl >> 1);
+      mt = t / p.num_n_tiles;
+      n0 = (t % p.num_n_tiles) * bn + (cl & 1) * (bn / 2);
+      width = bn / 2;
+    }
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       // per CTA; the leader announces the whole pair stage, the peer's loads only complete on it
-      const uint32_t stage_bytes = static_cast<uint32_t>(kAStageBytes + half * kBK * 2);
       int s = 0;
       uint32_t ph = 0;
       int issued = 0;
       bool ok = true;
-      for (int t = t_begin; t < t_end && ok; ++t) {
-        const int m0 = (t / p.num_n_tiles) * (2 * kBM) + static_cast<int>(rank) * kBM;
-        const int n0 = (t % p.num_n_tiles) * bn + static_cast<int>(rank) * half;
+      uint32_t x_read = 0;  // bit s: the current use of stage s is read by the reduction warps
+      uint32_t x_ph = 0;    // bit s: parity of the next xempty phase of stage s
+      int last_m = -1;
+      for (int i = 0; i < n_items && ok; ++i) {
+        int mt, n0t, width;
+        tile_at(i, mt, n0t, width);
+        const bool fresh = SCALE && mt != last_m;
+        last_m = mt;
+        const int m0 = mt * (2 * kBM) + static_cast<int>(rank) * kBM;
+        const int n0 = n0t + static_cast<int>(rank) * (width / 2);
+        const uint32_t stage_bytes = static_cast<uint32_t>(kAStageBytes + (width / 2) * kBK * 2);
+        const CUtensorMap* map_w = width == bn ? &tm_w : &tm_w2;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_cluster(&empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
+          if (SCALE && ((x_read >> s) & 1u)) {  // the previous use was also read by the reduction warps
+            if (!mbar_wait(&xempty[s], (x_ph >> s) & 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            x_ph ^= 1u << s;
+          }
+          x_read = fresh ? (x_read | (1u << s)) : (x_read & ~(1u << s));
           const uint32_t leader_full = dsmem_addr(&full[s], 0);
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * stage_bytes);
           tma_load_2d_pair(sA + s * kAStageBytes, &tm_x, leader_full, kb * kBK, m0);
-          tma_load_2d_pair(sB + s * kPairBStage, &tm_w, leader_full, kb * kBK, n0);
+          tma_load_2d_pair(sB + s * kPairBStage, map_w, leader_full, kb * kBK, n0);
           ++issued;
           if (++s == STAGES) {
             s = 0;
@@ -172,13 +216,18 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ pair MMA issuer (leader)
     if (lane == 0 && leader) {
-      const uint32_t idesc = make_idesc_bf16(2 * kBM, bn);
       int s = 0;
       uint32_t ph = 0;
       int acc = 0;
       uint32_t acc_ph = 0;
       bool ok = true;
-      for (int t = t_begin; t < t_end && ok; ++t) {
+      int last_m = -1;
+      for (int i = 0; i < n_items && ok; ++i) {
+        int mt, n0t, width;
+        tile_at(i, mt, n0t, width);
+        const uint32_t idesc = make_idesc_bf16(2 * kBM, width);
+        const bool fresh = SCALE && mt != last_m;
+        last_m = mt;
         if (!mbar_wait_cluster(&acc_empty[acc], acc_ph ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -191,7 +240,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
             break;
           }
           tc_fence_after_sync();
-          if (SCALE) {  // both CTAs' reduction warps may read their x tiles now
+          if (fresh) {  // both CTAs' reduction warps may read their x tiles now
             mbar_arrive(&xfull[s]);
             mbar_arrive_remote(dsmem_addr(&xfull[s], 1));
           }
@@ -230,9 +279,9 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
     uint32_t acc_ph = 0;
     int sb = 0;
     uint32_t sb_ph = 0;
-    for (int t = t_begin; t < t_end; ++t) {
-      const int mt = t / p.num_n_tiles;
-      const int nt = t % p.num_n_tiles;
+    for (int i = 0; i < n_items; ++i) {
+      int mt, n0t, width;
+      tile_at(i, mt, n0t, width);
       if (!mbar_wait_cluster(&acc_full[acc], acc_ph, abort_flag)) break;
       tc_fence_after_sync();
       float r = 1.0f, km = 0.0f;
@@ -251,8 +300,8 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * 256);
       constexpr int CC = pair_chunk_cols(OUT_F32);
       constexpr int kEsz = OUT_F32 ? 4 : 2;
-      const int ocols = EPI == EPI_GLU ? bn / 2 : bn;
-      const int ocol0 = nt * ocols;
+      const int ocols = EPI == EPI_GLU ? width / 2 : width;
+      const int ocol0 = EPI == EPI_GLU ? n0t / 2 : n0t;
       // 16-byte piece j (0..3) of row r sits at r*64 + ((j ^ (r >> 1)) & 3) * 16: conflict-free both for
       // a quarter-warp writing one piece of eight rows and for one reading two whole rows.
       auto put16 = [&](int j, uint4 v) {
@@ -260,7 +309,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
       };
       // The two warps of a lane quarter take alternate chunks; which one starts alternates from tile to
       // tile, so an odd chunk count does not always land on the same warp.
-      for (int ch = (hh + t - t_begin) & 1; ch * CC < ocols && ocol0 + ch * CC < p.n_out; ch += 2) {
+      for (int ch = (hh + i) & 1; ch * CC < ocols && ocol0 + ch * CC < p.n_out; ch += 2) {
         if (EPI == EPI_LINEAR || LN) {
           // CC accumulator columns -> CC outputs (4 pieces of 16 bytes): the deferred scale r, and for
           // LayerNorm also the rank-1 mean correction and the folded bias, y = r acc - (r mu) colsum + bias
@@ -360,29 +409,33 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
     const int q = warp & 3;
     const int row_in_tile = q * 32 + lane;
     int s = 0;
-    uint32_t ph = 0;
+    uint32_t x_ph = 0;  // bit s: parity of the next xfull phase of stage s (one phase per use read)
     int sb = 0;
     uint32_t sb_ph = 0;
     int last_m = -1;
     float r_row = 0.0f, km_row = 0.0f;
     bool ok = true;
-    for (int t = t_begin; t < t_end && ok; ++t) {
-      const int mt = t / p.num_n_tiles;
+    for (int i = 0; i < n_items && ok; ++i) {
+      int mt, n0t, width;
+      tile_at(i, mt, n0t, width);
       const bool fresh = mt != last_m;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
       float s0 = 0.f, s1 = 0.f;  // LayerNorm: sum of x
-      for (int kb = 0; kb < num_kb; ++kb) {
-        // As in the 1-CTA kernel: with this row block's 1/rms already known, release each stage use as
-        // soon as its previous use has completed, without reading it (off the refill's critical path).
-        if (!(fresh ? mbar_wait_cluster(&xfull[s], ph, abort_flag)
-                    : mbar_wait_cluster(&empty[s], ph ^ 1u, abort_flag))) {
+      if (!fresh) {
+        // this row block's 1/rms is known: the tile's stage uses pass without us
+        s = (s + num_kb) % STAGES;
+      }
+      for (int kb = 0; fresh && kb < num_kb; ++kb) {
+        // Every use read here is waited for in order, so this warp is never more than one xfull phase
+        // behind and the parity wait is unambiguous.
+        if (!mbar_wait_cluster(&xfull[s], (x_ph >> s) & 1u, abort_flag)) {
           ok = false;
           break;
         }
+        x_ph ^= 1u << s;
         const uint8_t* line = sA + s * kAStageBytes + row_in_tile * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          if (!fresh) break;
           const uint4 w = *reinterpret_cast<const uint4*>(line + (((c ^ lane) & 7) << 4));
           float f;
           f = bf16lo_to_f32(w.x); a0 = fmaf(f, f, a0); if (LN) s0 += f;
@@ -396,11 +449,8 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
         }
         fence_proxy_async_smem();  // reads above before the TMA refill our arrival permits
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-        if (++s == STAGES) {
-          s = 0;
-          ph ^= 1u;
-        }
+        if (lane == 0) mbar_arrive(&xempty[s]);
+        if (++s == STAGES) s = 0;
       }
       if (!ok) break;
       if (fresh) {

@@ -184,3 +184,40 @@ def test_header_is_plain_c_and_links(tmp_path):
     env = dict(os.environ, LD_LIBRARY_PATH=os.path.dirname(lib_path) + ":" + os.environ.get("LD_LIBRARY_PATH", ""))
     r = subprocess.run([str(exe)], capture_output=True, text=True, env=env, timeout=60)
     assert r.returncode == 0 and int(r.stdout) == len(names), (r.stdout, r.stderr)
+
+
+def test_noalloc_limit_matches_the_header():
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+FN_NOALLOC_MAX_ELEMS\s+\(?\s*([^\n/]+?)\)?\s*(?:/[/*].*)?$", text, flags=re.M)
+    assert m, "FN_NOALLOC_MAX_ELEMS not found in the header"
+    expr = m.group(1).replace("LL", "").replace("ll", "").replace("(int64_t)", "")
+    assert eval(expr, {"__builtins__": {}}) == fn.NOALLOC_MAX_ELEMS
+
+
+# flashnorm_linear_unfused_noalloc(x, g, W_kmajor, y, M, d, N, eps, out_dtype, stream): everything below is
+# decided before any CUDA call, so fake pointers never reach the device.
+@pytest.mark.parametrize("args,expected", [
+    ((P, P, P, P, 4, 576, 964, 1e-5, 0, NULL), fn.FN_ERR_INVALID_ARG),            # N % 8 != 0
+    ((NULL, P, P, P, 4, 576, 960, 1e-5, 0, NULL), fn.FN_ERR_INVALID_ARG),         # x NULL
+    ((P_MISALIGNED, P, P, P, 4, 576, 960, 1e-5, 0, NULL), fn.FN_ERR_ALIGN),       # x misaligned
+    ((P, P, P, P, 4, 576, 960, -1.0, 0, NULL), fn.FN_ERR_INVALID_ARG),            # eps < 0
+    ((P, P, P, P, fn.NOALLOC_MAX_ELEMS // 4096 + 1, 4096, 512, 1e-5, 0, NULL), fn.FN_ERR_UNSUPPORTED),
+    ((P, P, P, P, 0, 576, 960, 1e-5, 0, NULL), fn.FN_OK),                          # empty call
+])
+def test_noalloc_validation(lib, args, expected):
+    assert lib.flashnorm_linear_unfused_noalloc(*args) == expected
+    if expected != fn.FN_OK:
+        assert lib.flashnorm_last_error() != b""
+
+
+# flashnorm_linear_fp8_ex(x, Q, scales, y, M, d, N, eps, out_dtype, path, stream): rejected on the host
+@pytest.mark.parametrize("args,expected", [
+    ((P, P, P, P, 4, 576, 960, 1e-6, 0, 1, NULL), fn.FN_ERR_INVALID_ARG),    # the 1-CTA prefill path
+    ((P, P, P, P, 4, 576, 960, 1e-6, 0, 9, NULL), fn.FN_ERR_INVALID_ARG),    # unknown path
+    ((P, P, P, P, 17, 576, 960, 1e-6, 0, 0, NULL), fn.FN_ERR_UNSUPPORTED),   # decode only: M <= 16
+    ((P, P, P, P, 4, 584, 960, 1e-6, 0, 3, NULL), fn.FN_ERR_INVALID_ARG),    # d % 16 != 0
+    ((P, P, NULL, P, 4, 576, 960, 1e-6, 0, 3, NULL), fn.FN_ERR_INVALID_ARG),  # scales NULL
+    ((P, P, P, P, 0, 576, 960, 1e-6, 0, 3, NULL), fn.FN_OK),                  # empty call
+])
+def test_fp8_validation(lib, args, expected):
+    assert lib.flashnorm_linear_fp8_ex(*args) == expected

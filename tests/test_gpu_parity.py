@@ -6,9 +6,10 @@ bf16 outputs, two checks:
   (1) element by element, within half a bf16 ulp of that exact-operand fp64 result (plus the fp32
       slack above): the kernel computes the right value and rounds it once;
   (2) against the oracle's unfolded, undeferred chain, max|y - y_ref| / max|y_ref| <= 5e-3, the stated
-      bar -- unless the inputs make that bar unreachable for ANY bf16 result: rounding an output to bf16
-      alone can cost 2^-8 of max|y| (8 significant bits), and storing the folded W* in bf16 costs the
-      fold error the oracle measures on the same inputs. The bar is then that derived bound.
+      bar, flat. A few named inputs (DERIVED_BAR) put that bar out of reach of the method itself: the
+      folded W* is a bf16 tensor, so even the correctly rounded exact result on it misses 5e-3 there
+      (tests/test_parity_bar.py shows this on the CPU for each one). Only those take the derived bar:
+      2^-8 of max|y| for the output rounding plus the fold error the oracle measures on the same inputs.
 The fold is bit-exact. All calls go through the C ABI (the thin binding only passes pointers).
 """
 
@@ -31,32 +32,31 @@ def _wl(kind, M, d, N, eps=1e-5, seed=11, head_dim=0, eps2=0.0):
     return I.Workload("t", kind, M, d, N, eps, head_dim=head_dim, eps2=eps2, seed=seed)
 
 
-def check_bf16(y16, ref, ref_exact):
-    """The two bf16 checks described in the module docstring. Returns the error vs the unfolded oracle."""
+# Inputs, as (kind, M, d, N, seed), on which the flat 5e-3 bar is unreachable for the reformulated form
+# itself: the correctly rounded bf16 value of the exact result on the bf16 W* already misses it.
+DERIVED_BAR = {
+    ("linear", 16, 576, 960, 16 * 7 + 576): "bf16(exact) is 5.15e-3 from the definition",
+}
+
+
+def derived_bound(ref, ref_exact):
+    """Output rounding (up to 2^-8 of max|y|) plus the bf16 fold's own error on these inputs, plus fp32 slack."""
+    return 2.0 ** -8 * np.max(np.abs(ref_exact)) / np.max(np.abs(ref)) + O.rel_err(ref_exact, ref) + F32_TOL
+
+
+def check_bf16(y16, ref, ref_exact, derived=False):
+    """The two bf16 checks described in the module docstring. Returns the error vs the unfolded oracle.
+
+    derived=True only for the inputs named in DERIVED_BAR."""
     y16 = np.asarray(y16, dtype=np.float64)
     _, e = np.frexp(ref_exact)
     half_ulp = np.ldexp(1.0, e - 9)
     slack = F32_TOL * np.max(np.abs(ref_exact))
     assert np.all(np.abs(y16 - ref_exact) <= half_ulp + slack), "bf16 output not within half an ulp of fp64"
     err = O.rel_err(y16, ref)
-    bound = max(BF16_TOL, 2.0 ** -8 * np.max(np.abs(ref_exact)) / np.max(np.abs(ref)) + O.rel_err(ref_exact, ref)
-                + F32_TOL)
+    bound = derived_bound(ref, ref_exact) if derived else BF16_TOL
     assert err <= bound, (err, bound)
     return err
-
-
-def unfused_bound(ref, unf):
-    """check_bf16's derived bar with the unfused pipeline's bf16 intermediate in place of the bf16 fold."""
-    return max(BF16_TOL, 2.0 ** -8 * np.max(np.abs(unf)) / np.max(np.abs(ref)) + O.rel_err(unf, ref) + F32_TOL)
-
-
-def unfused_oracle(kind, bits, eps):
-    x64, g64, w64 = (O.bf16_to_f64(bits[k]) for k in ("x", "g", "w"))
-    unf = O.unfused_norm_then_project(x64, g64, w64, eps)
-    if kind == "glu":
-        F = unf.shape[1] // 2
-        unf = O.silu(unf[:, :F]) * unf[:, F:]
-    return unf
 
 
 def _exact(kind, bits, eps):
@@ -120,12 +120,14 @@ LINEAR_CASES = [
     (7, 576, 960, "decode"),     # partial last slab
     (5, 72, 136, "decode"),      # 2 k-blocks split over 2 CTAs, ragged K and N
     (16, 128, 200, "decode"),    # 2 k-blocks, 2 slabs
+    (5, 200, 12288, "decode"),   # 96 slabs: K split in two over 4 k-blocks, the last one ragged
 ]
 
 
 @pytest.mark.parametrize("M,d,N,path", LINEAR_CASES)
 def test_linear_parity(M, d, N, path):
-    bits = _wl("linear", M, d, N, seed=M * 7 + d).draw()
+    seed = M * 7 + d
+    bits = _wl("linear", M, d, N, seed=seed).draw()
     x = to_dev(bits["x"])
     ws = _fold(bits, False)
     y16 = fn.flashnorm_linear(x, ws, 1e-5, path=path)
@@ -133,7 +135,7 @@ def test_linear_parity(M, d, N, path):
     torch.cuda.synchronize()
     ref = O.reference_output("linear", bits, 1e-5)
     ref_exact = O.exact_operand_output("linear", bits, O.fold_bf16(bits["w"], bits["g"]), 1e-5)
-    check_bf16(to_host_f64(y16), ref, ref_exact)
+    check_bf16(to_host_f64(y16), ref, ref_exact, derived=("linear", M, d, N, seed) in DERIVED_BAR)
     assert O.rel_err(to_host_f64(y32), ref_exact) <= F32_TOL
 
 
@@ -151,6 +153,7 @@ GLU_CASES = [
     (1, 4096, 512, "decode"),
     (16, 576, 1536, "decode"),
     (3, 4096, 11008, "decode"),
+    (2048, 576, 4096, "pair"),   # bf16: 256 pair tiles on 74 pairs, the last 34 split into half tiles
 ]
 
 
@@ -179,7 +182,10 @@ POSTNORM_CASES = [
     (130, 256, 1024, 512),       # two 512-wide heads, ragged M
     (300, 320, 768, 384),        # two 384-wide heads: 3 slices x 2 K ranges
     (2048, 576, 512, 512),       # 16 row tiles, cluster split
-    (64, 320, 320, 320),         # 320-wide head: single-CTA 512-column path
+    (64, 320, 320, 320),         # 320-wide head: 2 x 80-column slices per column half
+    (100, 64, 512, 512),         # one k-block: no K split
+    (40, 128, 512, 512),         # two k-blocks: K split in two
+    (2048, 576, 4096, 512),      # eight 512-wide heads: 64 clusters, more than fit at once
 ]
 
 
@@ -198,6 +204,10 @@ def test_postnorm_parity(M, d, N, hd):
                                        head_dim=hd)
     check_bf16(to_host_f64(y16), ref, ref_exact)
     assert O.rel_err(to_host_f64(y32), ref_exact) <= F32_TOL
+    # the partial sums of K ranges and columns are combined in a fixed order: bitwise repeatable
+    again = fn.flashnorm_linear_postnorm(x, ws, g2, hd, 1e-6, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(again.view(torch.int32), y32.view(torch.int32))
 
 
 # ------------------------------------------------------------------------------------------ unfused baseline
@@ -215,7 +225,7 @@ def test_unfused_parity(kind, M, d, N):
     xn = fn.flashnorm_rmsnorm(x, g, 1e-5)
     torch.cuda.synchronize()
     ref = O.reference_output(kind, bits, 1e-5)
-    assert O.rel_err(to_host_f64(y), ref) <= unfused_bound(ref, unfused_oracle(kind, bits, 1e-5))
+    assert O.rel_err(to_host_f64(y), ref) <= BF16_TOL
     # the normalised intermediate itself: one bf16 rounding, at most 2^-8 of its magnitude, per element
     xn_ref = O.rmsnorm(O.bf16_to_f64(bits["x"]), O.bf16_to_f64(bits["g"]), 1e-5)
     assert np.all(np.abs(to_host_f64(xn) - xn_ref) <= 2.0 ** -8 * np.abs(xn_ref) + 1e-6 * np.max(np.abs(xn_ref)))
@@ -233,7 +243,7 @@ def test_folded_unfolded_oracle_agree_smollm2_m64():
     y_unf = to_host_f64(fn.flashnorm_linear_unfused(x, g, wk, wl.eps))
     ref = O.reference_output("linear", bits, wl.eps)
     check_bf16(y_fold, ref, _exact("linear", bits, wl.eps))
-    assert O.rel_err(y_unf, ref) <= unfused_bound(ref, unfused_oracle("linear", bits, wl.eps))
+    assert O.rel_err(y_unf, ref) <= BF16_TOL
 
 
 # ------------------------------------------------------------------------------------------ full sizes, sampled
@@ -353,7 +363,9 @@ def test_invalid_arguments_raise():
 
 @pytest.mark.parametrize("path", ["pair", "tensor"])
 @pytest.mark.parametrize("kind,M,d,N", [("linear", 2048, 576, 12288), ("glu", 2048, 576, 6144),
-                                         ("linear", 8192, 576, 960)])
+                                         ("linear", 8192, 576, 960),
+                                         # 256 pair tiles on 74 pairs: the last 34 run as 68 half tiles
+                                         ("linear", 4096, 576, 4096), ("glu", 2048, 576, 4096)])
 def test_many_tiles_per_cta_all_rows(kind, M, d, N, path):
     """Every row, with several tiles per persistent CTA, three launches. A race between the
     sum-of-squares warps' shared-memory reads and the TMA refill of the same stage once corrupted
@@ -367,6 +379,31 @@ def test_many_tiles_per_cta_all_rows(kind, M, d, N, path):
         y32 = f(x, ws, 1e-6, out_dtype=torch.float32, path=path)
         torch.cuda.synchronize()
         assert O.rel_err(to_host_f64(y32), ex) <= F32_TOL
+
+
+@pytest.mark.parametrize("path", ["pair", "tensor"])
+def test_row_block_transitions_many_launches(path):
+    """The Llama-7B QKV prefill shape (M = 2048, d = 4096, N = 12288), where several persistent CTAs'
+    tile ranges cross from one row block into the next: 40 launches back to back must give bitwise
+    identical fp32 outputs, and the first must match the oracle on every row of a sample. A parity
+    wait in the sum-of-squares warps that could be satisfied by a phase two uses back (fixed) made the
+    1/rms of a new row block read stale x tiles and left the stage barriers one arrival off."""
+    wl = I.WORKLOADS["llama7b_qkv_m2048"]
+    bits = wl.draw()
+    x = to_dev(bits["x"])
+    ws = _fold(bits, False)
+    first = fn.flashnorm_linear(x, ws, wl.eps, out_dtype=torch.float32, path=path)
+    y = torch.empty_like(first)
+    same = torch.ones((), dtype=torch.bool, device="cuda")
+    for _ in range(40):
+        fn.flashnorm_linear(x, ws, wl.eps, out_dtype=torch.float32, path=path, out=y)
+        same &= (y.view(torch.int32) == first.view(torch.int32)).all()
+    torch.cuda.synchronize()
+    fn.flashnorm_check_device_error()
+    assert bool(same.item())
+    rows = np.unique(np.concatenate([[0, wl.M - 1], np.random.default_rng(17).integers(0, wl.M, 24)]))
+    ex = O.exact_operand_output("linear", bits, O.fold_bf16(bits["w"], bits["g"]), wl.eps, rows=rows)
+    assert O.rel_err(to_host_f64(first)[rows], ex) <= F32_TOL
 
 
 @pytest.mark.parametrize("name", ["llama7b_qkv_m1", "llama7b_qkv_m4", "llama7b_qkv_m16"])
