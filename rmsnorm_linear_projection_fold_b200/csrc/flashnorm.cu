@@ -20,7 +20,6 @@
 #include "fp8.cuh"
 #include "fused_gemm_pair.cuh"
 #include "gemv.cuh"
-#include "postnorm_cluster.cuh"
 #include "postnorm_pair.cuh"
 
 namespace {
@@ -234,16 +233,20 @@ fn_status run_pair_path(const void* x, const void* w, void* y, int64_t M, int64_
   const int64_t num_n_tiles = (n_rows + bn - 1) / bn;
   const int64_t tiles = num_m_tiles * num_n_tiles;
   const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
-  // A last wave that fills at most half of the pairs is run as half tiles, one per pair.
-  int64_t num_main = tiles;
-  const int64_t rem = tiles % pairs;
-  if (tiles > pairs && rem > 0 && 2 * rem <= pairs && (bn / 2) % step == 0) num_main = tiles - rem;
+  // Pairs in groups of two sharing each W* tile (L2 reuse) when there are several waves to run and the
+  // row blocks and pairs pair up evenly.
+  const int group = (tiles > pairs && num_m_tiles % 2 == 0 && pairs % 2 == 0) ? 2 : 1;
+  const int64_t gtiles = tiles / group, groups = pairs / group;
+  // A last wave that fills at most half of the groups is run as half tiles, one per group.
+  int64_t num_main = gtiles;
+  const int64_t rem = gtiles % groups;
+  if (gtiles > groups && rem > 0 && 2 * rem <= groups && (bn / 2) % step == 0) num_main = gtiles - rem;
   CUtensorMap tx, tw, tw2;
   fn_status st = make_operand_map(&tx, x, d, M, fn::kBM);
   if (st != FN_OK) return st;
   st = make_operand_map(&tw, w, d, n_rows, bn / 2);
   if (st != FN_OK) return st;
-  st = make_operand_map(&tw2, w, d, n_rows, num_main < tiles ? bn / 4 : bn / 2);
+  st = make_operand_map(&tw2, w, d, n_rows, num_main < gtiles ? bn / 4 : bn / 2);
   if (st != FN_OK) return st;
   fn::GemmParams p;
   p.y = y;
@@ -256,6 +259,7 @@ fn_status run_pair_path(const void* x, const void* w, void* y, int64_t M, int64_
   p.head_dim = 0;
   p.num_m_tiles = static_cast<int>(num_m_tiles);
   p.num_n_tiles = static_cast<int>(num_n_tiles);
+  p.group = group;
   p.num_main = static_cast<int>(num_main);
   p.eps = eps;
   p.ln_colsum = ln_colsum;
@@ -326,61 +330,6 @@ fn_status run_tensor_path(const void* x, const void* w, void* y, const void* g2,
   if (bn <= 256) return FN_LAUNCH(256, 4, fn::EPI_POSTNORM, false);
   return FN_LAUNCH(512, 2, fn::EPI_POSTNORM, false);
 #undef FN_LAUNCH
-}
-
-// ------------------------------------------------------------------------------------------------
-// Wide-head post-norm: one cluster of (head_dim / 128) x KS CTAs per 128-row tile and head
-// (replaced by the CTA-pair kernel below; kept until that one is measured)
-// ------------------------------------------------------------------------------------------------
-
-template <bool OUT_F32>
-fn_status launch_postnorm_cluster_t(const CUtensorMap& tx, const CUtensorMap& tw, const fn::PostnormClusterParams& p,
-                                    int ctas, int dev, cudaStream_t stream) {
-  auto kern = fn::k_postnorm_cluster<OUT_F32>;
-  constexpr int smem = fn::postnorm_cluster_smem_bytes();
-  static bool configured[kMaxDevices] = {false};
-  if (!configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (post-norm cluster)");
-    configured[dev] = true;
-  }
-  cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(ctas)), dim3(fn::kPnThreads), smem, stream,
-                                static_cast<unsigned>(p.cn * p.ks), tx, tw, p);
-  if (e != cudaSuccess) return cuda_fail(e, "post-norm cluster launch");
-  return FN_OK;
-}
-
-fn_status run_postnorm_cluster(const void* x, const void* w, const void* g2, void* y, int64_t M, int64_t d, int64_t N,
-                               int64_t head_dim, float eps2, int out_dtype, cudaStream_t stream) {
-  int dev = 0;
-  const int sms = device_sm_count(&dev);
-  if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
-  fn::PostnormClusterParams p;
-  p.y = y;
-  p.g2 = static_cast<const uint16_t*>(g2);
-  p.M = static_cast<int>(M);
-  p.K = static_cast<int>(d);
-  p.N = static_cast<int>(N);
-  p.head_dim = static_cast<int>(head_dim);
-  p.num_m_tiles = static_cast<int>((M + 127) / 128);
-  p.cn = static_cast<int>(head_dim / fn::kPnCols);
-  p.eps2 = eps2;
-  const int64_t heads = N / head_dim;
-  const int64_t num_kb = (d + 63) / 64;
-  // Split K while that still adds SMs: at most 8 CTAs per cluster, about one CTA per SM.
-  int ks = 1;
-  if (p.cn * 2 <= 8 && p.num_m_tiles * heads * p.cn * 2 <= sms && num_kb >= 2) ks = 2;
-  p.ks = ks;
-  const int64_t ctas = p.num_m_tiles * heads * p.cn * ks;
-  if (ctas > INT32_MAX) return fail(FN_ERR_UNSUPPORTED, "too many tiles");
-  CUtensorMap tx, tw;
-  fn_status st = make_operand_map(&tx, x, d, M, 128);
-  if (st != FN_OK) return st;
-  st = make_operand_map(&tw, w, d, N, fn::kPnCols);
-  if (st != FN_OK) return st;
-  return out_dtype == FN_F32 ? launch_postnorm_cluster_t<true>(tx, tw, p, static_cast<int>(ctas), dev, stream)
-                             : launch_postnorm_cluster_t<false>(tx, tw, p, static_cast<int>(ctas), dev, stream);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -802,7 +751,7 @@ fn_status flashnorm_linear_postnorm_rope(const void* x, const void* Wstar, const
   fn_status st = check_common(x, Wstar, y, M, d, eps2, out_dtype);
   if (st != FN_OK) return st;
   if (head_dim < 16 || head_dim % 16 != 0) return fail(FN_ERR_INVALID_ARG, "head_dim = %lld must be a positive multiple of 16", (long long)head_dim);
-  if (head_dim > 512 || (head_dim > 256 && head_dim % fn::kPnCols == 0))
+  if (head_dim > 512 || (head_dim > 256 && head_dim % 128 == 0))
     return fail(FN_ERR_UNSUPPORTED, "RoPE is fused for heads of at most 256 (and 320) features, not %lld", (long long)head_dim);
   if (head_dim > 256 && head_dim % 32 != 0) return fail(FN_ERR_UNSUPPORTED, "head_dim in (256, 512] must be a multiple of 32");
   if (N < head_dim || N > kMaxDim || N % head_dim != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a multiple of head_dim", (long long)N);

@@ -65,7 +65,9 @@ struct GemmParams {
   // EPI_LN: fp32 [n_out] column sums of the folded W* and folded bias beta^T W
   const float* ln_colsum = nullptr;
   const float* ln_bias = nullptr;
-  // CTA-pair kernel: tiles 0 .. num_main-1 are full width, the rest are split in two halves
+  // CTA-pair kernel: pairs work in groups of `group` (1 or 2) on bands of `group` row blocks; group
+  // tiles 0 .. num_main-1 are full width, the rest are split in two halves
+  int group = 1;
   int num_main = 0;
 };
 

@@ -42,11 +42,16 @@ __host__ __device__ constexpr int gemm_pair_smem_bytes() {
 __host__ __device__ constexpr int pair_chunk_cols(bool out_f32) { return out_f32 ? 16 : 32; }
 
 // p.num_m_tiles counts 256-row pair tiles; p.bn is the pair tile width (W* rows), each CTA holding bn/2.
-// Tiles are handed to CTA pairs in contiguous ranges (row-block-major). When the tile count leaves a
-// short last wave, its tiles (the last num_tiles - p.num_main of them) are each split into two halves
-// of bn/2 columns, one half per pair: with 688 tiles on 74 pairs (Llama-7B SwiGLU, 2048 tokens) every
-// pair runs 9 full tiles and at most one half tile, 9.5 tile times instead of 10. tm_w loads the W*
-// rows of a full tile (bn/2 per CTA), tm_w2 those of a half tile (bn/4 per CTA).
+// Schedule. CTA pairs form groups of p.group (1 or 2); the pairs of a group work on the same W* column
+// tiles at the same time, each in its own row block, so that a W* tile fetched from HBM by one is found
+// in L2 by the other (W* is streamed once per group instead of once per pair: the Llama-7B SwiGLU
+// weights, 180 MB, do not fit in L2). A "group tile" is one column tile of a band of p.group row
+// blocks; groups take contiguous ranges of group tiles (band-major), so a pair stays in one row block
+// for most of its range and reads that block's x tiles for its sum of squares only once. When the
+// group tiles leave a short last wave, those past p.num_main are each split into two halves of bn/2
+// columns, one half per group: with 688 tiles on 74 pairs (Llama-7B SwiGLU, 2048 tokens) every pair
+// runs 9 full tiles and at most one half tile, 9.5 tile times instead of 10. tm_w loads the W* rows of
+// a full tile (bn/2 per CTA), tm_w2 those of a half tile (bn/4 per CTA).
 template <int STAGES, int EPI, bool SCALE, bool OUT_F32>
 __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
     k_fused_gemm_pair(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
@@ -117,26 +122,30 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
   const uint32_t tmem_base = *tmem_slot;
   grid_dep_wait();  // the previous kernel's outputs (our inputs, or buffers we overwrite) are complete
 
-  const int num_tiles = p.num_m_tiles * p.num_n_tiles;
-  const int cl = static_cast<int>(blockIdx.x) >> 1;
-  const int ncl = static_cast<int>(gridDim.x) >> 1;
-  const int t_begin = static_cast<int>(static_cast<long long>(cl) * p.num_main / ncl);
-  const int t_end = static_cast<int>(static_cast<long long>(cl + 1) * p.num_main / ncl);
-  const int num_halves = 2 * (num_tiles - p.num_main);
-  const int n_items = (t_end - t_begin) + (cl < num_halves ? 1 : 0);
+  const int G = p.group;
+  const int cl = static_cast<int>(blockIdx.x) >> 1;        // CTA pair
+  const int grp = cl / G, kg = cl % G;                    // group, and this pair's row block in the band
+  const int ngrp = (static_cast<int>(gridDim.x) >> 1) / G;
+  const int num_gtiles = (p.num_m_tiles / G) * p.num_n_tiles;
+  const int t_begin = static_cast<int>(static_cast<long long>(grp) * p.num_main / ngrp);
+  const int t_end = static_cast<int>(static_cast<long long>(grp + 1) * p.num_main / ngrp);
+  const int num_halves = 2 * (num_gtiles - p.num_main);
+  // the half tiles go to the last groups, whose ranges end nearest to them (fewer fresh row blocks)
+  const int half_id = grp - (ngrp - num_halves);
+  const int n_items = (t_end - t_begin) + (half_id >= 0 ? 1 : 0);
   const int num_kb = (p.K + kBK - 1) / kBK;
   const int bn = p.bn;
   // Item i of this pair: its row block, first W* row and width (full tiles first, then a half tile).
   auto tile_at = [&](int i, int& mt, int& n0, int& width) {
     if (i < t_end - t_begin) {
-      const int t = t_begin + i;
-      mt = t / p.num_n_tiles;
-      n0 = (t % p.num_n_tiles) * bn;
+      const int u = t_begin + i;
+      mt = (u / p.num_n_tiles) * G + kg;
+      n0 = (u % p.num_n_tiles) * bn;
       width = bn;
     } else {
-      const int t = p.num_main + (cl >> 1);
-      mt = t / p.num_n_tiles;
-      n0 = (t % p.num_n_tiles) * bn + (cl & 1) * (bn / 2);
+      const int u = p.num_main + (half_id >> 1);
+      mt = (u / p.num_n_tiles) * G + kg;
+      n0 = (u % p.num_n_tiles) * bn + (half_id & 1) * (bn / 2);
       width = bn / 2;
     }
   };
@@ -351,19 +360,27 @@ __global__ void __launch_bounds__(gemm_threads(EPI, SCALE), 1)
                                    pack_bf16x2(o[8 * jj + 4], o[8 * jj + 5]), pack_bf16x2(o[8 * jj + 6], o[8 * jj + 7])));
           }
         } else {
-          // CC output columns = CC/16 (gate 16, up 16) pairs of accumulator columns
+          // CC output columns = CC/16 (gate 16, up 16) pairs of accumulator columns, all loaded from tensor
+          // memory before one wait, so that the load latency is paid once per chunk
+          uint32_t gt[CC / 16][16], up[CC / 16][16];
 #pragma unroll
           for (int b = 0; b < CC / 16; ++b) {
-            uint32_t gt[16], up[16];
             const int acol = 2 * (ch * CC) + 32 * b;
-            tmem_ld16(t_row + acol, gt);
-            tmem_ld16(t_row + acol + 16, up);
-            tmem_ld_wait();
-            reg_fence16(gt);
-            reg_fence16(up);
+            tmem_ld16(t_row + acol, gt[b]);
+            tmem_ld16(t_row + acol + 16, up[b]);
+          }
+          tmem_ld_wait();
+#pragma unroll
+          for (int b = 0; b < CC / 16; ++b) {
+            reg_fence16(gt[b]);
+            reg_fence16(up[b]);
+          }
+#pragma unroll
+          for (int b = 0; b < CC / 16; ++b) {
             float o[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) o[j] = swiglu_deferred(__uint_as_float(gt[j]), __uint_as_float(up[j]), kr);
+            for (int j = 0; j < 16; ++j)
+              o[j] = swiglu_deferred(__uint_as_float(gt[b][j]), __uint_as_float(up[b][j]), kr);
             if (OUT_F32) {
 #pragma unroll
               for (int j = 0; j < 4; ++j)
