@@ -72,13 +72,14 @@ BENCH_WORKLOADS = {
     "llama7b_qkv_fp8_m16": ["llama7b_qkv_fp8_m16"],
     "llama7b_qkv_fp8_gemv_m1": ["llama7b_qkv_fp8_m1"],
     "llama7b_qkv_fp8_gemv_m4": ["llama7b_qkv_fp8_m4"],
+    "llama7b_qkv_fp8_tc_m1": ["llama7b_qkv_fp8_m1"],
     # the same decode projection on the CUDA-core GEMV instead of the tensor-core decode kernel
     "llama7b_qkv_gemv_m16": ["llama7b_qkv_m16"],
     "llama7b_qkv_gemv_m1": ["llama7b_qkv_m1"],
 }
 # Kernel family forced for a bench workload (default: the library's own choice, FN_PATH_AUTO).
 BENCH_PATHS = {"llama7b_qkv_gemv_m16": "gemv", "llama7b_qkv_gemv_m1": "gemv", "llama7b_qkv_fp8_gemv_m1": "gemv",
-               "llama7b_qkv_fp8_gemv_m4": "gemv"}
+               "llama7b_qkv_fp8_gemv_m4": "gemv", "llama7b_qkv_fp8_tc_m1": "decode"}
 DEFAULT_WORKLOAD = "llama7b_ffn_m2048"
 
 # DRAM traffic of the dominant kernel per launch (dram__bytes_read.sum + dram__bytes_write.sum of one
@@ -92,7 +93,8 @@ NCU_TRAFFIC = {
 # launches and this long, whatever --steps is, so that the clocks settle and samplers see the load.
 MIN_LAUNCHES = 200
 MIN_LOOP_S = 1.0
-UNFUSED_BLOCKS = 5
+UNFUSED_BLOCKS = 10
+UNFUSED_BLOCK_S = 0.1
 
 L2_BYTES = 126 * 1000 * 1000
 MAX_COPIES = 8
@@ -406,8 +408,8 @@ def run_ours(args, rank, world, device_index):
             graph = {"unavailable": f"{type(e).__name__}: {str(e)[:160]}"}
 
     # Unfused two-kernel baseline (same workload, same rotation), for what folding + deferral buy. The
-    # two arms alternate in UNFUSED_BLOCKS blocks of equal length, so that clock and power drift hit
-    # both; the reported ratio is the median of the per-block ratios.
+    # two arms alternate in UNFUSED_BLOCKS short blocks of equal length (about UNFUSED_BLOCK_S each), so
+    # that clock and power drift hit both alike; the reported ratio is the median of the per-block ratios.
     unfused = None
     if do_unfused:
         def unf_body(i):
@@ -417,7 +419,7 @@ def run_ours(args, rank, world, device_index):
         for i in range(args.warmup):
             unf_body(i)
         torch.cuda.synchronize()
-        n_blk = loop_count(ms_per_step, min_s=MIN_LOOP_S / 2)
+        n_blk = loop_count(ms_per_step, min_s=UNFUSED_BLOCK_S, min_launches=20)
         fused_ms, unf_ms = [], []
         for _ in range(UNFUSED_BLOCKS):
             f_ms, _ = _time_back_to_back(torch, n_blk, step)

@@ -202,11 +202,10 @@ FN_API fn_status flashnorm_layernorm_linear(const void* x, const void* Wstar, co
  *   the bytes of bf16 W*: y = (x . dec(Q)^T) * scales * 1/sqrt(mean(x^2) + eps). x bf16 [M, d];
  *   y [M, N] of out_dtype. Larger M returns FN_ERR_UNSUPPORTED. Runs flashnorm_linear_fp8_ex with
  *   FN_PATH_AUTO.
- * flashnorm_linear_fp8_ex: the same with a kernel choice. FN_PATH_AUTO or FN_PATH_DECODE: the tensor-core
- *   kernel (Q widened on chip, exactly, to f16; x given to the MMA as f16 after a per-token power-of-two
- *   scale that makes every bf16 value of the token down to 2^-29 of its largest an exact f16, undone in
- *   the epilogue; fp32 accumulation). FN_PATH_GEMV: the CUDA-core GEMV (x staged in shared memory, each
- *   16-byte load carries 16 weights). Other paths return FN_ERR_INVALID_ARG.
+ * flashnorm_linear_fp8_ex: the same with a kernel choice. FN_PATH_DECODE: the tensor-core kernel (Q widened
+ *   on chip, exactly, to bf16 in tensor memory; x as it is; fp32 accumulation). FN_PATH_GEMV: the
+ *   CUDA-core GEMV (x staged in shared memory, each 16-byte load carries 16 weights). FN_PATH_AUTO: the
+ *   GEMV for one token, the tensor-core kernel for more. Other paths return FN_ERR_INVALID_ARG.
  */
 FN_API fn_status flashnorm_fold_weights_fp8(const void* W, const void* g, void* Q, void* scales, int64_t d, int64_t N,
                                             void* stream);

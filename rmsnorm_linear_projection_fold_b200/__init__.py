@@ -267,7 +267,8 @@ def flashnorm_linear_fp8(x: torch.Tensor, Q: torch.Tensor, scales: torch.Tensor,
                          out_dtype=torch.bfloat16, out=None, path: str = "auto") -> torch.Tensor:
     """Decode (M <= 16) with FP8 weights: y = (x . dec(Q)^T) * scales * 1/sqrt(mean(x^2) + eps).
 
-    path "auto" / "decode": the tensor-core kernel; "gemv": the CUDA-core GEMV."""
+    path "decode": the tensor-core kernel; "gemv": the CUDA-core GEMV; "auto": the GEMV for one token, the
+    tensor-core kernel for more."""
     _need(x, "x", dim=2)
     _need(Q, "Q", torch.uint8, dim=2)
     _need(scales, "scales", torch.float32, dim=1)

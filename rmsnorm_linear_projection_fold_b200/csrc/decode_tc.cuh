@@ -27,6 +27,10 @@ constexpr int kDecWStage = kDecRows * 64 * 2;  // 16 KB
 constexpr int kDecXStage = kDecTok * 64 * 2;   // 2 KB
 constexpr int kDecThreads = 192;
 constexpr int kDecMaxSplit = 4;
+// Independent accumulators: the MMAs of a k-block go to four 16-column accumulators in turn, summed in
+// the epilogue in a fixed order. MMAs of N = 16 into one accumulator form a dependent chain that runs
+// at about one per 150 cycles; four chains overlap in the tensor pipe.
+constexpr int kDecAccs = 4;
 
 struct DecodeParams {
   void* y;
@@ -87,7 +91,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     tma_prefetch_desc(&tm_x);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 32);
+    tmem_alloc(tmem_slot, 64);
     tmem_relinquish();
   }
   tc_fence_before_sync();
@@ -157,9 +161,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const uint32_t a_addr = smem_u32(sW + s * kDecWStage);
         const uint32_t b_addr = smem_u32(sX + s * kDecXStage);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          tc_mma_bf16(tmem_base, make_sdesc_sw128(a_addr + k * 32), make_sdesc_sw128(b_addr + k * 32), idesc,
-                      (kb != kb0 || k != 0) ? 1u : 0u);
+        for (int k = 0; k < 4; ++k)  // MMA k of every k-block into accumulator k
+          tc_mma_bf16(tmem_base + static_cast<uint32_t>(k * kDecTok), make_sdesc_sw128(a_addr + k * 32),
+                      make_sdesc_sw128(b_addr + k * 32), idesc, kb != kb0 ? 1u : 0u);
         tc_commit(&empty[s]);
         if (++s == STAGES) {
           s = 0;
@@ -221,12 +225,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (ok && have_acc) ok = mbar_wait(acc_full, 0, abort_flag);
     if (have_acc && ok) {
       tc_fence_after_sync();
-      uint32_t r[16];
-      tmem_ld16(tmem_base + (static_cast<uint32_t>(q * 32) << 16), r);
+      uint32_t r0[16], r1[16], r2[16], r3[16];
+      const uint32_t lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      tmem_ld16(lanes, r0);
+      tmem_ld16(lanes + kDecTok, r1);
+      tmem_ld16(lanes + 2 * kDecTok, r2);
+      tmem_ld16(lanes + 3 * kDecTok, r3);
       tmem_ld_wait();
-      reg_fence16(r);
+      reg_fence16(r0);
+      reg_fence16(r1);
+      reg_fence16(r2);
+      reg_fence16(r3);
 #pragma unroll
-      for (int j = 0; j < kDecTok; ++j) v[j] = __uint_as_float(r[j]);
+      for (int j = 0; j < kDecTok; ++j)
+        v[j] = (__uint_as_float(r0[j]) + __uint_as_float(r1[j])) + (__uint_as_float(r2[j]) + __uint_as_float(r3[j]));
     } else {
       // an empty K range (more CTAs than k-blocks) contributes zero; a failed wait contributes NaN
 #pragma unroll
@@ -295,7 +307,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  if (warp == 1) tmem_dealloc(tmem_base, 32);
+  if (warp == 1) tmem_dealloc(tmem_base, 64);
 }
 
 }  // namespace fn

@@ -518,18 +518,19 @@ fn_status launch_gemv_fp8_t(const void* x, const void* q, const void* scales, vo
 // FP8 decode on the tensor cores
 // ------------------------------------------------------------------------------------------------
 
-template <int KSPLIT, bool OUT_F32>
-fn_status launch_decode_fp8_t(const CUtensorMap& tq, const fn::DecodeFp8Params& p, int slabs, int smem, int dev,
-                              cudaStream_t stream) {
-  auto kern = fn::k_decode_fp8<KSPLIT, OUT_F32>;
-  static int configured[kMaxDevices] = {0};
-  if (configured[dev] < smem) {
+template <int STAGES, int KSPLIT, bool OUT_F32>
+fn_status launch_decode_fp8_t(const CUtensorMap& tq, const CUtensorMap& tx, const fn::DecodeFp8Params& p, int slabs,
+                              int dev, cudaStream_t stream) {
+  auto kern = fn::k_decode_fp8<STAGES, KSPLIT, OUT_F32>;
+  constexpr int smem = fn::decode_fp8_smem_bytes<STAGES, KSPLIT>();
+  static bool configured[kMaxDevices] = {false};
+  if (!configured[dev]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (fp8 decode)");
-    configured[dev] = smem;
+    configured[dev] = true;
   }
-  cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(slabs * KSPLIT)), dim3(fn::kD8Threads),
-                                static_cast<size_t>(smem), stream, KSPLIT, tq, p);
+  cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(slabs * KSPLIT)), dim3(fn::kD8Threads), smem, stream,
+                                KSPLIT, tq, tx, p);
   if (e != cudaSuccess) return cuda_fail(e, "fp8 decode launch");
   return FN_OK;
 }
@@ -541,46 +542,33 @@ fn_status run_decode_fp8(const void* x, const void* q, const void* scales, void*
   if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
   const int64_t slabs = (N + fn::kD8Rows - 1) / fn::kD8Rows;
   const int64_t units = (d + fn::kD8KStage - 1) / fn::kD8KStage;
-  // K split: the one that leaves the least W* to the busiest SM (ceil(CTAs / SMs) CTAs of 1/ks slab each),
-  // among those whose CTA fits in shared memory; among equals the smaller split (fewer partial sums).
-  // Llama-7B QKV (96 slabs): in three, 288 CTAs of 112 KB, two on every SM.
-  int best = 0;
-  double best_load = 1e30;
-  for (int ks = 1; ks <= 4 && ks <= units; ++ks) {
-    if (fn::decode_fp8_smem_bytes(static_cast<int>((units + ks - 1) / ks), ks) > 227 * 1024) continue;
-    const double load = static_cast<double>((slabs * ks + sms - 1) / sms) / ks;
-    if (load < best_load - 1e-9) {
-      best_load = load;
-      best = ks;
-    }
-  }
-  if (best == 0) return fail(FN_ERR_UNSUPPORTED, "fp8 decode: d = %lld leaves no K split that fits in shared memory",
-                             (long long)d);
-  const int smem = fn::decode_fp8_smem_bytes(static_cast<int>((units + best - 1) / best), best);
-  CUtensorMap tq;
+  // K split as for the bf16 decode kernel: in two while there are at most as many slabs as SMs (two
+  // 5-stage CTAs fit one SM), in four when there are few slabs; otherwise one 10-stage CTA per slab.
+  int ksplit = 1;
+  if (slabs <= sms && units >= 2) ksplit = 2;
+  if (slabs * 4 <= sms && units >= 4) ksplit = 4;
+  CUtensorMap tq, tx;
   fn_status st = make_u8_map(&tq, q, d, N, fn::kD8Rows);
+  if (st != FN_OK) return st;
+  st = make_operand_map(&tx, x, d, M, fn::kD8Tok);
   if (st != FN_OK) return st;
   fn::DecodeFp8Params p;
   p.y = y;
-  p.x = static_cast<const uint16_t*>(x);
   p.scales = static_cast<const float*>(scales);
   p.M = static_cast<int>(M);
   p.K = static_cast<int>(d);
   p.N = static_cast<int>(N);
   p.ldy = static_cast<int>(N);
-  p.ksplit = best;
+  p.ksplit = ksplit;
   p.eps = eps;
   const int sl = static_cast<int>(slabs);
   const bool f32 = out_dtype == FN_F32;
-#define FN_D8(KS)                                                                                              \
-  (f32 ? launch_decode_fp8_t<KS, true>(tq, p, sl, smem, dev, stream)                                           \
-       : launch_decode_fp8_t<KS, false>(tq, p, sl, smem, dev, stream))
-  switch (best) {
-    case 1: return FN_D8(1);
-    case 2: return FN_D8(2);
-    case 3: return FN_D8(3);
-    default: return FN_D8(4);
-  }
+#define FN_D8(ST, KS)                                                                                          \
+  (f32 ? launch_decode_fp8_t<ST, KS, true>(tq, tx, p, sl, dev, stream)                                         \
+       : launch_decode_fp8_t<ST, KS, false>(tq, tx, p, sl, dev, stream))
+  if (ksplit == 1) return FN_D8(10, 1);
+  if (ksplit == 2) return FN_D8(5, 2);
+  return FN_D8(4, 4);
 #undef FN_D8
 }
 
@@ -841,7 +829,10 @@ fn_status flashnorm_linear_fp8_ex(const void* x, const void* Q, const void* scal
   if (M > FN_DECODE_MAX_M) return fail(FN_ERR_UNSUPPORTED, "the fp8 path is the decode GEMV: M <= %d", FN_DECODE_MAX_M);
   if ((st = check_ptr(scales, "scales")) != FN_OK) return st;
   if (M == 0) return FN_OK;
-  if (path != FN_PATH_GEMV)
+  // AUTO: one token on the CUDA-core GEMV (16.2 us for the Llama-7B QKV codes against 18.0 us on the
+  // tensor cores), more on the tensor-core kernel, whose time does not grow with M (the GEMV's does: 29 us
+  // at 4 tokens, 125 us at 16).
+  if (path == FN_PATH_DECODE || (path == FN_PATH_AUTO && M > 1))
     return run_decode_fp8(x, Q, scales, y, M, d, N, eps, out_dtype, static_cast<cudaStream_t>(stream));
   if (!gemv_fits(M, d)) return fail(FN_ERR_UNSUPPORTED, "x [%lld, %lld] does not fit in shared memory", (long long)M, (long long)d);
   int dev = 0;

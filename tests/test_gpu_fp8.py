@@ -82,3 +82,26 @@ def test_linear_fp8_token_scales_cover_a_wide_range():
     got = to_host_f64(y32)
     for m in range(6):  # row by row: the rows' scales differ by many decades
         assert O.rel_err(got[m], ex[m]) <= F32_TOL, m
+
+
+@pytest.mark.parametrize("path", ["decode", "gemv"])
+def test_linear_fp8_subnormal_codes(path):
+    """Every channel: one weight at the channel's maximum (code 448) and all others in E4M3's subnormal range
+    (|W*| / s below 2^-6). The subnormal codes carry about 1e-3 of each output, so a widening that flushed
+    them to zero would miss the fp32 bar by two orders of magnitude."""
+    M, d, N = 3, 1024, 256
+    bits = I.Workload("t", "linear_fp8", M, d, N, 1e-6, seed=31).draw()
+    rng = np.random.default_rng(8)
+    g = O.bf16_to_f64(bits["g"])
+    mag = rng.uniform(0.2, 0.9, size=(d, N)) * 2.0 ** -6 / 448.0
+    w = np.where(rng.random((d, N)) < 0.5, -mag, mag) / g[:, None]
+    k0 = rng.integers(0, d, size=N)
+    w[k0, np.arange(N)] = 1.0 / g[k0]
+    bits = dict(bits, w=I.f32_to_bf16_bits(w.astype(np.float32)))
+    codes, _ = O.fold_fp8(bits["w"], bits["g"])
+    assert np.mean((codes & 0x78) == 0) > 0.9  # exponent field zero: subnormal (or zero) codes
+    Q, s = fn.flashnorm_fold_weights_fp8(to_dev(bits["w"]), to_dev(bits["g"]))
+    y32 = fn.flashnorm_linear_fp8(to_dev(bits["x"]), Q, s, 1e-6, out_dtype=torch.float32, path=path)
+    torch.cuda.synchronize()
+    ex = O.exact_operand_fp8(bits, 1e-6)
+    assert O.rel_err(to_host_f64(y32), ex) <= F32_TOL
