@@ -87,6 +87,8 @@ DEFAULT_WORKLOAD = "llama7b_ffn_m2048"
 # hash differently now, traffic is reported as null.
 NCU_TRAFFIC = {
     # workload: (bytes per launch, sha256[:16] of the csrc/*.cu* sources at capture time)
+    "llama7b_ffn_m2048": (826738688, "bc8a4ae62a0459dd"),
+    "llama7b_qkv_fp8_m4": (50473984, "bc8a4ae62a0459dd"),
 }
 
 # The dominant-kernel loop and each block of the fused/unfused comparison run at least this many

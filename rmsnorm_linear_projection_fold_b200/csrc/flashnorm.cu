@@ -339,8 +339,8 @@ fn_status run_tensor_path(const void* x, const void* w, void* y, const void* g2,
 // Clusters of `csize` CTAs of the wide-head kernel that can be resident at once on this device.
 template <bool OUT_F32>
 int postnorm_pair_max_clusters(int csize, int dev) {
-  static int cache[kMaxDevices][3] = {{0}};
-  const int slot = csize == 16 ? 2 : csize == 8 ? 1 : 0;
+  static int cache[kMaxDevices][fn::kPpMaxKS + 1] = {{0}};
+  const int slot = csize / (2 * fn::kPpNP);  // K ranges per cluster
   if (cache[dev][slot] == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(csize));
@@ -391,12 +391,13 @@ fn_status run_postnorm_pair_t(const void* x, const void* w, const void* g2, void
   const int64_t num_kb = (d + 63) / 64;
   const int64_t nw = head_dim / 2;
   // K ranges per cluster: the split with the fewest (waves x k-blocks per range + a fixed cost of about
-  // six k-blocks for the pipeline fill, the reduce-scatter and the stores), among those whose column
-  // slices are whole 16-column chunks and whose K ranges are not empty.
+  // six k-blocks for the pipeline fill, the reduce-scatter and the stores), among those whose K ranges
+  // are not empty and whose slices are at least one 16-column chunk wide. Clusters of 12 (KS = 3) and 16
+  // are non-portable sizes; on a B200 at most 7 clusters of 16 are resident at once.
   int best_ks = 0;
   int64_t best_cost = INT64_MAX;
-  for (int ks = fn::kPpMaxKS; ks >= 1; ks /= 2) {
-    if ((nw / ks) % 16 != 0 || ks > num_kb) continue;
+  for (int ks = fn::kPpMaxKS; ks >= 1; --ks) {
+    if (nw / ks < 16 || ks > num_kb) continue;
     const int maxc = postnorm_pair_max_clusters<OUT_F32>(2 * fn::kPpNP * ks, dev);
     if (maxc <= 0) continue;
     const int64_t waves = (clusters + maxc - 1) / maxc;
@@ -602,8 +603,8 @@ fn_status run_decode_tc(const void* x, const void* w, void* y, int64_t M, int64_
   const int64_t num_kb = (d + 63) / 64;
   // Split K across a cluster so that more SMs stream W*: in two while there are at most as many slabs as
   // SMs (two 5-stage CTAs fit one SM), in four when there are few slabs. Llama-7B QKV (96 slabs): 22.7 ->
-  // 19-21 us with the split in two; in four, 25.5 us.
-  // (A split in three, 288 four-stage CTAs two to an SM, measured 27.0 us against 20.6 us in two.)
+  // 20.5 us with the split in two; in four, 25.6 us. (In three, 288 four-stage CTAs two to an SM:
+  // 27.0 us. In two with six stages, the partial sums moved into the idle W* stages: 21.8 us.)
   int ksplit = 1;
   if (slabs <= sms && num_kb >= 2) ksplit = 2;
   if (slabs * 4 <= sms && num_kb >= 4) ksplit = 4;

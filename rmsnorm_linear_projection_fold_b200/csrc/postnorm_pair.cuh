@@ -10,12 +10,13 @@
 //     x and half of the pair's W* rows, so each SM moves 32 KB per 64-deep k-block for a 128 x 256
 //     block of the product (twice the work per byte of a 1-CTA 128 x 128 tile);
 //   * NP = 2 column halves of the head, one pair each (MMA N = head_dim / 2);
-//   * KS = 1, 2 or 4 ranges of the contraction dimension d, one pair each.
+//   * KS = 1 to 4 ranges of the contraction dimension d, one pair each.
 // After the contraction the KS pairs of a column half hold partial sums of the same 256 x hd/2 block.
 // They reduce-scatter it through distributed shared memory: the block's columns are cut into KS
-// slices of w = hd / (2 KS), every CTA sends the slices it does not own into the (by then idle)
-// pipeline buffers of their owners and adds the ones it receives to its own slice, in a fixed order
-// of K ranges (deterministic). Each CTA then holds the complete u for 128 rows x w columns; the
+// slices of whole 16-column chunks (hd / (2 KS) wide, or nearly), every CTA sends the slices it does not
+// own into the (by then idle) pipeline buffers of their owners and adds the ones it receives to its own
+// slice, in a fixed order of K ranges (deterministic). Each CTA then holds the complete u for 128 rows
+// x its slice's columns; the
 // per-row sums of squares over those columns go to every CTA of the cluster that holds the same rows,
 // and each CTA scales and stores its own slice. No partial result goes through global memory.
 //
@@ -40,7 +41,7 @@ struct PostnormPairParams {
   const uint16_t* g2;  // bf16 [head_dim]
   int M, K, N, head_dim;
   int num_m_tiles;     // 256-row tiles
-  int ks;              // K ranges per cluster (1, 2 or 4); cluster = 2 * kPpNP * ks CTAs
+  int ks;              // K ranges per cluster (1 to kPpMaxKS); cluster = 2 * kPpNP * ks CTAs
   float eps2;
 };
 
@@ -49,9 +50,13 @@ __host__ __device__ constexpr int postnorm_pair_smem_bytes() {
          kPpMaxHead * 4 /* g2 */ + 512 /* barriers */;
 }
 
-// Row stride (floats) of a received slice: w plus one 16-byte pad, so that eight consecutive rows
-// written with 16-byte stores land in distinct bank groups.
+// Row stride (floats) of a received slice: its width plus one 16-byte pad, so that eight consecutive
+// rows written with 16-byte stores land in distinct bank groups.
 __host__ __device__ constexpr int pp_slice_stride(int w) { return w + 4; }
+
+// First column of slice k of nw columns cut into ks slices of whole 16-column chunks (the last takes
+// the remainder: 256 in three is 80, 80, 96).
+__host__ __device__ constexpr int pp_slice_begin(int k, int nw, int ks) { return k >= ks ? nw : (k * nw / ks) / 16 * 16; }
 
 template <bool OUT_F32>
 __global__ void __launch_bounds__(kPpThreads, 1)
@@ -88,8 +93,12 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   const int hd = p.head_dim;
   const int nw = hd / 2;          // MMA N: the pair's columns
   const int brows = hd / 4;       // W* rows this CTA stages
-  const int w = nw / KS;          // columns of the slice this CTA finishes
-  const int sstr = pp_slice_stride(w);
+  // the slice of the pair's columns this CTA finishes, and the widest slice (the receive slots' width)
+  const int c_own = pp_slice_begin(ks, nw, KS);
+  const int w = pp_slice_begin(ks + 1, nw, KS) - c_own;
+  int w_max = 0;
+  for (int k = 0; k < KS; ++k) w_max = max(w_max, pp_slice_begin(k + 1, nw, KS) - pp_slice_begin(k, nw, KS));
+  const int sstr = pp_slice_stride(w_max);
   const int m0 = mt * 256 + half * 128;
   const int col_pair = head * hd + np * nw;  // first output column / W* row of the pair
   const int num_kb = (p.K + 63) / 64;
@@ -247,9 +256,11 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       const int slot = ks < dst_ks ? ks : ks - 1;
       const uint32_t dst_rank = static_cast<uint32_t>((dst_ks * kPpNP + np) * 2 + half);
       const uint32_t dst = dsmem_addr(recv + (slot * 128 + row) * sstr, dst_rank);
-      for (int ch = h2; ch < nchunks; ch += 2) {
+      const int c_dst = pp_slice_begin(dst_ks, nw, KS);
+      const int n_dst = (pp_slice_begin(dst_ks + 1, nw, KS) - c_dst) / 16;
+      for (int ch = h2; ch < n_dst; ch += 2) {
         float u[16];
-        load_acc(dst_ks * w + ch * 16, u);
+        load_acc(c_dst + ch * 16, u);
 #pragma unroll
         for (int j = 0; j < 16; j += 4)
           dsmem_st_v4(dst + static_cast<uint32_t>((ch * 16 + j) * 4), u[j], u[j + 1], u[j + 2], u[j + 3]);
@@ -266,7 +277,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     for (int k = 0; k < KS; ++k) {
       float part[16];
       if (k == ks) {
-        load_acc(ks * w + ch * 16, part);
+        load_acc(c_own + ch * 16, part);
       } else {
         const int slot = k < ks ? k : k - 1;
         const float4* src = reinterpret_cast<const float4*>(recv + (slot * 128 + row) * sstr + ch * 16);
@@ -306,7 +317,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     for (int ch = h2; ch < nchunks; ch += 2) {
       float u[16];
       slice_u(ch, u);
-      const int lc = np * nw + ks * w + ch * 16;  // column within the head
+      const int lc = np * nw + c_own + ch * 16;  // column within the head
       float o[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) o[j] = u[j] * r2 * g2s[lc + j];
