@@ -16,9 +16,9 @@
 // slices of whole 16-column chunks (hd / (2 KS) wide, or nearly), every CTA sends the slices it does not
 // own into the (by then idle) pipeline buffers of their owners and adds the ones it receives to its own
 // slice, in a fixed order of K ranges (deterministic). Each CTA then holds the complete u for 128 rows
-// x its slice's columns; the
-// per-row sums of squares over those columns go to every CTA of the cluster that holds the same rows,
-// and each CTA scales and stores its own slice. No partial result goes through global memory.
+// x its slice's columns; the per-row sums of squares over those columns go to every CTA of the cluster
+// that holds the same rows, and each CTA scales and stores its own slice. No partial result goes
+// through global memory.
 //
 // Warps: 0 = TMA producer, 1 = TMEM allocator + pair MMA issuer (leader CTA of the pair),
 // 2..9 = epilogue (two warps per tensor-memory lane quarter, splitting a slice's columns).
