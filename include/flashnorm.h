@@ -146,6 +146,34 @@ FN_API fn_status flashnorm_linear_postnorm(const void* x, const void* Wstar, con
                                     void* stream);
 
 /*
+ * flashnorm_linear_postnorm_ws — flashnorm_linear_postnorm with a caller-provided workspace. The same
+ * result (same definition, same tolerances); what changes is how a wide head (256 < head_dim <= 512)
+ * is scheduled when it has few 256-row tiles. Without a workspace, each tile's whole contraction runs in
+ * one thread-block cluster that keeps its partial sums on chip (few such clusters are resident, so
+ * 2048 rows of one 512-wide head occupy 64 SMs). With one, the contraction dimension d is split over
+ * independent CTA pairs that fill the device, each writing an fp32 partial product to the workspace,
+ * and a second kernel adds the partials in a fixed order (deterministic) and applies the norm.
+ *   workspace        device memory, 16-byte aligned, caller-owned, or NULL (no split). Its contents
+ *                    are scratch: overwritten by the call and read by its second kernel, so calls whose
+ *                    kernels overlap on the GPU (different streams, host threads) must not share one.
+ *   workspace_bytes  its size. A non-NULL workspace smaller than flashnorm_postnorm_workspace_bytes
+ *                    reports for this shape returns FN_ERR_INVALID_ARG and launches nothing.
+ * Shapes for which the split does not apply (head_dim <= 256, or enough row tiles to fill the device
+ * without it: the size query returns 0) ignore the workspace.
+ */
+FN_API fn_status flashnorm_linear_postnorm_ws(const void* x, const void* Wstar, const void* g2, void* y, int64_t M,
+                                              int64_t d, int64_t N, int64_t head_dim, float eps2, int out_dtype,
+                                              void* workspace, int64_t workspace_bytes, void* stream);
+
+/*
+ * flashnorm_postnorm_workspace_bytes — the workspace flashnorm_linear_postnorm_ws uses for this shape on
+ * the current device, written to *bytes: K ranges x M x N x 4 (fp32 partial products), or 0 where the
+ * split does not apply. FN_ERR_INVALID_ARG for a shape flashnorm_linear_postnorm rejects as invalid.
+ */
+FN_API fn_status flashnorm_postnorm_workspace_bytes(int64_t M, int64_t d, int64_t N, int64_t head_dim,
+                                                    int64_t* bytes);
+
+/*
  * flashnorm_linear_postnorm_rope — flashnorm_linear_postnorm followed, in the same epilogue, by rotary
  * position embedding of the normalised query/key heads. The FlashNorm Abstract lists RoPE-based
  * attention among the cases the technique extends to, and the paper builds on RoFormer; the rotation is

@@ -29,6 +29,7 @@ __all__ = [
     "flashnorm_linear",
     "flashnorm_glu",
     "flashnorm_linear_postnorm",
+    "flashnorm_postnorm_workspace_bytes",
     "flashnorm_linear_postnorm_rope",
     "flashnorm_rope_table",
     "flashnorm_fold_layernorm",
@@ -68,6 +69,8 @@ _SIGNATURES = {
     "flashnorm_glu": [_P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_glu_ex": [_P, _P, _P, _I64, _I64, _I64, _F, _INT, _INT, _P],
     "flashnorm_linear_postnorm": [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _F, _INT, _P],
+    "flashnorm_linear_postnorm_ws": [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _F, _INT, _P, _I64, _P],
+    "flashnorm_postnorm_workspace_bytes": [_I64, _I64, _I64, _I64, _P],
     "flashnorm_linear_postnorm_rope": [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_rope_table": [_P, _I64, _I64, ctypes.c_double, _P],
     "flashnorm_fold_layernorm": [_P, _P, _P, _P, _P, _P, _I64, _I64, _P],
@@ -136,8 +139,11 @@ def _same_device(lead: torch.Tensor, **others) -> None:
 def _invoke(entry: str, lead: torch.Tensor, *args, report: str | None = None) -> None:
     """Call the library's `entry` with `lead`'s device current: the library launches on, and looks up
     its per-device state for, the current device."""
+    _invoke_on(lead.device.index, entry, *args, report=report)
+
+
+def _invoke_on(dev: int, entry: str, *args, report: str | None = None) -> None:
     lib = load_library()
-    dev = lead.device.index
     if dev == torch.cuda.current_device():
         status = getattr(lib, entry)(*args)
     else:
@@ -230,9 +236,25 @@ def flashnorm_glu(x: torch.Tensor, Wstar_gu: torch.Tensor, eps: float, out_dtype
     return y
 
 
+def flashnorm_postnorm_workspace_bytes(M: int, d: int, N: int, head_dim: int, device=None) -> int:
+    """Workspace bytes flashnorm_linear_postnorm uses for this shape on `device` (0: no split)."""
+    dev = torch.cuda.current_device() if device is None else torch.device(device).index
+    if dev is None:
+        dev = torch.cuda.current_device()
+    nbytes = ctypes.c_int64(0)
+    _invoke_on(dev, "flashnorm_postnorm_workspace_bytes", int(M), int(d), int(N), int(head_dim),
+               ctypes.c_void_p(ctypes.addressof(nbytes)))
+    return int(nbytes.value)
+
+
 def flashnorm_linear_postnorm(x: torch.Tensor, Wstar: torch.Tensor, g2: torch.Tensor, head_dim: int, eps2: float,
-                              out_dtype=torch.bfloat16, out=None) -> torch.Tensor:
-    """Per-head RMSNorm(x . W*; g2, eps2) with the first RMSNorm elided (its gain folded into W*)."""
+                              out_dtype=torch.bfloat16, out=None, workspace="auto") -> torch.Tensor:
+    """Per-head RMSNorm(x . W*; g2, eps2) with the first RMSNorm elided (its gain folded into W*).
+
+    workspace: "auto" allocates the scratch that lets a wide head (256 < head_dim <= 512) with few row
+    tiles split its contraction over the whole device (flashnorm_postnorm_workspace_bytes; nothing for
+    other shapes); None runs without one (a wide head then stays in one thread-block cluster per row tile);
+    or a caller-owned uint8 CUDA tensor of at least that many bytes."""
     _need(x, "x", dim=2)
     _need(Wstar, "Wstar", dim=2)
     _need(g2, "g2", dim=1)
@@ -244,8 +266,20 @@ def flashnorm_linear_postnorm(x: torch.Tensor, Wstar: torch.Tensor, g2: torch.Te
         raise ValueError("g2 must have head_dim elements")
     _same_device(x, Wstar=Wstar, g2=g2)
     y = _output(out, (M, N), out_dtype, x)
-    _invoke("flashnorm_linear_postnorm", x, _ptr(x), _ptr(Wstar), _ptr(g2), _ptr(y), M, d, N, int(head_dim),
-            float(eps2), _out_code(out_dtype), _stream_ptr(x))
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError('workspace must be "auto", None or a uint8 CUDA tensor')
+        nbytes = flashnorm_postnorm_workspace_bytes(M, d, N, head_dim, x.device) if M > 0 else 0
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=x.device) if nbytes > 0 else None
+    elif workspace is None:
+        ws = None
+    else:
+        _need(workspace, "workspace", torch.uint8, dim=1)
+        _same_device(x, workspace=workspace)
+        ws = workspace
+    _invoke("flashnorm_linear_postnorm_ws", x, _ptr(x), _ptr(Wstar), _ptr(g2), _ptr(y), M, d, N, int(head_dim),
+            float(eps2), _out_code(out_dtype), _ptr(ws), ws.numel() if ws is not None else 0, _stream_ptr(x),
+            report="flashnorm_linear_postnorm")
     return y
 
 

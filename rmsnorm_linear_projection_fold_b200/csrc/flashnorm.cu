@@ -21,6 +21,7 @@
 #include "fused_gemm_pair.cuh"
 #include "gemv.cuh"
 #include "postnorm_pair.cuh"
+#include "postnorm_split.cuh"
 
 namespace {
 
@@ -126,6 +127,21 @@ fn_status make_u8_map(CUtensorMap* map, const void* ptr, int64_t k, int64_t rows
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  return FN_OK;
+}
+
+// 3-D fp32 [planes][rows][cols] (the split post-norm's partial products) with a 32-column x 128-row box
+// and 128-byte swizzle, for TMA stores.
+fn_status make_partial_map(CUtensorMap* map, void* ptr, int64_t cols, int64_t rows, int64_t planes) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 4, static_cast<cuuint64_t>(cols * rows) * 4};
+  cuuint32_t box[3] = {32u, 128u, 1u};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
   return FN_OK;
 }
@@ -429,6 +445,108 @@ fn_status run_postnorm_pair(const void* x, const void* w, const void* g2, void* 
 }
 
 // ------------------------------------------------------------------------------------------------
+// Wide-head post-norm with the contraction split over independent CTA pairs (workspace) + finalize
+// ------------------------------------------------------------------------------------------------
+
+// CTA pairs of the split GEMM that can be resident at once on this device.
+int postnorm_split_max_pairs(int dev) {
+  static int cache[kMaxDevices] = {0};
+  if (cache[dev] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(fn::k_postnorm_split_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         fn::postnorm_split_smem_bytes());
+    int n = 0;
+    if (e == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2);
+      cfg.blockDim = dim3(fn::kPsThreads);
+      cfg.dynamicSmemBytes = fn::postnorm_split_smem_bytes();
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 2;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      e = cudaOccupancyMaxActiveClusters(&n, fn::k_postnorm_split_gemm, &cfg);
+    }
+    if (e != cudaSuccess || n < 0) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    cache[dev] = n > 0 ? n : -1;
+  }
+  return cache[dev];
+}
+
+// K ranges of the split kernel for this shape: as many as keep all CTA pairs in one wave (at most
+// kPsMaxKS, each range at least four 64-deep k-blocks). 0 where fewer than two fit: there the cluster
+// kernel, which keeps its partial sums on chip, has enough row tiles to fill the device by itself. Also 0
+// for heads that are not a multiple of 64 wide (the cluster kernel takes those).
+int postnorm_split_ks(int64_t M, int64_t d, int64_t N, int64_t head_dim) {
+  // the partial product leaves in 32-column boxes: each pair's head_dim / 2 columns must fill whole boxes
+  if (head_dim <= 256 || head_dim % 64 != 0 || M <= 0) return 0;
+  int dev = 0;
+  if (device_sm_count(&dev) <= 0) return 0;
+  const int max_pairs = postnorm_split_max_pairs(dev);
+  if (max_pairs <= 0) return 0;
+  const int64_t pairs_per_range = ((M + 255) / 256) * (N / head_dim) * 2;
+  const int64_t num_kb = (d + 63) / 64;
+  int64_t ks = max_pairs / pairs_per_range;
+  if (ks > fn::kPsMaxKS) ks = fn::kPsMaxKS;
+  while (ks > 1 && num_kb < 4 * ks) --ks;
+  return ks >= 2 ? static_cast<int>(ks) : 0;
+}
+
+fn_status run_postnorm_split(const void* x, const void* w, const void* g2, void* y, int64_t M, int64_t d, int64_t N,
+                             int64_t head_dim, float eps2, int out_dtype, int ks, void* ws, cudaStream_t stream) {
+  int dev = 0;
+  const int sms = device_sm_count(&dev);
+  if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
+  fn::PostnormSplitParams p;
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(d);
+  p.N = static_cast<int>(N);
+  p.head_dim = static_cast<int>(head_dim);
+  p.num_m_tiles = static_cast<int>((M + 255) / 256);
+  p.heads = static_cast<int>(N / head_dim);
+  p.ks = ks;
+  const int64_t ctas = static_cast<int64_t>(p.num_m_tiles) * p.heads * 2 * ks * 2;
+  if (ctas > INT32_MAX) return fail(FN_ERR_UNSUPPORTED, "too many tiles");
+  CUtensorMap tx, tw;
+  fn_status st = make_operand_map(&tx, x, d, M, 128);
+  if (st != FN_OK) return st;
+  st = make_operand_map(&tw, w, d, N, static_cast<int>(head_dim / 4));
+  if (st != FN_OK) return st;
+  CUtensorMap tws;
+  st = make_partial_map(&tws, ws, N, M, ks);
+  if (st != FN_OK) return st;
+  // the attribute was set when the occupancy was queried (postnorm_split_max_pairs)
+  cudaError_t e = launch_kernel(fn::k_postnorm_split_gemm, dim3(static_cast<unsigned>(ctas)), dim3(fn::kPsThreads),
+                                fn::postnorm_split_smem_bytes(), stream, 2u, tx, tw, tws, p);
+  if (e != cudaSuccess) return cuda_fail(e, "wide-head split GEMM launch");
+  fn::PostnormFinalizeParams f;
+  f.ws = static_cast<const float*>(ws);
+  f.g2 = static_cast<const uint16_t*>(g2);
+  f.y = y;
+  f.M = p.M;
+  f.N = p.N;
+  f.head_dim = p.head_dim;
+  f.heads = p.heads;
+  f.ks = ks;
+  f.eps2 = eps2;
+  const int64_t items = M * p.heads;
+  int64_t blocks = (items + fn::kPfWarps - 1) / fn::kPfWarps;
+  if (blocks > 8LL * sms) blocks = 8LL * sms;
+  e = out_dtype == FN_F32
+          ? launch_kernel(fn::k_postnorm_finalize<true>, dim3(static_cast<unsigned>(blocks)), dim3(fn::kPfWarps * 32),
+                          0, stream, 1u, f)
+          : launch_kernel(fn::k_postnorm_finalize<false>, dim3(static_cast<unsigned>(blocks)),
+                          dim3(fn::kPfWarps * 32), 0, stream, 1u, f);
+  if (e != cudaSuccess) return cuda_fail(e, "wide-head post-norm finalize launch");
+  return FN_OK;
+}
+
+// ------------------------------------------------------------------------------------------------
 // GEMV (decode) path
 // ------------------------------------------------------------------------------------------------
 
@@ -662,6 +780,17 @@ fn_status projection(const void* x, const void* w, void* y, int64_t M, int64_t d
                          glu ? fn::EPI_GLU : fn::EPI_LINEAR, true, s);
 }
 
+fn_status check_postnorm(const void* x, const void* Wstar, const void* g2, const void* y, int64_t M, int64_t d,
+                         int64_t N, int64_t head_dim, float eps2, int out_dtype) {
+  fn_status st = check_common(x, Wstar, y, M, d, eps2, out_dtype);
+  if (st != FN_OK) return st;
+  if (head_dim < 16 || head_dim % 16 != 0) return fail(FN_ERR_INVALID_ARG, "head_dim = %lld must be a positive multiple of 16", (long long)head_dim);
+  if (head_dim > 512) return fail(FN_ERR_UNSUPPORTED, "head_dim = %lld > 512 (one tensor memory)", (long long)head_dim);
+  if (head_dim > 256 && head_dim % 32 != 0) return fail(FN_ERR_UNSUPPORTED, "head_dim in (256, 512] must be a multiple of 32");
+  if (N < head_dim || N > kMaxDim || N % head_dim != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a multiple of head_dim", (long long)N);
+  return check_ptr(g2, "g2");
+}
+
 }  // namespace
 
 extern "C" {
@@ -715,21 +844,46 @@ fn_status flashnorm_glu(const void* x, const void* Wstar_gu, void* y, int64_t M,
   return flashnorm_glu_ex(x, Wstar_gu, y, M, d, F, eps, out_dtype, FN_PATH_AUTO, stream);
 }
 
+fn_status flashnorm_postnorm_workspace_bytes(int64_t M, int64_t d, int64_t N, int64_t head_dim, int64_t* bytes) {
+  g_last_error[0] = '\0';
+  if (bytes == nullptr) return fail(FN_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = 0;
+  if (M < 0 || M > kMaxDim) return fail(FN_ERR_INVALID_ARG, "M = %lld out of range", (long long)M);
+  if (d < 8 || d > kMaxDim || d % 8 != 0) return fail(FN_ERR_INVALID_ARG, "d = %lld must be a positive multiple of 8", (long long)d);
+  if (head_dim < 16 || head_dim % 16 != 0 || head_dim > 512) return fail(FN_ERR_INVALID_ARG, "head_dim = %lld out of range", (long long)head_dim);
+  if (N < head_dim || N > kMaxDim || N % head_dim != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a multiple of head_dim", (long long)N);
+  const int ks = postnorm_split_ks(M, d, N, head_dim);
+  *bytes = static_cast<int64_t>(ks) * M * N * 4;
+  return FN_OK;
+}
+
+fn_status flashnorm_linear_postnorm_ws(const void* x, const void* Wstar, const void* g2, void* y, int64_t M, int64_t d,
+                                       int64_t N, int64_t head_dim, float eps2, int out_dtype, void* workspace,
+                                       int64_t workspace_bytes, void* stream) {
+  g_last_error[0] = '\0';
+  fn_status st = check_postnorm(x, Wstar, g2, y, M, d, N, head_dim, eps2, out_dtype);
+  if (st != FN_OK) return st;
+  if (workspace_bytes < 0) return fail(FN_ERR_INVALID_ARG, "workspace_bytes is negative");
+  if (M == 0) return FN_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (head_dim > 256) {
+    const int ks = workspace != nullptr ? postnorm_split_ks(M, d, N, head_dim) : 0;
+    if (ks > 0) {
+      const int64_t need = static_cast<int64_t>(ks) * M * N * 4;
+      if (workspace_bytes < need)
+        return fail(FN_ERR_INVALID_ARG, "workspace of %lld bytes; this shape needs %lld",
+                    (long long)workspace_bytes, (long long)need);
+      if ((st = check_ptr(workspace, "workspace")) != FN_OK) return st;
+      return run_postnorm_split(x, Wstar, g2, y, M, d, N, head_dim, eps2, out_dtype, ks, workspace, s);
+    }
+    return run_postnorm_pair(x, Wstar, g2, y, M, d, N, head_dim, eps2, out_dtype, s);
+  }
+  return run_tensor_path(x, Wstar, y, g2, M, d, N, N, head_dim, eps2, out_dtype, fn::EPI_POSTNORM, false, s);
+}
+
 fn_status flashnorm_linear_postnorm(const void* x, const void* Wstar, const void* g2, void* y, int64_t M, int64_t d,
                                     int64_t N, int64_t head_dim, float eps2, int out_dtype, void* stream) {
-  g_last_error[0] = '\0';
-  fn_status st = check_common(x, Wstar, y, M, d, eps2, out_dtype);
-  if (st != FN_OK) return st;
-  if (head_dim < 16 || head_dim % 16 != 0) return fail(FN_ERR_INVALID_ARG, "head_dim = %lld must be a positive multiple of 16", (long long)head_dim);
-  if (head_dim > 512) return fail(FN_ERR_UNSUPPORTED, "head_dim = %lld > 512 (one tensor memory)", (long long)head_dim);
-  if (head_dim > 256 && head_dim % 32 != 0) return fail(FN_ERR_UNSUPPORTED, "head_dim in (256, 512] must be a multiple of 32");
-  if (N < head_dim || N > kMaxDim || N % head_dim != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a multiple of head_dim", (long long)N);
-  if ((st = check_ptr(g2, "g2")) != FN_OK) return st;
-  if (M == 0) return FN_OK;
-  if (head_dim > 256)
-    return run_postnorm_pair(x, Wstar, g2, y, M, d, N, head_dim, eps2, out_dtype, static_cast<cudaStream_t>(stream));
-  return run_tensor_path(x, Wstar, y, g2, M, d, N, N, head_dim, eps2, out_dtype, fn::EPI_POSTNORM, false,
-                         static_cast<cudaStream_t>(stream));
+  return flashnorm_linear_postnorm_ws(x, Wstar, g2, y, M, d, N, head_dim, eps2, out_dtype, nullptr, 0, stream);
 }
 
 fn_status flashnorm_linear_postnorm_rope(const void* x, const void* Wstar, const void* g2, const void* rope_cs,

@@ -88,6 +88,28 @@ def test_glu_postnorm_fold_validation(lib):
     assert lib.flashnorm_rmsnorm(P, P, P, 4, 12, 1e-5, NULL) == fn.FN_ERR_INVALID_ARG
 
 
+def test_postnorm_workspace_validation(lib):
+    """The workspace entry point validates like flashnorm_linear_postnorm, and its size query rejects
+    shapes the call would reject."""
+    assert lib.flashnorm_linear_postnorm_ws(P, P, P, P, 4, 576, 1024, 1024, 1e-6, 0, NULL, 0, NULL) == \
+        fn.FN_ERR_UNSUPPORTED
+    assert lib.flashnorm_linear_postnorm_ws(P, P, P, P, 4, 576, 960, 128, 1e-6, 0, NULL, 0, NULL) == \
+        fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_linear_postnorm_ws(P, P, P, P, 4, 576, 512, 512, 1e-6, 0, P, -1, NULL) == \
+        fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_linear_postnorm_ws(P, P, P, P, 0, 576, 512, 512, 1e-6, 0, NULL, 0, NULL) == fn.FN_OK
+    nbytes = ctypes.c_int64(-7)
+    out = ctypes.c_void_p(ctypes.addressof(nbytes))
+    assert lib.flashnorm_postnorm_workspace_bytes(2048, 5120, 512, 512, NULL) == fn.FN_ERR_INVALID_ARG
+    for shape in [(2048, 5120, 500, 512), (2048, 5120, 512, 24), (2048, 12, 512, 512), (-1, 5120, 512, 512),
+                  (2048, 5120, 1024, 1024)]:
+        assert lib.flashnorm_postnorm_workspace_bytes(*shape, out) == fn.FN_ERR_INVALID_ARG, shape
+    # heads of at most 256 features never split; an empty call needs nothing
+    for shape in [(2048, 5120, 1024, 256), (0, 5120, 512, 512)]:
+        assert lib.flashnorm_postnorm_workspace_bytes(*shape, out) == fn.FN_OK
+        assert nbytes.value == 0
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
 

@@ -66,6 +66,24 @@ def test_postnorm_writes_stay_in_bounds(M, d, N, hd):
     assert O.rel_err(to_host_f64(y), ex) <= 1e-5
 
 
+@pytest.mark.parametrize("M,d,N,hd", [(700, 1000, 320, 320), (150, 5120, 1024, 512)])
+def test_postnorm_split_writes_stay_in_bounds(M, d, N, hd):
+    """The split wide-head schedule: its partial products stay inside the workspace size the query
+    reports, and the finalize kernel writes exactly y."""
+    need = fn.flashnorm_postnorm_workspace_bytes(M, d, N, hd)
+    assert need > 0
+    bits = I.Workload("t", "postnorm", M, d, N, 1e-6, head_dim=hd, eps2=1e-6, seed=M + 1).draw()
+    ws = fn.flashnorm_fold_weights(to_dev(bits["w"]), to_dev(bits["g"]))
+    flat_ws, wsp, n_ws = _guarded((need // 4,), torch.float32)
+    flat, y, n = _guarded((M, N), torch.bfloat16)
+    fn.flashnorm_linear_postnorm(to_dev(bits["x"]), ws, to_dev(bits["g2"]), hd, 1e-6, out=y,
+                                 workspace=wsp.view(torch.uint8))
+    torch.cuda.synchronize()
+    assert _intact(flat_ws, n_ws) and _intact(flat, n)
+    ex = O.exact_operand_output("postnorm", bits, O.fold_bf16(bits["w"], bits["g"]), 1e-6, eps2=1e-6, head_dim=hd)
+    assert O.rel_err(to_host_f64(y), ex) <= 5e-3
+
+
 def test_rope_layernorm_fp8_unfused_writes_stay_in_bounds():
     # RoPE on the post-norm path
     M, d, hd, H = 77, 256, 64, 3

@@ -186,17 +186,24 @@ POSTNORM_CASES = [
     (100, 64, 512, 512),         # one k-block: no K split
     (40, 128, 512, 512),         # two k-blocks: K split in two
     (2048, 576, 4096, 512),      # eight 512-wide heads: 64 clusters, more than fit at once
+    (300, 2048, 768, 384),       # two 384-wide heads, ragged M: split over K in independent pairs
+    (700, 1000, 320, 320),       # ragged M, d not a multiple of the 64-deep k-block, 320-wide head
 ]
 
 
+@pytest.mark.parametrize("workspace", ["auto", None])
 @pytest.mark.parametrize("M,d,N,hd", POSTNORM_CASES)
-def test_postnorm_parity(M, d, N, hd):
+def test_postnorm_parity(M, d, N, hd, workspace):
+    """Both schedules of a wide head: "auto" splits the contraction over independent CTA pairs through a
+    workspace where that applies, None keeps each row tile in one cluster."""
+    if workspace is None and (hd <= 256 or fn.flashnorm_postnorm_workspace_bytes(M, d, N, hd) == 0):
+        pytest.skip("no workspace is used for this shape: the same kernel as the auto case")
     bits = _wl("postnorm", M, d, N, eps=1e-6, eps2=1e-6, head_dim=hd, seed=M + hd).draw()
     x = to_dev(bits["x"])
     ws = _fold(bits, False)
     g2 = to_dev(bits["g2"])
-    y16 = fn.flashnorm_linear_postnorm(x, ws, g2, hd, 1e-6)
-    y32 = fn.flashnorm_linear_postnorm(x, ws, g2, hd, 1e-6, out_dtype=torch.float32)
+    y16 = fn.flashnorm_linear_postnorm(x, ws, g2, hd, 1e-6, workspace=workspace)
+    y32 = fn.flashnorm_linear_postnorm(x, ws, g2, hd, 1e-6, out_dtype=torch.float32, workspace=workspace)
     torch.cuda.synchronize()
     # bf16 against the FULL chain, first RMSNorm included
     ref = O.reference_output("postnorm", bits, 1e-6, eps2=1e-6, head_dim=hd)
@@ -205,9 +212,34 @@ def test_postnorm_parity(M, d, N, hd):
     check_bf16(to_host_f64(y16), ref, ref_exact)
     assert O.rel_err(to_host_f64(y32), ref_exact) <= F32_TOL
     # the partial sums of K ranges and columns are combined in a fixed order: bitwise repeatable
-    again = fn.flashnorm_linear_postnorm(x, ws, g2, hd, 1e-6, out_dtype=torch.float32)
+    again = fn.flashnorm_linear_postnorm(x, ws, g2, hd, 1e-6, out_dtype=torch.float32, workspace=workspace)
     torch.cuda.synchronize()
     assert torch.equal(again.view(torch.int32), y32.view(torch.int32))
+
+
+def test_postnorm_split_applies_where_expected():
+    """The split schedule is taken for the MLA latent shape (2048 rows, one 512-wide head: eight row tiles,
+    too few to fill the device), sized K ranges x M x N x 4 bytes, and not for shapes that fill it."""
+    nbytes = fn.flashnorm_postnorm_workspace_bytes(2048, 5120, 512, 512)
+    assert nbytes > 0 and nbytes % (2048 * 512 * 4) == 0 and 2 <= nbytes // (2048 * 512 * 4) <= 8
+    assert fn.flashnorm_postnorm_workspace_bytes(2048, 576, 4096, 512) == 0   # 64 row-tile x head units
+    assert fn.flashnorm_postnorm_workspace_bytes(2048, 5120, 1024, 128) == 0  # narrow heads: 1-CTA tiles
+    assert fn.flashnorm_postnorm_workspace_bytes(2048, 64, 512, 512) == 0     # one k-block: nothing to split
+
+
+def test_postnorm_workspace_too_small_is_rejected():
+    bits = _wl("postnorm", 256, 1024, 512, eps=1e-6, eps2=1e-6, head_dim=512, seed=9).draw()
+    x, ws, g2 = to_dev(bits["x"]), _fold(bits, False), to_dev(bits["g2"])
+    need = fn.flashnorm_postnorm_workspace_bytes(256, 1024, 512, 512)
+    assert need > 0
+    small = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(fn.FlashNormError, match="workspace"):
+        fn.flashnorm_linear_postnorm(x, ws, g2, 512, 1e-6, workspace=small)
+    exact = torch.empty(need, dtype=torch.uint8, device="cuda")
+    y = fn.flashnorm_linear_postnorm(x, ws, g2, 512, 1e-6, out_dtype=torch.float32, workspace=exact)
+    torch.cuda.synchronize()
+    ex = O.exact_operand_output("postnorm", bits, O.fold_bf16(bits["w"], bits["g"]), 1e-6, eps2=1e-6, head_dim=512)
+    assert O.rel_err(to_host_f64(y), ex) <= F32_TOL
 
 
 # ------------------------------------------------------------------------------------------ unfused baseline
