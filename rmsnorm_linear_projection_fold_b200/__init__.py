@@ -131,15 +131,16 @@ def _check(name: str, status: int) -> None:
 
 def _same_device(lead: torch.Tensor, **others) -> None:
     """Every tensor of a call must live on the device of `lead` (the C ABI takes bare pointers)."""
+    ld = lead.get_device()  # the CUDA device index, or -1 for any other device (compared in full below)
     for name, t in others.items():
-        if t is not None and t.device != lead.device:
+        if t is not None and (ld < 0 or t.get_device() != ld) and t.device != lead.device:
             raise ValueError(f"{name} is on {t.device}, expected {lead.device}")
 
 
 def _invoke(entry: str, lead: torch.Tensor, *args, report: str | None = None) -> None:
     """Call the library's `entry` with `lead`'s device current: the library launches on, and looks up
     its per-device state for, the current device."""
-    _invoke_on(lead.device.index, entry, *args, report=report)
+    _invoke_on(lead.get_device(), entry, *args, report=report)
 
 
 def _invoke_on(dev: int, entry: str, *args, report: str | None = None) -> None:
@@ -152,12 +153,20 @@ def _invoke_on(dev: int, entry: str, *args, report: str | None = None) -> None:
     _check(report or entry, status)
 
 
+# The current stream's cudaStream_t as an integer; torch's internal accessor skips building a Stream object
+# (about 2 us a call), with the public route where it is absent.
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream_ptr(t: torch.Tensor):
-    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+    if _raw_stream is not None:
+        return _raw_stream(t.get_device())
+    return torch.cuda.current_stream(t.device).cuda_stream
 
 
 def _ptr(t):
-    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+    """A tensor's device address for a void* argument (None passes NULL)."""
+    return t.data_ptr() if t is not None else None
 
 
 def _need(t: torch.Tensor, name: str, dtype=torch.bfloat16, dim=None) -> None:
@@ -236,14 +245,22 @@ def flashnorm_glu(x: torch.Tensor, Wstar_gu: torch.Tensor, eps: float, out_dtype
     return y
 
 
+_ws_bytes_cache = {}
+
+
 def flashnorm_postnorm_workspace_bytes(M: int, d: int, N: int, head_dim: int, device=None) -> int:
     """Workspace bytes flashnorm_linear_postnorm uses for this shape on `device` (0: no split)."""
     dev = torch.cuda.current_device() if device is None else torch.device(device).index
     if dev is None:
         dev = torch.cuda.current_device()
+    key = (dev, int(M), int(d), int(N), int(head_dim))
+    hit = _ws_bytes_cache.get(key)
+    if hit is not None:
+        return hit
     nbytes = ctypes.c_int64(0)
     _invoke_on(dev, "flashnorm_postnorm_workspace_bytes", int(M), int(d), int(N), int(head_dim),
-               ctypes.c_void_p(ctypes.addressof(nbytes)))
+               ctypes.addressof(nbytes))
+    _ws_bytes_cache[key] = int(nbytes.value)  # a function of the shape and the device's SM count only
     return int(nbytes.value)
 
 
@@ -269,7 +286,7 @@ def flashnorm_linear_postnorm(x: torch.Tensor, Wstar: torch.Tensor, g2: torch.Te
     if isinstance(workspace, str):
         if workspace != "auto":
             raise ValueError('workspace must be "auto", None or a uint8 CUDA tensor')
-        nbytes = flashnorm_postnorm_workspace_bytes(M, d, N, head_dim, x.device) if M > 0 else 0
+        nbytes = flashnorm_postnorm_workspace_bytes(M, d, N, head_dim, x.get_device()) if M > 0 else 0
         ws = torch.empty(nbytes, dtype=torch.uint8, device=x.device) if nbytes > 0 else None
     elif workspace is None:
         ws = None

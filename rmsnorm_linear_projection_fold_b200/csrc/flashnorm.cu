@@ -101,32 +101,76 @@ EncodeTiledFn encode_fn() {
   return fn_ptr;
 }
 
+// An encoded tensor map is a pure function of its arguments, so calls that pass the same buffer with the
+// same geometry reuse the previous encoding: a small per-thread cache keyed on every argument (a buffer
+// freed and allocated again at the same address with the same geometry gets a map that is still right).
+struct MapKey {
+  void* ptr;
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3];
+  int dtype, rank, swizzle, promo;
+};
+constexpr int kMapCacheSlots = 64;
+struct MapCacheEntry {
+  MapKey key;
+  CUtensorMap map;
+  bool valid;
+};
+
+CUresult encode_cached(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* ptr, const cuuint64_t* dims,
+                       const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swizzle,
+                       CUtensorMapL2promotion promo) {
+  MapKey k;
+  std::memset(&k, 0, sizeof(k));  // padding included: the key is compared byte for byte
+  k.ptr = ptr;
+  for (int i = 0; i < rank; ++i) k.dims[i] = dims[i], k.box[i] = box[i];
+  for (int i = 0; i + 1 < rank; ++i) k.strides[i] = strides[i];
+  k.dtype = static_cast<int>(dtype);
+  k.rank = rank;
+  k.swizzle = static_cast<int>(swizzle);
+  k.promo = static_cast<int>(promo);
+  uint64_t h = 1469598103934665603ull;  // FNV-1a over the key's bytes
+  const unsigned char* b = reinterpret_cast<const unsigned char*>(&k);
+  for (size_t i = 0; i < sizeof(k); ++i) h = (h ^ b[i]) * 1099511628211ull;
+  thread_local MapCacheEntry cache[kMapCacheSlots];
+  MapCacheEntry& e = cache[h % kMapCacheSlots];
+  if (e.valid && std::memcmp(&e.key, &k, sizeof(k)) == 0) {
+    *map = e.map;
+    return CUDA_SUCCESS;
+  }
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return CUDA_ERROR_NOT_FOUND;
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, dtype, static_cast<cuuint32_t>(rank), ptr, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r == CUDA_SUCCESS) {
+    e.key = k;
+    e.map = *map;
+    e.valid = true;
+  }
+  return r;
+}
+
 // 2-D bf16 K-major operand [rows, k] with a (64 x box_rows) box and 128-byte swizzle.
 fn_status make_operand_map(CUtensorMap* map, const void* ptr, int64_t k, int64_t rows, int box_rows) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(k) * 2};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(fn::kBK), static_cast<cuuint32_t>(box_rows)};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = encode_cached(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  if (r == CUDA_ERROR_NOT_FOUND) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   if (r != CUDA_SUCCESS) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
   return FN_OK;
 }
 
 // 2-D one-byte operand [rows, k] (FP8 E4M3 codes) with a (128 x box_rows) box and 128-byte swizzle.
 fn_status make_u8_map(CUtensorMap* map, const void* ptr, int64_t k, int64_t rows, int box_rows) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(k)};
   cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = encode_cached(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  if (r == CUDA_ERROR_NOT_FOUND) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   if (r != CUDA_SUCCESS) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
   return FN_OK;
 }
@@ -134,14 +178,12 @@ fn_status make_u8_map(CUtensorMap* map, const void* ptr, int64_t k, int64_t rows
 // 3-D fp32 [planes][rows][cols] (the split post-norm's partial products) with a 32-column x 128-row box
 // and 128-byte swizzle, for TMA stores.
 fn_status make_partial_map(CUtensorMap* map, void* ptr, int64_t cols, int64_t rows, int64_t planes) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(planes)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 4, static_cast<cuuint64_t>(cols * rows) * 4};
   cuuint32_t box[3] = {32u, 128u, 1u};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = encode_cached(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE);
+  if (r == CUDA_ERROR_NOT_FOUND) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   if (r != CUDA_SUCCESS) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
   return FN_OK;
 }
