@@ -579,11 +579,24 @@ fn_status run_postnorm_split(const void* x, const void* w, const void* g2, void*
   const int64_t items = M * p.heads;
   int64_t blocks = (items + fn::kPfWarps - 1) / fn::kPfWarps;
   if (blocks > 8LL * sms) blocks = 8LL * sms;
-  e = out_dtype == FN_F32
-          ? launch_kernel(fn::k_postnorm_finalize<true>, dim3(static_cast<unsigned>(blocks)), dim3(fn::kPfWarps * 32),
-                          0, stream, 1u, f)
-          : launch_kernel(fn::k_postnorm_finalize<false>, dim3(static_cast<unsigned>(blocks)),
-                          dim3(fn::kPfWarps * 32), 0, stream, 1u, f);
+  const dim3 fgrid(static_cast<unsigned>(blocks)), fblock(fn::kPfWarps * 32);
+#define FN_FIN(KS)                                                                                    \
+  case KS:                                                                                            \
+    e = out_dtype == FN_F32 ? launch_kernel(fn::k_postnorm_finalize<KS, true>, fgrid, fblock, 0, stream, 1u, f) \
+                            : launch_kernel(fn::k_postnorm_finalize<KS, false>, fgrid, fblock, 0, stream, 1u, f); \
+    break
+  switch (ks) {
+    FN_FIN(2);
+    FN_FIN(3);
+    FN_FIN(4);
+    FN_FIN(5);
+    FN_FIN(6);
+    FN_FIN(7);
+    FN_FIN(8);
+    default:
+      return fail(FN_ERR_UNSUPPORTED, "split post-norm with %d K ranges", ks);
+  }
+#undef FN_FIN
   if (e != cudaSuccess) return cuda_fail(e, "wide-head post-norm finalize launch");
   return FN_OK;
 }

@@ -258,9 +258,11 @@ __global__ void __launch_bounds__(kPsThreads, 1)
 }
 
 // One warp per (row, head). Lane l holds the head's columns 4l + 128j .. 4l + 128j + 3 (j = 0..3), so
-// each load and store of a warp covers 512 (fp32) or 256 (bf16) contiguous bytes.
-template <bool OUT_F32>
-__global__ void __launch_bounds__(kPfWarps * 32) k_postnorm_finalize(PostnormFinalizeParams p) {
+// each load and store of a warp covers 512 (fp32) or 256 (bf16) contiguous bytes. KS (the number of K
+// ranges) is a compile-time constant so that all KS x 4 loads of a row are issued before the first add:
+// one round trip to L2 per row instead of one per K range.
+template <int KS, bool OUT_F32>
+__global__ void __launch_bounds__(kPfWarps * 32, 2) k_postnorm_finalize(PostnormFinalizeParams p) {
   const int warp = static_cast<int>(threadIdx.x) >> 5;
   const int lane = static_cast<int>(threadIdx.x) & 31;
   const int hd = p.head_dim;
@@ -284,22 +286,22 @@ __global__ void __launch_bounds__(kPfWarps * 32) k_postnorm_finalize(PostnormFin
     const int h = static_cast<int>(it % p.heads);
     const size_t off = static_cast<size_t>(m) * p.N + static_cast<size_t>(h) * hd;
     // every K range's partials first (independent loads in flight), then their sum in range order
-    float4 part[kPsMaxKS][4];
+    float4 part[KS][4];
 #pragma unroll
-    for (int k = 0; k < kPsMaxKS; ++k)
+    for (int k = 0; k < KS; ++k)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int c = 4 * lane + 128 * j;
-        part[k][j] = (k < p.ks && c < hd) ? __ldcg(reinterpret_cast<const float4*>(p.ws + k * plane + off + c))
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        part[k][j] = c < hd ? __ldcg(reinterpret_cast<const float4*>(p.ws + k * plane + off + c))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     float u[16];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       float4 a = part[0][j];
 #pragma unroll
-      for (int k = 1; k < kPsMaxKS; ++k)
-        if (k < p.ks) a = make_float4(a.x + part[k][j].x, a.y + part[k][j].y, a.z + part[k][j].z, a.w + part[k][j].w);
+      for (int k = 1; k < KS; ++k)
+        a = make_float4(a.x + part[k][j].x, a.y + part[k][j].y, a.z + part[k][j].z, a.w + part[k][j].w);
       u[4 * j] = a.x, u[4 * j + 1] = a.y, u[4 * j + 2] = a.z, u[4 * j + 3] = a.w;
     }
     float ss = 0.f;
