@@ -145,6 +145,8 @@ __global__ void __launch_bounds__(kD8Threads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_x);
+    // the first ring's worth of this CTA's codes into L2 while the previous kernel drains
+    for (int u = u0; u < u1 && u < u0 + STAGES; ++u) tma_prefetch_l2_2d(&tm_q, u * kD8KStage, n0);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 256);

@@ -89,6 +89,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_w);
     tma_prefetch_desc(&tm_x);
+    // the first ring's worth of this CTA's W* into L2 while the previous kernel drains
+    for (int kb = kb0; kb < kb1 && kb < kb0 + STAGES; ++kb) tma_prefetch_l2_2d(&tm_w, kb * 64, n0);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 64);

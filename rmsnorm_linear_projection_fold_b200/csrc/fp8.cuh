@@ -131,6 +131,11 @@ __global__ void __launch_bounds__(kGemvThreads) k_gemv_fp8(const uint16_t* __res
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kc = K >> 3;   // x chunks per row
   const int qc = K >> 4;   // 16-weight chunks per W* row
+  {
+    // this warp's first group of codes into L2 (up to 4 KB a row) while the previous kernel drains
+    const int u = (static_cast<int>(blockIdx.x) * (kGemvThreads / 32) + warp) * R + lane;
+    if (lane < R && u < N) bulk_prefetch_l2(q + static_cast<size_t>(u) * K, static_cast<uint32_t>(min(K, 4096) & ~15));
+  }
   grid_dep_wait();
 
   for (int i = threadIdx.x; i < MT * kc; i += kGemvThreads) {

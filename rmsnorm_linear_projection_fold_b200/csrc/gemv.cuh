@@ -57,6 +57,14 @@ __global__ void __launch_bounds__(kGemvThreads) k_gemv(const uint16_t* __restric
   float* rs = reinterpret_cast<float*>(reinterpret_cast<uint16_t*>(smem_v) + MT * K);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kc = K >> 3;
+  {
+    // this warp's first group of W* rows into L2 (up to 4 KB a row) while the previous kernel drains
+    const int u = (static_cast<int>(blockIdx.x) * (kGemvThreads / 32) + warp) * R + (lane >> 1);
+    if (lane < 2 * R && u < n_units && (GLU || (lane & 1) == 0)) {
+      const int row = GLU ? ((u >> 4) << 5) + (u & 15) + (lane & 1) * 16 : u;
+      bulk_prefetch_l2(w + static_cast<size_t>(row) * K, static_cast<uint32_t>(min(2 * K, 4096) & ~15));
+    }
+  }
   grid_dep_wait();
 
   for (int i = threadIdx.x; i < MT * kc; i += kGemvThreads) {

@@ -258,6 +258,22 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
       : "memory");
 }
 
+// L2 prefetch of one 2-D box through a tensor map: no shared memory written, no barrier signalled. It is a
+// hint that changes no value any thread reads (L2 is where global memory is coherent), so a kernel may issue
+// it before griddepcontrol.wait and overlap its first loads' DRAM latency with the previous kernel's tail.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int c_inner, int c_outer) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(c_inner), "r"(c_outer)
+               : "memory");
+}
+
+// L2 prefetch of `bytes` (a multiple of 16) contiguous bytes at a 16-byte aligned address; a hint, like
+// tma_prefetch_l2_2d.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+
 // TMA tiled store of one 3-D box from shared memory, completion tracked by the bulk async-group.
 // Coordinates in elements, innermost first; the parts of the box outside the tensor are not written.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int c0, int c1, int c2) {
