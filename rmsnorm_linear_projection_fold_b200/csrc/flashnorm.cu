@@ -718,6 +718,7 @@ fn_status run_decode_fp8(const void* x, const void* q, const void* scales, void*
   const int64_t units = (d + fn::kD8KStage - 1) / fn::kD8KStage;
   // K split as for the bf16 decode kernel: in two while there are at most as many slabs as SMs (two
   // 5-stage CTAs fit one SM), in four when there are few slabs; otherwise one 10-stage CTA per slab.
+  // (In three, two 4-stage CTAs on every SM, the Llama-7B QKV codes took 23.9 us against 17.3 us.)
   int ksplit = 1;
   if (slabs <= sms && units >= 2) ksplit = 2;
   if (slabs * 4 <= sms && units >= 4) ksplit = 4;

@@ -35,7 +35,7 @@ def test_fold_fp8_zero_channel():
 
 @pytest.mark.parametrize("path", ["decode", "gemv"])
 @pytest.mark.parametrize("M,d,N", [(1, 4096, 1024), (3, 576, 960), (4, 4096, 2048), (7, 208, 136), (16, 576, 512),
-                                   (2, 64, 8), (16, 4096, 12288), (5, 400, 200)])
+                                   (2, 64, 8), (16, 4096, 12288), (5, 400, 200), (5, 1008, 6000)])
 def test_linear_fp8_parity(M, d, N, path):
     bits = I.Workload("t", "linear_fp8", M, d, N, 1e-6, seed=M * 13 + d).draw()
     Q, s = fn.flashnorm_fold_weights_fp8(to_dev(bits["w"]), to_dev(bits["g"]))
