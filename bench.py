@@ -67,6 +67,7 @@ BENCH_WORKLOADS = {
     "gemma_qkvnorm_hd128_m2048": ["gemma_qkvnorm_hd128_m2048"],
     "gemma_qkvnorm_rope_hd256_m2048": ["gemma_qkvnorm_rope_hd256_m2048"],
     "layernorm_qkv_m8192": ["layernorm_qkv_m8192"],
+    "layernorm_llama7b_qkv_m4": ["layernorm_llama7b_qkv_m4"],
     "llama7b_qkv_fp8_m1": ["llama7b_qkv_fp8_m1"],
     "llama7b_qkv_fp8_m4": ["llama7b_qkv_fp8_m4"],
     "llama7b_qkv_fp8_m16": ["llama7b_qkv_fp8_m16"],

@@ -167,6 +167,9 @@ WORKLOADS = {
     "llama7b_qkv_fp8_m16": Workload("llama7b_qkv_fp8_m16", "linear_fp8", 16, 4096, 12288, 1e-6, seed=BASE_SEED + 2),
     # LayerNorm (gain and bias) before the SmolLM2-sized QKV projection, 8192 tokens
     "layernorm_qkv_m8192": Workload("layernorm_qkv_m8192", "layernorm", 8192, 576, 960, 1e-5, seed=BASE_SEED + 7),
+    # LayerNorm before the Llama-7B-sized QKV projection at decode, 4 tokens
+    "layernorm_llama7b_qkv_m4": Workload("layernorm_llama7b_qkv_m4", "layernorm", 4, 4096, 12288, 1e-5,
+                                         seed=BASE_SEED + 8),
     # The same with RoPE fused after the per-head norm on the query and key heads (8 q + 4 k heads of 256,
     # then 4 value heads), positions 0 .. 2047 of a prefill.
     "gemma_qkvnorm_rope_hd256_m2048": Workload("gemma_qkvnorm_rope_hd256_m2048", "postnorm_rope", 2048, 2560, 4096,

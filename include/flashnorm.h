@@ -207,8 +207,9 @@ FN_API fn_status flashnorm_linear_postnorm_rope(const void* x, const void* Wstar
  * flashnorm_fold_layernorm: W bf16 [d, N] row-major, gamma bf16 [d], beta bf16 [d] or NULL (no bias) ->
  *   Wstar bf16 [N, d] (exactly flashnorm_fold_weights(W, gamma, glu = 0)), colsum fp32 [N] = sum over k of the
  *   bf16 W*[n][k], bias fp32 [N] = sum over k of beta[k] W[k][n] (fp32). All caller-owned device memory.
- * flashnorm_layernorm_linear: x bf16 [M, d] -> y [M, N] of out_dtype, on the CTA-pair tensor-core kernel
- *   for every M. Constraints: d % 8 == 0, N % 8 == 0, eps >= 0. The variance is taken as
+ * flashnorm_layernorm_linear: x bf16 [M, d] -> y [M, N] of out_dtype: M <= FN_DECODE_MAX_M on the
+ *   tensor-core decode kernel (the weights stream once), larger M on the CTA-pair tensor-core kernel.
+ *   Constraints: d % 8 == 0, N % 8 == 0, eps >= 0. The variance is taken as
  *   E[x^2] - mu^2 in fp32 (clamped at 0), accurate while |mu| is not large against the spread of x.
  */
 FN_API fn_status flashnorm_fold_layernorm(const void* W, const void* gamma, const void* beta, void* Wstar,

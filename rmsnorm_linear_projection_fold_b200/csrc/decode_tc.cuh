@@ -14,6 +14,10 @@
 // cluster's distributed shared memory, and the leader adds them, scales and stores. A CTA whose bounded
 // wait gave up sends NaN partial sums, so the outputs they feed are NaN rather than plausible values.
 //
+// LayerNorm (LN): the same four warps also add up x per token, and the epilogue applies the rank-1 form
+// of the fold, y = r (x . W*) - (r mu) colsum(W*) + beta^T W, with mu the token's mean and
+// r = 1/sqrt(E[x^2] - mu^2 + eps) (see flashnorm_fold_layernorm).
+//
 // Warps: 0 = TMA producer, 1 = TMEM allocator + MMA issuer, 2..5 = sum of squares, then epilogue.
 #pragma once
 
@@ -41,17 +45,21 @@ struct DecodeParams {
   int ldy;
   int ksplit;  // CTAs per cluster sharing one slab (1, 2 or 4)
   float eps;
+  // LN: fp32 [n_out] column sums of the folded W* and folded bias beta^T W
+  const float* ln_colsum = nullptr;
+  const float* ln_bias = nullptr;
 };
 
 template <int STAGES, int KSPLIT>
 __host__ __device__ constexpr int decode_smem_bytes() {
-  return 1024 + STAGES * (kDecWStage + kDecXStage) + (KSPLIT > 1 ? KSPLIT * (kDecRows * kDecTok + kDecTok) * 4 : 0) +
-         1024;
+  return 1024 + STAGES * (kDecWStage + kDecXStage) +
+         (KSPLIT > 1 ? KSPLIT * (kDecRows * kDecTok + 2 * kDecTok) * 4 : 0) + 1024;
 }
 
-template <int STAGES, int KSPLIT, bool GLU, bool OUT_F32>
+template <int STAGES, int KSPLIT, bool GLU, bool OUT_F32, bool LN = false>
 __global__ void __launch_bounds__(kDecThreads, 1)
     k_decode_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, DecodeParams p) {
+  static_assert(!(LN && GLU), "LayerNorm is fused into the linear epilogue only");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -59,12 +67,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   uint8_t* sX = sW + STAGES * kDecWStage;
   float* part_d = reinterpret_cast<float*>(sX + STAGES * kDecXStage);      // [KSPLIT][128][16] (leader)
   float* part_ss = part_d + (KSPLIT > 1 ? KSPLIT * kDecRows * kDecTok : 0);  // [KSPLIT][16]
-  uint64_t* full = reinterpret_cast<uint64_t*>(part_ss + (KSPLIT > 1 ? KSPLIT * kDecTok : 0));
+  float* part_sx = part_ss + (KSPLIT > 1 ? KSPLIT * kDecTok : 0);             // [KSPLIT][16], LN
+  uint64_t* full = reinterpret_cast<uint64_t*>(part_sx + (KSPLIT > 1 ? KSPLIT * kDecTok : 0));
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* drain = acc_full + 1;
   float* rs = reinterpret_cast<float*>(drain + 1);  // [16] 1/rms per token
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rs + kDecTok);
+  float* kms = rs + kDecTok;                        // [16] LN: r * mu per token
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(kms + kDecTok);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x) >> 5, 0);
@@ -189,22 +199,21 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    float ss = 0.f;
+    float ss = 0.f, sx = 0.f;
     for (int kb = kb0; kb < kb1; ++kb) {
       if (!mbar_wait(&full[s], ph, abort_flag)) {
         ok = false;
         break;
       }
       const uint4 w = *reinterpret_cast<const uint4*>(sX + s * kDecXStage + tok * 128 + chunk * 16);
-      float f;
-      f = bf16lo_to_f32(w.x); ss = fmaf(f, f, ss);
-      f = bf16hi_to_f32(w.x); ss = fmaf(f, f, ss);
-      f = bf16lo_to_f32(w.y); ss = fmaf(f, f, ss);
-      f = bf16hi_to_f32(w.y); ss = fmaf(f, f, ss);
-      f = bf16lo_to_f32(w.z); ss = fmaf(f, f, ss);
-      f = bf16hi_to_f32(w.z); ss = fmaf(f, f, ss);
-      f = bf16lo_to_f32(w.w); ss = fmaf(f, f, ss);
-      f = bf16hi_to_f32(w.w); ss = fmaf(f, f, ss);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float lo = bf16lo_to_f32(ws[i]), hi = bf16hi_to_f32(ws[i]);
+        ss = fmaf(lo, lo, ss);
+        ss = fmaf(hi, hi, ss);
+        if (LN) sx += lo + hi;
+      }
       fence_proxy_async_smem();  // the reads above come before the TMA refill this arrival permits
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
@@ -218,9 +227,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const float kNaN = __int_as_float(0x7fc00000);
     if (!ok) ss = kNaN;
     // the eight threads of a token are eight consecutive lanes
-    ss += __shfl_xor_sync(0xffffffffu, ss, 4);
-    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) {
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (LN) sx += __shfl_xor_sync(0xffffffffu, sx, o);
+    }
 
     float v[kDecTok];
     const bool have_acc = ok && kb1 > kb0;
@@ -253,6 +264,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
         for (int j = 0; j < kDecTok; j += 4) dsmem_st_v4(dst + j * 4, v[j], v[j + 1], v[j + 2], v[j + 3]);
         if (chunk == 0) dsmem_st_f32(dsmem_addr(part_ss + rank * kDecTok + tok, 0), ss);
+        if (LN && chunk == 0) dsmem_st_f32(dsmem_addr(part_sx + rank * kDecTok + tok, 0), sx);
       }
     }
     if (KSPLIT > 1) cluster_sync_all();  // every thread of the cluster, also warps 0 and 1 (below)
@@ -262,17 +274,30 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
           for (int j = 0; j < kDecTok; ++j) v[j] += part_d[(rr * kDecRows + row) * kDecTok + j];
           if (chunk == 0) ss += part_ss[rr * kDecTok + tok];
+          if (LN && chunk == 0) sx += part_sx[rr * kDecTok + tok];
         }
       }
-      if (chunk == 0) rs[tok] = 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps);
+      if (chunk == 0) {
+        if (LN) {
+          // biased variance E[x^2] - mu^2, clamped at 0 against rounding; eps inside the root
+          const float mu = sx / static_cast<float>(p.K);
+          const float var = fmaxf(ss / static_cast<float>(p.K) - mu * mu, 0.0f);
+          rs[tok] = 1.0f / sqrtf(var + p.eps);
+          kms[tok] = rs[tok] * mu;
+        } else {
+          rs[tok] = 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps);
+        }
+      }
       named_bar_sync(1, 128);
       {
         if (!GLU) {
           const int n = n0 + row;
+          float cn = 0.f, bn = 0.f;
+          if (LN && n < p.n_out) cn = __ldg(p.ln_colsum + n), bn = __ldg(p.ln_bias + n);
 #pragma unroll
           for (int m = 0; m < kDecTok; ++m) {
             if (m >= p.M) break;
-            const float o = v[m] * rs[m];
+            const float o = LN ? fmaf(v[m], rs[m], fmaf(-kms[m], cn, bn)) : v[m] * rs[m];
             if (n < p.n_out) {
               if (OUT_F32)
                 static_cast<float*>(p.y)[static_cast<size_t>(m) * p.ldy + n] = o;

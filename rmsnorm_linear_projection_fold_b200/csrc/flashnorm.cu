@@ -751,10 +751,10 @@ fn_status run_decode_fp8(const void* x, const void* q, const void* scales, void*
 // Tensor-core decode path
 // ------------------------------------------------------------------------------------------------
 
-template <int STAGES, int KSPLIT, bool GLU, bool OUT_F32>
+template <int STAGES, int KSPLIT, bool GLU, bool OUT_F32, bool LN>
 fn_status launch_decode_t(const CUtensorMap& tw, const CUtensorMap& tx, const fn::DecodeParams& p, int slabs,
                           int dev, cudaStream_t stream) {
-  auto kern = fn::k_decode_tc<STAGES, KSPLIT, GLU, OUT_F32>;
+  auto kern = fn::k_decode_tc<STAGES, KSPLIT, GLU, OUT_F32, LN>;
   constexpr int smem = fn::decode_smem_bytes<STAGES, KSPLIT>();
   static bool configured[kMaxDevices] = {false};
   if (!configured[dev]) {
@@ -768,8 +768,10 @@ fn_status launch_decode_t(const CUtensorMap& tw, const CUtensorMap& tx, const fn
   return FN_OK;
 }
 
+// colsum / bias non-null: the LayerNorm epilogue (linear only).
 fn_status run_decode_tc(const void* x, const void* w, void* y, int64_t M, int64_t d, int64_t n_rows, int64_t n_out,
-                        float eps, int out_dtype, bool glu, cudaStream_t stream) {
+                        float eps, int out_dtype, bool glu, cudaStream_t stream, const float* colsum = nullptr,
+                        const float* bias = nullptr) {
   int dev = 0;
   const int sms = device_sm_count(&dev);
   if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
@@ -796,13 +798,18 @@ fn_status run_decode_tc(const void* x, const void* w, void* y, int64_t M, int64_
   p.ldy = static_cast<int>(n_out);
   p.ksplit = ksplit;
   p.eps = eps;
+  p.ln_colsum = colsum;
+  p.ln_bias = bias;
+  const bool ln = colsum != nullptr;
   const int sl = static_cast<int>(slabs);
   const bool f32 = out_dtype == FN_F32;
 #define FN_DEC(ST, KS)                                                                                          \
-  (glu ? (f32 ? launch_decode_t<ST, KS, true, true>(tw, tx, p, sl, dev, stream)                              \
-              : launch_decode_t<ST, KS, true, false>(tw, tx, p, sl, dev, stream))                            \
-       : (f32 ? launch_decode_t<ST, KS, false, true>(tw, tx, p, sl, dev, stream)                             \
-              : launch_decode_t<ST, KS, false, false>(tw, tx, p, sl, dev, stream)))
+  (ln    ? (f32 ? launch_decode_t<ST, KS, false, true, true>(tw, tx, p, sl, dev, stream)                     \
+                : launch_decode_t<ST, KS, false, false, true>(tw, tx, p, sl, dev, stream))                   \
+   : glu ? (f32 ? launch_decode_t<ST, KS, true, true, false>(tw, tx, p, sl, dev, stream)                     \
+                : launch_decode_t<ST, KS, true, false, false>(tw, tx, p, sl, dev, stream))                   \
+         : (f32 ? launch_decode_t<ST, KS, false, true, false>(tw, tx, p, sl, dev, stream)                    \
+                : launch_decode_t<ST, KS, false, false, false>(tw, tx, p, sl, dev, stream)))
   if (ksplit == 1) return FN_DEC(12, 1);
   if (ksplit == 2) return FN_DEC(5, 2);
   return FN_DEC(3, 4);
@@ -999,6 +1006,10 @@ fn_status flashnorm_layernorm_linear(const void* x, const void* Wstar, const voi
   if ((st = check_ptr(colsum, "colsum")) != FN_OK) return st;
   if ((st = check_ptr(bias, "bias")) != FN_OK) return st;
   if (M == 0) return FN_OK;
+  // decode-sized batches on the tensor-core decode kernel (the weights stream once), larger on CTA pairs
+  if (M <= FN_DECODE_MAX_M)
+    return run_decode_tc(x, Wstar, y, M, d, N, N, eps, out_dtype, false, static_cast<cudaStream_t>(stream),
+                         static_cast<const float*>(colsum), static_cast<const float*>(bias));
   return run_pair_path(x, Wstar, y, M, d, N, N, eps, out_dtype, fn::EPI_LN, true, static_cast<cudaStream_t>(stream),
                        static_cast<const float*>(colsum), static_cast<const float*>(bias));
 }

@@ -84,6 +84,20 @@ def test_postnorm_split_writes_stay_in_bounds(M, d, N, hd):
     assert O.rel_err(to_host_f64(y), ex) <= 5e-3
 
 
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_layernorm_decode_writes_stay_in_bounds(out_dtype):
+    """LayerNorm at decode size (the tensor-core decode kernel, ragged N, K split over a cluster)."""
+    bits = I.Workload("t", "layernorm", 5, 576, 200, 1e-5, seed=41).draw()
+    Ws, cs, bias = fn.flashnorm_fold_layernorm(to_dev(bits["w"]), to_dev(bits["g"]), to_dev(bits["beta"]))
+    flat, y, n = _guarded((5, 200), out_dtype)
+    fn.flashnorm_layernorm_linear(to_dev(bits["x"]), Ws, cs, bias, 1e-5, out_dtype=out_dtype, out=y)
+    torch.cuda.synchronize()
+    assert _intact(flat, n)
+    tol = 1e-5 if out_dtype == torch.float32 else 5e-3
+    ex = O.exact_operand_layernorm(bits, O.fold_bf16(bits["w"], bits["g"]), 1e-5)
+    assert O.rel_err(to_host_f64(y), ex if out_dtype == torch.float32 else O.reference_layernorm(bits, 1e-5)) <= tol
+
+
 def test_rope_layernorm_fp8_unfused_writes_stay_in_bounds():
     # RoPE on the post-norm path
     M, d, hd, H = 77, 256, 64, 3

@@ -35,7 +35,10 @@ def test_fold_outputs():
 
 
 @pytest.mark.parametrize("M,d,N", [(300, 576, 960), (17, 576, 960), (130, 72, 200), (600, 4096, 512),
-                                   (257, 256, 1536)])
+                                   (257, 256, 1536),
+                                   # decode-sized: the tensor-core decode kernel (K split in 2 and in 4)
+                                   (1, 4096, 1024), (4, 576, 960), (16, 256, 1536), (7, 200, 136),
+                                   (16, 4096, 12288)])
 def test_layernorm_parity(M, d, N):
     bits = I.Workload("t", "layernorm", M, d, N, 1e-5, seed=M + d).draw()
     Ws, cs, b = _fold(bits)
@@ -71,4 +74,18 @@ def test_layernorm_many_tiles_all_rows():
     y32 = fn.flashnorm_layernorm_linear(to_dev(bits["x"]), Ws, cs, b, 1e-6, out_dtype=torch.float32)
     torch.cuda.synchronize()
     ex = O.exact_operand_layernorm(bits, O.fold_bf16(bits["w"], bits["g"]), 1e-6)
+    assert O.rel_err(to_host_f64(y32), ex) <= F32_TOL
+
+
+def test_layernorm_decode_full_size():
+    """The benchmark's LayerNorm decode shape (4 tokens, Llama-7B QKV): every output against the oracle."""
+    wl = I.WORKLOADS["layernorm_llama7b_qkv_m4"]
+    bits = wl.draw()
+    Ws, cs, b = _fold(bits)
+    x = to_dev(bits["x"])
+    y16 = fn.flashnorm_layernorm_linear(x, Ws, cs, b, wl.eps)
+    y32 = fn.flashnorm_layernorm_linear(x, Ws, cs, b, wl.eps, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ex = O.exact_operand_layernorm(bits, O.fold_bf16(bits["w"], bits["g"]), wl.eps)
+    check_bf16(to_host_f64(y16), O.reference_layernorm(bits, wl.eps), ex)
     assert O.rel_err(to_host_f64(y32), ex) <= F32_TOL

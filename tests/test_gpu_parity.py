@@ -339,6 +339,37 @@ def test_no_stale_output_back_to_back(path, M, T):
         prev = ref
 
 
+@pytest.mark.parametrize("workspace", ["shared", "auto"])
+def test_postnorm_split_back_to_back(workspace):
+    """The split wide-head schedule over many calls back to back with no host sync: each call's GEMM
+    overwrites the partial products that the previous call's finalize kernel reads, so a GEMM that started
+    writing before that finalize had finished would corrupt the previous output. Every output, copied out
+    right after its call, must equal (bitwise) the same call run alone, and match the oracle."""
+    M, d, N, hd, T = 256, 1024, 512, 512, 120
+    assert fn.flashnorm_postnorm_workspace_bytes(M, d, N, hd) > 0
+    bits = _wl("postnorm", M, d, N, eps=1e-6, eps2=1e-6, head_dim=hd, seed=21).draw()
+    W, g2 = _fold(bits, False), to_dev(bits["g2"])
+    xs_bits = [I.activations(M, d, 3000 + t) for t in range(T)]
+    xs = [to_dev(b) for b in xs_bits]
+    wsp = torch.empty(fn.flashnorm_postnorm_workspace_bytes(M, d, N, hd), dtype=torch.uint8, device="cuda")
+    use = wsp if workspace == "shared" else "auto"
+    y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    outs = []
+    torch.cuda.synchronize()
+    for t in range(T):
+        fn.flashnorm_linear_postnorm(xs[t], W, g2, hd, 1e-6, out_dtype=torch.float32, out=y, workspace=use)
+        outs.append(y.clone())
+    torch.cuda.synchronize()
+    for t in range(T):
+        alone = fn.flashnorm_linear_postnorm(xs[t], W, g2, hd, 1e-6, out_dtype=torch.float32, workspace=wsp)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[t].view(torch.int32), alone.view(torch.int32)), t
+    for t in (0, T // 2, T - 1):
+        b = dict(bits, x=xs_bits[t])
+        ex = O.exact_operand_output("postnorm", b, O.fold_bf16(bits["w"], bits["g"]), 1e-6, eps2=1e-6, head_dim=hd)
+        assert O.rel_err(to_host_f64(outs[t]), ex) <= F32_TOL
+
+
 def test_two_streams_and_determinism():
     bits = _wl("glu", 500, 576, 1536, seed=9).draw()
     x = to_dev(bits["x"])
