@@ -133,12 +133,6 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_addr, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_addr),
-               "r"(bytes)
-               : "memory");
-}
-
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -201,18 +195,6 @@ __device__ __forceinline__ void dsmem_st_f32(uint32_t addr, float a) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(a) : "memory");
 }
 
-// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory to another CTA's shared memory
-// in the cluster; completion is counted (complete_tx) on `remote_bar`, an mbarrier in the
-// destination CTA. Both remote addresses come from dsmem_addr().
-__device__ __forceinline__ void bulk_push_dsmem(uint32_t remote_dst, const void* local_src, uint32_t bytes,
-                                                uint32_t remote_bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          remote_dst),
-      "r"(smem_u32(local_src)), "r"(bytes), "r"(remote_bar)
-      : "memory");
-}
-
 // Every thread of every CTA in the cluster arrives; writes before it (including to other CTAs'
 // shared memory) are visible to all threads after it. Not the .aligned form: the lanes of a warp may
 // reach it at different times.
@@ -234,16 +216,6 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
       "[%2];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c_inner), "r"(c_outer)
-      : "memory");
-}
-
-// Same with an L2 eviction-priority hint (a createpolicy cache policy).
-__device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
-                                                 int c_inner, int c_outer, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
-      "[%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c_inner), "r"(c_outer), "l"(policy)
       : "memory");
 }
 
@@ -294,18 +266,6 @@ __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.w
 // Lets the next kernel of the stream (if launched as above) be scheduled once every CTA of this grid
 // has issued it or exited. Only scheduling moves earlier; the next kernel still waits for our completion.
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
-__device__ __forceinline__ uint64_t l2_policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
-__device__ __forceinline__ uint64_t l2_policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
 
 // ---------------------------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation MMA.
