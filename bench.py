@@ -63,6 +63,8 @@ BENCH_WORKLOADS = {
     "llama7b_qkv_m2048": ["llama7b_qkv_m2048"],
     "llama7b_ffn_m2048": ["llama7b_ffn_m2048"],
     "mla_latent_m2048": ["mla_latent_m2048"],
+    # the same without a workspace: the wide-head kernel that keeps each row tile in one cluster
+    "mla_latent_cluster_m2048": ["mla_latent_m2048"],
     "gemma_qkvnorm_hd256_m2048": ["gemma_qkvnorm_hd256_m2048"],
     "gemma_qkvnorm_hd128_m2048": ["gemma_qkvnorm_hd128_m2048"],
     "gemma_qkvnorm_rope_hd256_m2048": ["gemma_qkvnorm_rope_hd256_m2048"],
@@ -80,7 +82,8 @@ BENCH_WORKLOADS = {
 }
 # Kernel family forced for a bench workload (default: the library's own choice, FN_PATH_AUTO).
 BENCH_PATHS = {"llama7b_qkv_gemv_m16": "gemv", "llama7b_qkv_gemv_m1": "gemv", "llama7b_qkv_fp8_gemv_m1": "gemv",
-               "llama7b_qkv_fp8_gemv_m4": "gemv", "llama7b_qkv_fp8_tc_m1": "decode"}
+               "llama7b_qkv_fp8_gemv_m4": "gemv", "llama7b_qkv_fp8_tc_m1": "decode",
+               "mla_latent_cluster_m2048": "cluster"}
 DEFAULT_WORKLOAD = "llama7b_ffn_m2048"
 
 # DRAM traffic of the dominant kernel per launch (dram__bytes_read.sum + dram__bytes_write.sum of one
@@ -272,7 +275,7 @@ class Projection:
         # a wide head with few row tiles splits its contraction through a workspace (allocated once here,
         # as a serving loop would); 0 bytes where the split does not apply
         self.pn_ws = None
-        if wl.kind == "postnorm":
+        if wl.kind == "postnorm" and path != "cluster":
             need = fn.flashnorm_postnorm_workspace_bytes(wl.M, wl.d, wl.N, wl.head_dim)
             self.pn_ws = torch.empty(need, dtype=torch.uint8, device="cuda") if need > 0 else None
         if wl.kind == "postnorm_rope":  # the (cos, sin) table and the row positions are set up once
