@@ -91,8 +91,19 @@ DEFAULT_WORKLOAD = "llama7b_ffn_m2048"
 # hash differently now, traffic is reported as null.
 NCU_TRAFFIC = {
     # workload: (bytes per launch, sha256[:16] of the csrc/*.cu* sources at capture time)
-    "llama7b_ffn_m2048": (826738688, "bc8a4ae62a0459dd"),
-    "llama7b_qkv_fp8_m4": (50473984, "bc8a4ae62a0459dd"),
+    "llama7b_ffn_m2048": (854593024, "9df93328d7be0c0a"),
+    "llama7b_qkv_m2048": (502012928, "9df93328d7be0c0a"),
+    "smollm2_ffn_m8192": (13023488, "9df93328d7be0c0a"),
+    "layernorm_qkv_m8192": (10594048, "9df93328d7be0c0a"),
+    "smollm2_qkv_m64": (1216000, "9df93328d7be0c0a"),
+    "gemma_qkvnorm_hd256_m2048": (31505408, "9df93328d7be0c0a"),
+    "gemma_qkvnorm_rope_hd256_m2048": (33614592, "9df93328d7be0c0a"),
+    "llama7b_qkv_m16": (104636160, "9df93328d7be0c0a"),
+    "layernorm_llama7b_qkv_m4": (104762624, "9df93328d7be0c0a"),
+    "llama7b_qkv_gemv_m16": (104215552, "9df93328d7be0c0a"),
+    "llama7b_qkv_fp8_m1": (50429440, "9df93328d7be0c0a"),
+    "llama7b_qkv_fp8_m4": (50467072, "9df93328d7be0c0a"),
+    "mla_latent_cluster_m2048": (26264320, "9df93328d7be0c0a"),
 }
 
 # The dominant-kernel loop and each block of the fused/unfused comparison run at least this many
