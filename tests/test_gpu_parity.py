@@ -387,6 +387,53 @@ def test_two_streams_and_determinism():
     assert torch.equal(a.view(torch.int16), c.view(torch.int16))
 
 
+def test_cuda_graph_replay_matches_eager():
+    """Calls captured once in a CUDA graph (the launch mode of a serving loop) and replayed on new inputs
+    copied into the captured buffers: the split wide-head post-norm with its workspace drawn inside the
+    capture, a decode projection, the FP8 decode kernel and a SwiGLU projection on CTA pairs. Each replay
+    must equal, bitwise, the same calls run eagerly on the same inputs."""
+    pn = _wl("postnorm", 256, 1024, 512, eps=1e-6, eps2=1e-6, head_dim=512, seed=31).draw()
+    dc = _wl("linear", 4, 1024, 1024, seed=32).draw()
+    gl = _wl("glu", 300, 576, 1536, seed=33).draw()
+    f8 = I.Workload("t", "linear_fp8", 5, 1024, 768, 1e-6, seed=34).draw()
+    W_pn, g2 = _fold(pn, False), to_dev(pn["g2"])
+    W_dc, W_gl = _fold(dc, False), _fold(gl, True)
+    Q, sc = fn.flashnorm_fold_weights_fp8(to_dev(f8["w"]), to_dev(f8["g"]))
+    x_pn, x_dc, x_gl, x_f8 = to_dev(pn["x"]), to_dev(dc["x"]), to_dev(gl["x"]), to_dev(f8["x"])
+
+    def step():
+        return (fn.flashnorm_linear_postnorm(x_pn, W_pn, g2, 512, 1e-6, out_dtype=torch.float32),
+                fn.flashnorm_linear(x_dc, W_dc, 1e-5),
+                fn.flashnorm_linear_fp8(x_f8, Q, sc, 1e-6),
+                fn.flashnorm_glu(x_gl, W_gl, 1e-5))
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()  # warm-up on the capture stream (per-device setup happens outside the capture)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        outs = step()
+    for t in range(3):
+        for x, m, d in ((x_pn, 256, 1024), (x_dc, 4, 1024), (x_gl, 300, 576), (x_f8, 5, 1024)):
+            x.copy_(to_dev(I.activations(m, d, 4000 + 10 * t + d % 7)))
+        g.replay()
+        torch.cuda.synchronize()
+        eager = step()
+        torch.cuda.synchronize()
+        for a, b in zip(outs, eager):
+            ia = a.view(torch.int32) if a.dtype == torch.float32 else a.view(torch.int16)
+            ib = b.view(torch.int32) if b.dtype == torch.float32 else b.view(torch.int16)
+            assert torch.equal(ia, ib), t
+    # the replayed post-norm output is also the oracle's
+    b = dict(pn, x=I.activations(256, 1024, 4000 + 20 + 1024 % 7))
+    ex = O.exact_operand_output("postnorm", b, O.fold_bf16(pn["w"], pn["g"]), 1e-6, eps2=1e-6, head_dim=512)
+    assert O.rel_err(to_host_f64(outs[0]), ex) <= F32_TOL
+    del g
+
+
 # ------------------------------------------------------------------------------------------ edge cases
 def test_empty_and_zero_rows():
     d, N = 576, 960
