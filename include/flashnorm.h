@@ -244,6 +244,36 @@ FN_API fn_status flashnorm_linear_fp8_ex(const void* x, const void* Q, const voi
                                          int64_t d, int64_t N, float eps, int out_dtype, int path, void* stream);
 
 /*
+ * flashnorm_linear_fp8_ws — flashnorm_linear_fp8_ex with a caller-provided workspace. The same result
+ * (same definition, same tolerances); what changes is how the tensor-core kernel splits the contraction
+ * d. Without a workspace, the CTAs that share one 128-row slab of Q form a thread-block cluster and add
+ * their partial sums on chip. With one, they are independent CTAs, enough for two on every SM, that write
+ * fp32 partials to the workspace; the last of a slab's CTAs to finish adds them in a fixed order
+ * (deterministic, whichever CTA comes last) and writes the output. FN_PATH_AUTO then takes the
+ * tensor-core kernel for one token as well.
+ *   workspace        device memory, 16-byte aligned, caller-owned, or NULL (no workspace). Its first
+ *                    1024 bytes are arrival counters: zero them (cudaMemset) before the workspace's
+ *                    first use; every call leaves them zero again. The rest is scratch. Calls whose
+ *                    kernels may overlap on the GPU (different streams, host threads) must not share
+ *                    one; successive calls on one stream may, whatever their shapes.
+ *   workspace_bytes  its size. A non-NULL workspace smaller than flashnorm_fp8_workspace_bytes reports
+ *                    for this shape returns FN_ERR_INVALID_ARG and launches nothing.
+ * Shapes for which the split does not apply (more 128-row slabs than SMs: the size query returns 0),
+ * and FN_PATH_GEMV, ignore the workspace.
+ */
+FN_API fn_status flashnorm_linear_fp8_ws(const void* x, const void* Q, const void* scales, void* y, int64_t M,
+                                         int64_t d, int64_t N, float eps, int out_dtype, int path, void* workspace,
+                                         int64_t workspace_bytes, void* stream);
+
+/*
+ * flashnorm_fp8_workspace_bytes — the workspace flashnorm_linear_fp8_ws uses for this shape on the current
+ * device, written to *bytes: 1024 + slabs x K ranges x (128 x 16 + 16) x 4, or 0 where the split does not
+ * apply (M == 0 or M > FN_DECODE_MAX_M included). FN_ERR_INVALID_ARG for a shape flashnorm_linear_fp8
+ * rejects as invalid (d % 16 != 0, N % 8 != 0, out-of-range sizes).
+ */
+FN_API fn_status flashnorm_fp8_workspace_bytes(int64_t M, int64_t d, int64_t N, int64_t* bytes);
+
+/*
  * flashnorm_rope_table — fills rope_cs (fp32 [max_pos][head_dim / 2][2], caller-owned device memory,
  * 16-byte aligned) with cos and sin of p * base^(-2i/head_dim), computed in double precision and
  * rounded once to fp32. head_dim even, max_pos >= 1, base > 1 (RoFormer uses 10000). Asynchronous on

@@ -35,7 +35,7 @@ __all__ = [
     "flashnorm_fold_layernorm",
     "flashnorm_fold_weights_fp8",
     "flashnorm_linear_fp8",
-    "flashnorm_linear_fp8_ex",
+    "flashnorm_fp8_workspace_bytes",
     "flashnorm_layernorm_linear",
     "flashnorm_rmsnorm",
     "flashnorm_linear_unfused",
@@ -45,6 +45,8 @@ __all__ = [
     "flashnorm_check_device_error",
     "flashnorm_selftest_timeout",
     "flashnorm_version",
+    "prepare",
+    "PreparedCall",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -77,6 +79,8 @@ _SIGNATURES = {
     "flashnorm_fold_weights_fp8": [_P, _P, _P, _P, _I64, _I64, _P],
     "flashnorm_linear_fp8": [_P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_linear_fp8_ex": [_P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _INT, _P],
+    "flashnorm_linear_fp8_ws": [_P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _INT, _P, _I64, _P],
+    "flashnorm_fp8_workspace_bytes": [_I64, _I64, _I64, _P],
     "flashnorm_layernorm_linear": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_rmsnorm": [_P, _P, _P, _I64, _I64, _F, _P],
     "flashnorm_linear_unfused": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
@@ -143,7 +147,16 @@ def _invoke(entry: str, lead: torch.Tensor, *args, report: str | None = None) ->
     _invoke_on(lead.get_device(), entry, *args, report=report)
 
 
+# While prepare() records: the library calls made (size queries excepted) and every tensor whose address
+# was taken, which the prepared call keeps alive.
+_recording = None
+_recording_keep = None
+
+
 def _invoke_on(dev: int, entry: str, *args, report: str | None = None) -> None:
+    if _recording is not None and not entry.endswith("_workspace_bytes"):
+        _recording.append((dev, entry, args, report or entry))
+        return
     lib = load_library()
     if dev == torch.cuda.current_device():
         status = getattr(lib, entry)(*args)
@@ -166,7 +179,57 @@ def _stream_ptr(t: torch.Tensor):
 
 def _ptr(t):
     """A tensor's device address for a void* argument (None passes NULL)."""
-    return t.data_ptr() if t is not None else None
+    if t is None:
+        return None
+    if _recording_keep is not None:
+        _recording_keep.append(t)
+    return t.data_ptr()
+
+
+class PreparedCall:
+    """One library call whose checks and argument marshalling were done once (see prepare). Calling it
+    launches the same C-ABI entry point with the same device pointers on the same stream and returns the
+    output tensor of the original call; it keeps every tensor whose address it holds alive."""
+
+    __slots__ = ("_fn", "_args", "_dev", "_report", "_keep", "result", "entry")
+
+    def __init__(self, fn, args, dev, report, keep, result, entry):
+        self._fn, self._args, self._dev, self._report = fn, args, dev, report
+        self._keep, self.result, self.entry = keep, result, entry
+
+    def __call__(self):
+        if self._dev == torch.cuda.current_device():
+            status = self._fn(*self._args)
+        else:
+            with torch.cuda.device(self._dev):
+                status = self._fn(*self._args)
+        _check(self._report, status)
+        return self.result
+
+
+def prepare(func, *args, **kwargs) -> PreparedCall:
+    """Plan once, launch many: run func(*args, **kwargs), one of this module's calls that launch work (a
+    projection, a fold, the RMSNorm), for its checks and argument marshalling only, and return a
+    PreparedCall that launches that call again at the cost of one C call. For loops that repeat one call
+    on the same buffers (a serving step, a benchmark). What is fixed at this point: the device addresses
+    (rewrite the inputs in place, and read the outputs from .result), the stream (the one current now),
+    and any scratch the call chose (a workspace="auto" buffer is allocated here and kept)."""
+    global _recording, _recording_keep
+    if _recording is not None:
+        raise RuntimeError("prepare() does not nest")
+    rec, keep = [], []
+    _recording, _recording_keep = rec, keep
+    try:
+        result = func(*args, **kwargs)
+    finally:
+        _recording, _recording_keep = None, None
+    if len(rec) != 1:
+        raise ValueError(f"prepare() takes a call that makes one library call; this one made {len(rec)}")
+    dev, entry, cargs, report = rec[0]
+    f = getattr(load_library(), entry)
+    # ctypes skips its per-call conversion for arguments that already have the declared types
+    conv = tuple(a if isinstance(a, t) else t(a) for t, a in zip(f.argtypes, cargs))
+    return PreparedCall(f, conv, dev, report, keep, result, entry)
 
 
 def _need(t: torch.Tensor, name: str, dtype=torch.bfloat16, dim=None) -> None:
@@ -314,12 +377,47 @@ def flashnorm_fold_weights_fp8(W: torch.Tensor, g: torch.Tensor):
     return Q, scales
 
 
+_fp8_ws_bytes_cache = {}
+_fp8_ws_cache = {}
+
+
+def flashnorm_fp8_workspace_bytes(M: int, d: int, N: int, device=None) -> int:
+    """Workspace bytes flashnorm_linear_fp8 uses for this shape on `device` (0: no split)."""
+    dev = torch.cuda.current_device() if device is None else torch.device(device).index
+    if dev is None:
+        dev = torch.cuda.current_device()
+    key = (dev, int(M), int(d), int(N))
+    hit = _fp8_ws_bytes_cache.get(key)
+    if hit is not None:
+        return hit
+    nbytes = ctypes.c_int64(0)
+    _invoke_on(dev, "flashnorm_fp8_workspace_bytes", int(M), int(d), int(N), ctypes.addressof(nbytes))
+    _fp8_ws_bytes_cache[key] = int(nbytes.value)  # a function of the shape and the device's SM count only
+    return int(nbytes.value)
+
+
+def _fp8_stream_workspace(x: torch.Tensor, nbytes: int) -> torch.Tensor:
+    """A zero-initialised workspace of at least `nbytes` kept for x's device and current stream. Calls on
+    one stream run in order, and each leaves the workspace's counters at zero, so they can share it."""
+    key = (x.get_device(), _stream_ptr(x))
+    ws = _fp8_ws_cache.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=x.device)
+        _fp8_ws_cache[key] = ws
+    return ws
+
+
 def flashnorm_linear_fp8(x: torch.Tensor, Q: torch.Tensor, scales: torch.Tensor, eps: float,
-                         out_dtype=torch.bfloat16, out=None, path: str = "auto") -> torch.Tensor:
+                         out_dtype=torch.bfloat16, out=None, path: str = "auto", workspace="auto") -> torch.Tensor:
     """Decode (M <= 16) with FP8 weights: y = (x . dec(Q)^T) * scales * 1/sqrt(mean(x^2) + eps).
 
-    path "decode": the tensor-core kernel; "gemv": the CUDA-core GEMV; "auto": the GEMV for one token, the
-    tensor-core kernel for more."""
+    path "decode": the tensor-core kernel; "gemv": the CUDA-core GEMV; "auto": the tensor-core kernel,
+    except for one token without a workspace (the GEMV).
+    workspace: "auto" uses a zero-initialised scratch kept per device and stream, which lets the
+    tensor-core kernel split its contraction over independent CTAs (flashnorm_fp8_workspace_bytes; nothing
+    for shapes that do not split); None runs without one (the split then stays inside thread-block
+    clusters); or a caller-owned uint8 CUDA tensor of at least that many bytes whose first 1024 bytes were
+    zero before its first use (every call leaves them zero)."""
     _need(x, "x", dim=2)
     _need(Q, "Q", torch.uint8, dim=2)
     _need(scales, "scales", torch.float32, dim=1)
@@ -329,8 +427,20 @@ def flashnorm_linear_fp8(x: torch.Tensor, Q: torch.Tensor, scales: torch.Tensor,
         raise ValueError("Q [N, d] and scales [N] must match x [M, d]")
     _same_device(x, Q=Q, scales=scales)
     y = _output(out, (M, N), out_dtype, x)
-    _invoke("flashnorm_linear_fp8_ex", x, _ptr(x), _ptr(Q), _ptr(scales), _ptr(y), M, d, N, float(eps),
-            _out_code(out_dtype), PATHS[path], _stream_ptr(x), report="flashnorm_linear_fp8")
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError('workspace must be "auto", None or a uint8 CUDA tensor')
+        nbytes = flashnorm_fp8_workspace_bytes(M, d, N, x.get_device()) if 0 < M <= 16 else 0
+        ws = _fp8_stream_workspace(x, nbytes) if nbytes > 0 else None
+    elif workspace is None:
+        ws = None
+    else:
+        _need(workspace, "workspace", torch.uint8, dim=1)
+        _same_device(x, workspace=workspace)
+        ws = workspace
+    _invoke("flashnorm_linear_fp8_ws", x, _ptr(x), _ptr(Q), _ptr(scales), _ptr(y), M, d, N, float(eps),
+            _out_code(out_dtype), PATHS[path], _ptr(ws), ws.numel() if ws is not None else 0, _stream_ptr(x),
+            report="flashnorm_linear_fp8")
     return y
 
 

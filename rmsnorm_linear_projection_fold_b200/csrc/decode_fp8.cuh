@@ -18,13 +18,19 @@
 // Per CTA, one slab of 128 W* rows (the MMA's M side; the <= 16 tokens are its N side) over one range
 // of K, in stages of 128 k (128 codes per W* row, 16 KB, and 16 x 128 bf16 of x, 4 KB):
 //   warp 0      TMA producer
-//   warp 1      tensor-memory allocator; one lane issues the MMAs (A from tensor memory, B = the x tile)
+//   warp 1      tensor-memory allocator; lane 0 issues the MMAs of every kD8Issuers-th stage (A from
+//               tensor memory, B = the x tile); warps 6.. issue the others'
 //   warps 2-5   converters: each thread widens its W* row of a stage to bf16 into an A buffer in tensor
 //               memory (tcgen05.st) and adds up x^2 for one token over 16 of the stage's k (the
 //               deferred norm, from the same staged x tiles the MMA reads); then the epilogue
 // A stage is refilled once the converters have read it and the MMA that read its x tile has completed.
-// When there are few slabs, K is split across a cluster of `ksplit` CTAs; the partial accumulators and
-// sums of squares are added in the leader CTA through distributed shared memory, in a fixed order.
+// When there are few slabs, K is split in `ksplit` ranges, one CTA each. Either the CTAs of a slab form a
+// cluster and the partial accumulators and sums of squares are added in the leader CTA through
+// distributed shared memory (KSPLIT > 1), or (KSPLIT == 0, a caller workspace) they are independent CTAs
+// that write their partials to the workspace and count their arrivals on the slab's counter: the CTA
+// that arrives last adds the partials in K order and writes the output. Nothing waits on another CTA,
+// the sum is in a fixed order whichever CTA comes last, and the ranges need no co-scheduling, so two
+// 5-stage CTAs can share every SM.
 #pragma once
 
 #include "sm100.cuh"
@@ -38,11 +44,26 @@ constexpr int kD8WStage = kD8Rows * kD8KStage;     // 16 KB of codes
 constexpr int kD8XStage = kD8Tok * kD8KStage * 2;  // 4 KB of x: two 64-k atoms of 16 rows x 128 bytes
 constexpr int kD8ABufs = 3;                        // bf16 A tiles in tensor memory, 64 columns each
 constexpr int kD8ACol0 = 64;                       // first A column (the accumulators take columns 0..63)
-// Independent accumulators: MMA j of a stage goes to accumulator j % 4, the four summed in the epilogue
-// in a fixed order. MMAs of N = 16 into one accumulator form a dependent chain that runs at about one
-// per 150 cycles, which alone made this kernel take 0.75 us per 128-k stage; four chains overlap.
+// MMA issuers: stage i of a CTA's K range is issued by issuer i % kD8Issuers, into that issuer's own
+// kD8Accs / kD8Issuers accumulators (MMA j of the stage into the issuer's accumulator j % that count);
+// the epilogue adds the kD8Accs accumulators in a fixed order. One thread issuing back-to-back
+// M = 128, N = 16 MMAs gets one through every ~60 cycles, and every ~125 while other warps store to
+// tensor memory (the converters do): per-issuer cost, not tensor-core throughput, so issuers in
+// separate warps overlap almost linearly.
 constexpr int kD8Accs = 4;
-constexpr int kD8Threads = 192;
+constexpr int kD8Issuers = 2;
+constexpr int kD8AccPer = kD8Accs / kD8Issuers;
+static_assert(kD8Accs % kD8Issuers == 0, "each issuer owns the same number of accumulators");
+// The issuer of stage i + kD8ABufs (which reuses stage i's A buffer) last waited on stage
+// i + kD8ABufs - kD8Issuers; that must not come before stage i, or its parity wait on the buffer's
+// barrier could see stage i's phase, one phase early. Likewise for the stage ring (at least 4 stages).
+static_assert(kD8Issuers <= kD8ABufs && kD8Issuers <= 4, "an issuer would run a barrier phase ahead");
+// warp 0 TMA, warp 1 allocator + issuer 0, warps 2-5 converters, warps 6.. issuers 1..
+constexpr int kD8Threads = 192 + 32 * (kD8Issuers - 1);
+// Workspace of the KSPLIT == 0 kernel: kD8MaxWsSlabs arrival counters (uint32), then the partials
+// [slab][range][128 rows][16 tokens] fp32, then the partial sums of squares [slab][range][16] fp32.
+constexpr int kD8MaxWsSlabs = 256;
+constexpr int kD8WsCounterBytes = kD8MaxWsSlabs * 4;
 
 struct DecodeFp8Params {
   void* y;
@@ -50,6 +71,9 @@ struct DecodeFp8Params {
   int M, K, N, ldy;
   int ksplit;
   float eps;
+  unsigned* counters;  // KSPLIT == 0: one per slab, zero between calls
+  float* part;         // KSPLIT == 0: [slabs][ksplit][128][16]
+  float* part_ss;      // KSPLIT == 0: [slabs][ksplit][16]
 };
 
 template <int STAGES, int KSPLIT>
@@ -114,19 +138,21 @@ __global__ void __launch_bounds__(kD8Threads, 1)
   uint64_t* afull = empty + STAGES;
   uint64_t* aempty = afull + kD8ABufs;
   uint64_t* acc_full = aempty + kD8ABufs;
-  uint64_t* drain = acc_full + 1;
-  float* rs = reinterpret_cast<float*>(drain + 1);  // [16] 1/rms per token (leader)
+  uint64_t* drain = acc_full + 1;                             // [kD8Issuers]
+  float* rs = reinterpret_cast<float*>(drain + kD8Issuers);  // [16] 1/rms per token (leader)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rs + kD8Tok);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;  // KSPLIT == 0: this CTA arrived last on its slab
 
   const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x) >> 5, 0);
   const int lane = static_cast<int>(threadIdx.x) & 31;
-  const uint32_t rank = KSPLIT > 1 ? cluster_ctarank() : 0;
-  const int slab = static_cast<int>(blockIdx.x) / KSPLIT;
+  const int ks = KSPLIT == 0 ? p.ksplit : KSPLIT;  // K ranges per slab
+  const uint32_t rank = KSPLIT == 0 ? blockIdx.x % static_cast<uint32_t>(ks) : (KSPLIT > 1 ? cluster_ctarank() : 0);
+  const int slab = static_cast<int>(blockIdx.x) / ks;
   const int n0 = slab * kD8Rows;
   const int num_units = (p.K + kD8KStage - 1) / kD8KStage;  // stages of 128 over all of K
-  const int u0 = static_cast<int>((static_cast<long long>(rank) * num_units) / KSPLIT);
-  const int u1 = static_cast<int>((static_cast<long long>(rank + 1) * num_units) / KSPLIT);
+  const int u0 = static_cast<int>((static_cast<long long>(rank) * num_units) / ks);
+  const int u1 = static_cast<int>((static_cast<long long>(rank + 1) * num_units) / ks);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -137,8 +163,8 @@ __global__ void __launch_bounds__(kD8Threads, 1)
       mbar_init(&afull[b], 4);   // the four converter warps
       mbar_init(&aempty[b], 1);  // the MMA's commit
     }
-    mbar_init(acc_full, 1);
-    mbar_init(drain, 1);
+    mbar_init(acc_full, kD8Issuers);  // each issuer's last commit
+    for (int i = 0; i < kD8Issuers; ++i) mbar_init(&drain[i], 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -205,14 +231,16 @@ __global__ void __launch_bounds__(kD8Threads, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp >= 6) {
+    // ------------------------------------------------------------------ MMA issuers
+    const int iss = warp == 1 ? 0 : warp - 5;  // stages iss, iss + kD8Issuers, ... of this CTA's range
     if (lane == 0) {
       const uint32_t idesc = make_idesc_bf16(kD8Rows, kD8Tok);
-      int s = 0, b = 0;
-      uint32_t ph = 0, bph = 0;
+      const uint32_t acc0 = tmem_base + static_cast<uint32_t>(iss * kD8AccPer * kD8Tok);
       bool ok = true;
-      for (int u = u0; u < u1; ++u) {
+      for (int i = iss; u0 + i < u1; i += kD8Issuers) {
+        const int s = i % STAGES, b = i % kD8ABufs;
+        const uint32_t ph = static_cast<uint32_t>(i / STAGES) & 1u, bph = static_cast<uint32_t>(i / kD8ABufs) & 1u;
         // the x tile of this stage (TMA) and the widened codes in A buffer b (the converters)
         if (!mbar_wait(&full[s], ph, abort_flag) || !mbar_wait(&afull[b], bph, abort_flag)) {
           ok = false;
@@ -223,24 +251,16 @@ __global__ void __launch_bounds__(kD8Threads, 1)
         const uint32_t x_st = smem_u32(sX + s * kD8XStage);
 #pragma unroll
         for (int j = 0; j < kD8KStage / 16; ++j)  // 8 MMAs of K = 16: 8 columns of A, 32 bytes of a B row
-          tc_mma_bf16_ts(tmem_base + static_cast<uint32_t>((j % kD8Accs) * kD8Tok), a_col + j * 8,
+          tc_mma_bf16_ts(acc0 + static_cast<uint32_t>((j % kD8AccPer) * kD8Tok), a_col + j * 8,
                          make_sdesc_sw128(x_st + (j >> 2) * 2048 + (j & 3) * 32), idesc,
-                         (u != u0 || j >= kD8Accs) ? 1u : 0u);
+                         (i != iss || j >= kD8AccPer) ? 1u : 0u);
         tc_commit(&aempty[b]);  // A buffer b may be refilled once these MMAs have read it
         tc_commit(&empty[s]);   // and the stage, whose x tile they read
-        if (++s == STAGES) {
-          s = 0;
-          ph ^= 1u;
-        }
-        if (++b == kD8ABufs) {
-          b = 0;
-          bph ^= 1u;
-        }
       }
-      tc_commit(ok ? acc_full : drain);
+      tc_commit(ok ? acc_full : &drain[iss]);
       if (!ok) {
         const unsigned long long t0 = globaltimer_ns();
-        while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+        while (!mbar_try_wait(&drain[iss], 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
         }
       }
     }
@@ -255,6 +275,8 @@ __global__ void __launch_bounds__(kD8Threads, 1)
     uint32_t ph = 0, bph = 0;
     bool ok = true;
     float ss = 0.f;
+    // this row's dequantization scale, loaded now so that its latency hides under the main loop
+    const float sc = n0 + row < p.N ? p.scales[n0 + row] : 0.f;
     for (int u = u0; u < u1; ++u) {
       if (!mbar_wait(&full[s], ph, abort_flag) || !mbar_wait(&aempty[b], bph ^ 1u, abort_flag)) {
         ok = false;
@@ -330,9 +352,13 @@ __global__ void __launch_bounds__(kD8Threads, 1)
       reg_fence16(r1);
       reg_fence16(r2);
       reg_fence16(r3);
+      // accumulator a belongs to issuer a / kD8AccPer, which wrote it only if this range has a stage for it
+      const int nst = u1 - u0;
+      const bool w0 = nst > 0 / kD8AccPer, w1 = nst > 1 / kD8AccPer, w2 = nst > 2 / kD8AccPer, w3 = nst > 3 / kD8AccPer;
 #pragma unroll
       for (int j = 0; j < kD8Tok; ++j)
-        v[j] = (__uint_as_float(r0[j]) + __uint_as_float(r1[j])) + (__uint_as_float(r2[j]) + __uint_as_float(r3[j]));
+        v[j] = ((w0 ? __uint_as_float(r0[j]) : 0.f) + (w1 ? __uint_as_float(r1[j]) : 0.f)) +
+               ((w2 ? __uint_as_float(r2[j]) : 0.f) + (w3 ? __uint_as_float(r3[j]) : 0.f));
     } else {
       // an empty K range contributes zero; a wait that gave up contributes NaN
 #pragma unroll
@@ -345,7 +371,53 @@ __global__ void __launch_bounds__(kD8Threads, 1)
       if (sub == 0) dsmem_st_f32(dsmem_addr(part_ss + rank * kD8Tok + tok, 0), ss);
     }
     if (KSPLIT > 1) cluster_sync_all();  // the partial sums have reached the leader
-    if (rank == 0) {
+    bool writer = rank == 0;  // this CTA writes the slab's output
+    if (KSPLIT == 0 && ks > 1) {
+      // this range's partials to the workspace, then count the arrival; the last of the slab's ranges
+      // to arrive adds them all, range 0 first (the same order whichever range comes last)
+      const size_t rec = static_cast<size_t>(slab) * static_cast<size_t>(ks);  // the slab's first record
+      float* mine = p.part + ((rec + rank) * kD8Rows + row) * kD8Tok;
+#pragma unroll
+      for (int j = 0; j < kD8Tok; j += 4)
+        __stcg(reinterpret_cast<float4*>(mine + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
+      if (sub == 0) __stcg(p.part_ss + (rec + rank) * kD8Tok + tok, ss);
+      named_bar_sync(1, 128);  // the CTA's partials come before its arrival (barrier, then release)
+      if (t == 0) {
+        // acquire-release at GPU scope: releases this CTA's partials, and for the last arrival acquires
+        // the other ranges' (each released by its own arrival); the barrier below passes that on
+        const bool last = atom_add_acq_rel_gpu(p.counters + slab, 1u) == static_cast<unsigned>(ks - 1);
+        if (last) st_relaxed_gpu(p.counters + slab, 0u);  // every range has arrived: zero for the next call
+        *last_flag = last ? 1 : 0;
+      }
+      named_bar_sync(1, 128);
+      writer = *last_flag != 0;
+      if (writer) {
+        float tot[kD8Tok];
+        float sst = 0.f;
+        for (int rr = 0; rr < ks; ++rr) {
+          float q[kD8Tok];
+          if (rr == static_cast<int>(rank)) {
+#pragma unroll
+            for (int j = 0; j < kD8Tok; ++j) q[j] = v[j];
+          } else {
+            const float* src = p.part + ((rec + rr) * kD8Rows + row) * kD8Tok;
+#pragma unroll
+            for (int j = 0; j < kD8Tok; j += 4) {
+              const float4 f = __ldcg(reinterpret_cast<const float4*>(src + j));
+              q[j] = f.x, q[j + 1] = f.y, q[j + 2] = f.z, q[j + 3] = f.w;
+            }
+          }
+          const float qs = rr == static_cast<int>(rank) ? ss : (sub == 0 ? __ldcg(p.part_ss + (rec + rr) * kD8Tok + tok) : 0.f);
+#pragma unroll
+          for (int j = 0; j < kD8Tok; ++j) tot[j] = rr == 0 ? q[j] : tot[j] + q[j];
+          sst = rr == 0 ? qs : sst + qs;
+        }
+#pragma unroll
+        for (int j = 0; j < kD8Tok; ++j) v[j] = tot[j];
+        ss = sst;
+      }
+    }
+    if (writer) {
       if (KSPLIT > 1) {
         for (int rr = 1; rr < KSPLIT; ++rr) {
 #pragma unroll
@@ -357,7 +429,6 @@ __global__ void __launch_bounds__(kD8Threads, 1)
       named_bar_sync(1, 128);
       const int n = n0 + row;
       if (n < p.N) {
-        const float sc = p.scales[n];
 #pragma unroll
         for (int m = 0; m < kD8Tok; ++m) {
           if (m >= p.M) break;
@@ -371,7 +442,7 @@ __global__ void __launch_bounds__(kD8Threads, 1)
       }
     }
   }
-  if (KSPLIT > 1 && warp < 2) cluster_sync_all();
+  if (KSPLIT > 1 && (warp < 2 || warp >= 6)) cluster_sync_all();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();

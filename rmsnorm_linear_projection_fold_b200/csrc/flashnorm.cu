@@ -703,25 +703,52 @@ fn_status launch_decode_fp8_t(const CUtensorMap& tq, const CUtensorMap& tx, cons
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (fp8 decode)");
     configured[dev] = true;
   }
-  cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(slabs * KSPLIT)), dim3(fn::kD8Threads), smem, stream,
-                                KSPLIT, tq, tx, p);
+  // KSPLIT == 0: p.ksplit independent CTAs per slab (no cluster)
+  const int ks = KSPLIT == 0 ? p.ksplit : KSPLIT;
+  cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(slabs * ks)), dim3(fn::kD8Threads), smem, stream,
+                                KSPLIT == 0 ? 1 : KSPLIT, tq, tx, p);
   if (e != cudaSuccess) return cuda_fail(e, "fp8 decode launch");
   return FN_OK;
 }
 
+// K ranges per slab of the FP8 decode kernel with a workspace: enough independent CTAs for two on every
+// SM (each holds 5 stages: two fit one SM's shared and tensor memory), while there are at most as many
+// slabs as SMs; 1 (no split, no workspace) otherwise.
+int fp8_ws_ksplit(int64_t N, int64_t d, int sms) {
+  const int64_t slabs = (N + fn::kD8Rows - 1) / fn::kD8Rows;
+  const int64_t units = (d + fn::kD8KStage - 1) / fn::kD8KStage;
+  if (slabs > fn::kD8MaxWsSlabs || slabs > sms) return 1;
+  int64_t ks = (2 * static_cast<int64_t>(sms)) / slabs;
+  ks = std::min<int64_t>(std::min<int64_t>(ks, units), 16);
+  return ks >= 2 ? static_cast<int>(ks) : 1;
+}
+
+int64_t fp8_ws_bytes(int64_t N, int ks) {
+  if (ks < 2) return 0;
+  const int64_t slabs = (N + fn::kD8Rows - 1) / fn::kD8Rows;
+  return fn::kD8WsCounterBytes + slabs * ks * (fn::kD8Rows * fn::kD8Tok + fn::kD8Tok) * 4;
+}
+
 fn_status run_decode_fp8(const void* x, const void* q, const void* scales, void* y, int64_t M, int64_t d, int64_t N,
-                         float eps, int out_dtype, cudaStream_t stream) {
+                         float eps, int out_dtype, void* workspace, cudaStream_t stream) {
   int dev = 0;
   const int sms = device_sm_count(&dev);
   if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
   const int64_t slabs = (N + fn::kD8Rows - 1) / fn::kD8Rows;
   const int64_t units = (d + fn::kD8KStage - 1) / fn::kD8KStage;
-  // K split as for the bf16 decode kernel: in two while there are at most as many slabs as SMs (two
-  // 5-stage CTAs fit one SM), in four when there are few slabs; otherwise one 10-stage CTA per slab.
-  // (In three, two 4-stage CTAs on every SM, the Llama-7B QKV codes took 23.9 us against 17.3 us.)
+  // With a workspace: K in fp8_ws_ksplit ranges of independent CTAs, two on every SM. Without one, K is
+  // split in a cluster as for the bf16 decode kernel: in two while there are at most as many slabs as SMs
+  // (two 5-stage CTAs fit one SM), in four when there are few slabs; otherwise one 10-stage CTA per slab.
+  // (A cluster of three, two 4-stage CTAs on every SM, took 23.9 us against 17.3 us on the Llama-7B QKV
+  // codes: clusters of three do not all fit at once.)
   int ksplit = 1;
-  if (slabs <= sms && units >= 2) ksplit = 2;
-  if (slabs * 4 <= sms && units >= 4) ksplit = 4;
+  const int ws_ks = workspace != nullptr ? fp8_ws_ksplit(N, d, sms) : 1;
+  if (ws_ks >= 2) {
+    ksplit = ws_ks;
+  } else {
+    if (slabs <= sms && units >= 2) ksplit = 2;
+    if (slabs * 4 <= sms && units >= 4) ksplit = 4;
+  }
   CUtensorMap tq, tx;
   fn_status st = make_u8_map(&tq, q, d, N, fn::kD8Rows);
   if (st != FN_OK) return st;
@@ -736,11 +763,19 @@ fn_status run_decode_fp8(const void* x, const void* q, const void* scales, void*
   p.ldy = static_cast<int>(N);
   p.ksplit = ksplit;
   p.eps = eps;
+  p.counters = nullptr;
+  p.part = p.part_ss = nullptr;
   const int sl = static_cast<int>(slabs);
   const bool f32 = out_dtype == FN_F32;
 #define FN_D8(ST, KS)                                                                                          \
   (f32 ? launch_decode_fp8_t<ST, KS, true>(tq, tx, p, sl, dev, stream)                                         \
        : launch_decode_fp8_t<ST, KS, false>(tq, tx, p, sl, dev, stream))
+  if (ws_ks >= 2) {
+    p.counters = static_cast<unsigned*>(workspace);
+    p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + fn::kD8WsCounterBytes);
+    p.part_ss = p.part + slabs * ksplit * fn::kD8Rows * fn::kD8Tok;
+    return FN_D8(5, 0);
+  }
   if (ksplit == 1) return FN_D8(10, 1);
   if (ksplit == 2) return FN_D8(5, 2);
   return FN_D8(4, 4);
@@ -1039,8 +1074,24 @@ fn_status flashnorm_fold_weights_fp8(const void* W, const void* g, void* Q, void
   return FN_OK;
 }
 
-fn_status flashnorm_linear_fp8_ex(const void* x, const void* Q, const void* scales, void* y, int64_t M, int64_t d,
-                                  int64_t N, float eps, int out_dtype, int path, void* stream) {
+fn_status flashnorm_fp8_workspace_bytes(int64_t M, int64_t d, int64_t N, int64_t* bytes) {
+  g_last_error[0] = '\0';
+  if (bytes == nullptr) return fail(FN_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = 0;
+  if (M < 0 || M > kMaxDim) return fail(FN_ERR_INVALID_ARG, "M = %lld out of range", (long long)M);
+  if (d < 16 || d > kMaxDim || d % 16 != 0) return fail(FN_ERR_INVALID_ARG, "d = %lld must be a positive multiple of 16", (long long)d);
+  if (N < 8 || N > kMaxDim || N % 8 != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a positive multiple of 8", (long long)N);
+  if (M == 0 || M > FN_DECODE_MAX_M) return FN_OK;
+  int dev = 0;
+  const int sms = device_sm_count(&dev);
+  if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
+  *bytes = fp8_ws_bytes(N, fp8_ws_ksplit(N, d, sms));
+  return FN_OK;
+}
+
+fn_status flashnorm_linear_fp8_ws(const void* x, const void* Q, const void* scales, void* y, int64_t M, int64_t d,
+                                  int64_t N, float eps, int out_dtype, int path, void* workspace,
+                                  int64_t workspace_bytes, void* stream) {
   g_last_error[0] = '\0';
   if (path != FN_PATH_AUTO && path != FN_PATH_DECODE && path != FN_PATH_GEMV)
     return fail(FN_ERR_INVALID_ARG, "fp8 path %d: AUTO, DECODE or GEMV", path);
@@ -1050,12 +1101,27 @@ fn_status flashnorm_linear_fp8_ex(const void* x, const void* Q, const void* scal
   if (N < 8 || N > kMaxDim || N % 8 != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a positive multiple of 8", (long long)N);
   if (M > FN_DECODE_MAX_M) return fail(FN_ERR_UNSUPPORTED, "the fp8 path is the decode GEMV: M <= %d", FN_DECODE_MAX_M);
   if ((st = check_ptr(scales, "scales")) != FN_OK) return st;
+  if (workspace_bytes < 0) return fail(FN_ERR_INVALID_ARG, "workspace_bytes is negative");
   if (M == 0) return FN_OK;
-  // AUTO: one token on the CUDA-core GEMV (16.2 us for the Llama-7B QKV codes against 18.0 us on the
-  // tensor cores), more on the tensor-core kernel, whose time does not grow with M (the GEMV's does: 29 us
-  // at 4 tokens, 125 us at 16).
-  if (path == FN_PATH_DECODE || (path == FN_PATH_AUTO && M > 1))
-    return run_decode_fp8(x, Q, scales, y, M, d, N, eps, out_dtype, static_cast<cudaStream_t>(stream));
+  void* ws = nullptr;  // the workspace, where the tensor-core kernel's K split uses one for this shape
+  if (workspace != nullptr && path != FN_PATH_GEMV) {
+    int dev = 0;
+    const int sms = device_sm_count(&dev);
+    if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
+    const int64_t need = fp8_ws_bytes(N, fp8_ws_ksplit(N, d, sms));
+    if (need > 0) {
+      if (workspace_bytes < need)
+        return fail(FN_ERR_INVALID_ARG, "workspace of %lld bytes; this shape needs %lld", (long long)workspace_bytes,
+                    (long long)need);
+      if ((st = check_ptr(workspace, "workspace")) != FN_OK) return st;
+      ws = workspace;
+    }
+  }
+  // AUTO: the tensor-core kernel, whose time does not grow with M (the GEMV's does: 29 us at 4 tokens,
+  // 125 us at 16), except for one token without a workspace, where the CUDA-core GEMV (16.2 us for the
+  // Llama-7B QKV codes) beats the cluster-split kernel (18.0 us).
+  if (path == FN_PATH_DECODE || (path == FN_PATH_AUTO && (M > 1 || ws != nullptr)))
+    return run_decode_fp8(x, Q, scales, y, M, d, N, eps, out_dtype, ws, static_cast<cudaStream_t>(stream));
   if (!gemv_fits(M, d)) return fail(FN_ERR_UNSUPPORTED, "x [%lld, %lld] does not fit in shared memory", (long long)M, (long long)d);
   int dev = 0;
   const int sms = device_sm_count(&dev);
@@ -1073,6 +1139,11 @@ fn_status flashnorm_linear_fp8_ex(const void* x, const void* Q, const void* scal
     default: return FN_G8(16, 1);
   }
 #undef FN_G8
+}
+
+fn_status flashnorm_linear_fp8_ex(const void* x, const void* Q, const void* scales, void* y, int64_t M, int64_t d,
+                                  int64_t N, float eps, int out_dtype, int path, void* stream) {
+  return flashnorm_linear_fp8_ws(x, Q, scales, y, M, d, N, eps, out_dtype, path, nullptr, 0, stream);
 }
 
 fn_status flashnorm_linear_fp8(const void* x, const void* Q, const void* scales, void* y, int64_t M, int64_t d,

@@ -257,6 +257,17 @@ __device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk
 // Every committed bulk store complete (its writes performed), not only its shared-memory reads.
 __device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Atomic add with acquire-release semantics at GPU scope; returns the previous value.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ void st_relaxed_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Programmatic dependent launch. A kernel launched with programmatic stream serialization may start
 // while the previous kernel in its stream is still running: it sets up its barriers and tensor memory,
 // then waits here until that kernel has completed and its writes are visible, before touching global

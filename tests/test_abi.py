@@ -164,7 +164,7 @@ def test_layernorm_validation(lib):
     assert lib.flashnorm_fold_layernorm(P, P, P, P, P, NULL, 64, 64, NULL) == fn.FN_ERR_INVALID_ARG
 
 
-def test_fp8_validation(lib):
+def test_fp8_fold_validation(lib):
     assert lib.flashnorm_fold_weights_fp8(P, P, P, P, 24, 64, NULL) == fn.FN_ERR_INVALID_ARG   # d % 16
     assert lib.flashnorm_fold_weights_fp8(P, P, P, P, 64, 60, NULL) == fn.FN_ERR_INVALID_ARG   # N % 8
     assert lib.flashnorm_linear_fp8(P, P, P, P, 17, 64, 64, 1e-6, 0, NULL) == fn.FN_ERR_UNSUPPORTED  # M > 16
@@ -243,3 +243,43 @@ def test_noalloc_validation(lib, args, expected):
 ])
 def test_fp8_validation(lib, args, expected):
     assert lib.flashnorm_linear_fp8_ex(*args) == expected
+
+
+def test_fp8_workspace_validation(lib):
+    """The workspace entry point validates like flashnorm_linear_fp8_ex before it looks at the device,
+    and its size query rejects shapes the call would reject (no device needed for either)."""
+    ws = fn._SIGNATURES["flashnorm_linear_fp8_ws"]
+    assert len(ws) == 13
+    assert lib.flashnorm_linear_fp8_ws(P, P, P, P, 4, 576, 960, 1e-6, 0, 9, NULL, 0, NULL) == fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_linear_fp8_ws(P, P, P, P, 17, 576, 960, 1e-6, 0, 0, NULL, 0, NULL) == fn.FN_ERR_UNSUPPORTED
+    assert lib.flashnorm_linear_fp8_ws(P, P, P, P, 4, 584, 960, 1e-6, 0, 3, NULL, 0, NULL) == fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_linear_fp8_ws(P, P, P, P, 4, 576, 960, 1e-6, 0, 3, P, -1, NULL) == fn.FN_ERR_INVALID_ARG
+    assert lib.flashnorm_linear_fp8_ws(P, P, P, P, 0, 576, 960, 1e-6, 0, 3, P, 16, NULL) == fn.FN_OK
+    nbytes = ctypes.c_int64(-7)
+    out = ctypes.c_void_p(ctypes.addressof(nbytes))
+    assert lib.flashnorm_fp8_workspace_bytes(4, 4096, 12288, NULL) == fn.FN_ERR_INVALID_ARG
+    for shape in [(4, 4104, 12288), (4, 4096, 12284), (-1, 4096, 12288), (4, 0, 12288)]:
+        assert lib.flashnorm_fp8_workspace_bytes(*shape, out) == fn.FN_ERR_INVALID_ARG, shape
+    # an empty call and M above the decode limit need nothing (and no device to say so)
+    for shape in [(0, 4096, 12288), (17, 4096, 12288)]:
+        nbytes.value = -7
+        assert lib.flashnorm_fp8_workspace_bytes(*shape, out) == fn.FN_OK
+        assert nbytes.value == 0
+
+
+def test_binding_names_resolve():
+    """Every name the package exports exists (a star import would fail otherwise)."""
+    for name in fn.__all__:
+        assert hasattr(fn, name), name
+
+
+def test_prepare_propagates_errors_and_resets():
+    """prepare() runs the call's own checks: a rejected call raises as it would directly, and leaves no
+    recording state behind (a second prepare is not taken for a nested one)."""
+    import torch
+
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    for _ in range(2):
+        with pytest.raises((ValueError, TypeError, fn.FlashNormError)):
+            fn.prepare(fn.flashnorm_linear, x, x, 1e-5)
+    assert fn._recording is None and fn._recording_keep is None

@@ -33,15 +33,21 @@ def test_fold_fp8_zero_channel():
     assert s[5].item() == 1.0 and int(Q[5].abs().sum().item()) == 0
 
 
-@pytest.mark.parametrize("path", ["decode", "gemv"])
+# (path, workspace): the tensor-core kernel with its contraction split over independent CTAs through a
+# workspace ("auto") or inside thread-block clusters (None); the CUDA-core GEMV
+PATHS_WS = [("decode", "auto"), ("decode", None), ("gemv", None)]
+
+
+@pytest.mark.parametrize("path,workspace", PATHS_WS)
 @pytest.mark.parametrize("M,d,N", [(1, 4096, 1024), (3, 576, 960), (4, 4096, 2048), (7, 208, 136), (16, 576, 512),
-                                   (2, 64, 8), (16, 4096, 12288), (5, 400, 200), (5, 1008, 6000)])
-def test_linear_fp8_parity(M, d, N, path):
+                                   (2, 64, 8), (16, 4096, 12288), (5, 400, 200), (5, 1008, 6000), (1, 4096, 20480),
+                                   (9, 2048, 128), (4, 128, 12288)])
+def test_linear_fp8_parity(M, d, N, path, workspace):
     bits = I.Workload("t", "linear_fp8", M, d, N, 1e-6, seed=M * 13 + d).draw()
     Q, s = fn.flashnorm_fold_weights_fp8(to_dev(bits["w"]), to_dev(bits["g"]))
     x = to_dev(bits["x"])
-    y16 = fn.flashnorm_linear_fp8(x, Q, s, 1e-6, path=path)
-    y32 = fn.flashnorm_linear_fp8(x, Q, s, 1e-6, out_dtype=torch.float32, path=path)
+    y16 = fn.flashnorm_linear_fp8(x, Q, s, 1e-6, path=path, workspace=workspace)
+    y32 = fn.flashnorm_linear_fp8(x, Q, s, 1e-6, out_dtype=torch.float32, path=path, workspace=workspace)
     torch.cuda.synchronize()
     ex = O.exact_operand_fp8(bits, 1e-6)
     ref = O.reference_output("linear", bits, 1e-6)  # the unquantized definition
@@ -52,14 +58,15 @@ def test_linear_fp8_parity(M, d, N, path):
     assert O.rel_err(ex, ref) <= 5e-2
 
 
-@pytest.mark.parametrize("path", ["decode", "gemv"])
+@pytest.mark.parametrize("path,workspace", PATHS_WS)
 @pytest.mark.parametrize("name", ["llama7b_qkv_fp8_m1", "llama7b_qkv_fp8_m4", "llama7b_qkv_fp8_m16"])
-def test_linear_fp8_full_size(name, path):
+def test_linear_fp8_full_size(name, path, workspace):
     """The Llama-7B QKV decode shapes the benchmark runs, every output against the quantized operands."""
     wl = I.WORKLOADS[name]
     bits = wl.draw()
     Q, s = fn.flashnorm_fold_weights_fp8(to_dev(bits["w"]), to_dev(bits["g"]))
-    y32 = fn.flashnorm_linear_fp8(to_dev(bits["x"]), Q, s, wl.eps, out_dtype=torch.float32, path=path)
+    y32 = fn.flashnorm_linear_fp8(to_dev(bits["x"]), Q, s, wl.eps, out_dtype=torch.float32, path=path,
+                                  workspace=workspace)
     torch.cuda.synchronize()
     assert O.rel_err(to_host_f64(y32), O.exact_operand_fp8(bits, wl.eps)) <= F32_TOL
 
@@ -84,8 +91,8 @@ def test_linear_fp8_token_scales_cover_a_wide_range():
         assert O.rel_err(got[m], ex[m]) <= F32_TOL, m
 
 
-@pytest.mark.parametrize("path", ["decode", "gemv"])
-def test_linear_fp8_subnormal_codes(path):
+@pytest.mark.parametrize("path,workspace", PATHS_WS)
+def test_linear_fp8_subnormal_codes(path, workspace):
     """Every channel: one weight at the channel's maximum (code 448) and all others in E4M3's subnormal range
     (|W*| / s below 2^-6). The subnormal codes carry about 1e-3 of each output, so a widening that flushed
     them to zero would miss the fp32 bar by two orders of magnitude."""
@@ -101,7 +108,75 @@ def test_linear_fp8_subnormal_codes(path):
     codes, _ = O.fold_fp8(bits["w"], bits["g"])
     assert np.mean((codes & 0x78) == 0) > 0.9  # exponent field zero: subnormal (or zero) codes
     Q, s = fn.flashnorm_fold_weights_fp8(to_dev(bits["w"]), to_dev(bits["g"]))
-    y32 = fn.flashnorm_linear_fp8(to_dev(bits["x"]), Q, s, 1e-6, out_dtype=torch.float32, path=path)
+    y32 = fn.flashnorm_linear_fp8(to_dev(bits["x"]), Q, s, 1e-6, out_dtype=torch.float32, path=path,
+                                  workspace=workspace)
     torch.cuda.synchronize()
     ex = O.exact_operand_fp8(bits, 1e-6)
     assert O.rel_err(to_host_f64(y32), ex) <= F32_TOL
+
+
+def _fp8_case(M, d, N, seed):
+    bits = I.Workload("t", "linear_fp8", M, d, N, 1e-6, seed=seed).draw()
+    Q, s = fn.flashnorm_fold_weights_fp8(to_dev(bits["w"]), to_dev(bits["g"]))
+    return bits, to_dev(bits["x"]), Q, s
+
+
+def test_fp8_workspace_applies_where_expected():
+    """The split takes a workspace while there are at most as many 128-row slabs as SMs."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert fn.flashnorm_fp8_workspace_bytes(4, 4096, 12288) > 1024
+    assert fn.flashnorm_fp8_workspace_bytes(4, 4096, 128 * sms) > 1024
+    assert fn.flashnorm_fp8_workspace_bytes(4, 4096, 128 * sms + 128) == 0
+    assert fn.flashnorm_fp8_workspace_bytes(0, 4096, 12288) == 0
+
+
+def test_fp8_workspace_too_small_is_rejected():
+    bits, x, Q, s = _fp8_case(4, 4096, 12288, 3)
+    need = fn.flashnorm_fp8_workspace_bytes(4, 4096, 12288)
+    small = torch.zeros(need - 16, dtype=torch.uint8, device="cuda")
+    y = torch.full((4, 12288), float("nan"), dtype=torch.float32, device="cuda")
+    with pytest.raises(fn.FlashNormError):
+        fn.flashnorm_linear_fp8(x, Q, s, 1e-6, out_dtype=torch.float32, out=y, path="decode", workspace=small)
+    torch.cuda.synchronize()
+    assert torch.isnan(y).all()  # nothing was launched
+
+
+def test_fp8_workspace_shared_back_to_back():
+    """One workspace serves calls of different shapes on one stream, one after another: each call leaves
+    the counters at zero, every repeat is bitwise the first result, and the first is the oracle's."""
+    cases = [(4, 4096, 12288, 5), (1, 576, 960, 6), (16, 2048, 1024, 7), (3, 208, 136, 8)]
+    need = max(fn.flashnorm_fp8_workspace_bytes(M, d, N) for M, d, N, _ in cases)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    data = [_fp8_case(M, d, N, seed) for M, d, N, seed in cases]
+    first = []
+    for bits, x, Q, s in data:
+        first.append(fn.flashnorm_linear_fp8(x, Q, s, 1e-6, out_dtype=torch.float32, workspace=ws))
+    outs = []
+    for it in range(60):
+        bits, x, Q, s = data[it % len(data)]
+        outs.append(fn.flashnorm_linear_fp8(x, Q, s, 1e-6, out_dtype=torch.float32, workspace=ws))
+    torch.cuda.synchronize()
+    for it, y in enumerate(outs):
+        assert torch.equal(y.view(torch.int32), first[it % len(data)].view(torch.int32)), it
+    for (bits, x, Q, s), y in zip(data, first):
+        assert O.rel_err(to_host_f64(y), O.exact_operand_fp8(bits, 1e-6)) <= F32_TOL
+    assert int(ws[:1024].count_nonzero().item()) == 0
+
+
+def test_fp8_workspace_auto_per_stream():
+    """workspace="auto" on two streams: each stream gets its own scratch, and both results are exact."""
+    bits, x, Q, s = _fp8_case(4, 4096, 12288, 9)
+    ref = fn.flashnorm_linear_fp8(x, Q, s, 1e-6, out_dtype=torch.float32, workspace=None)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    ys = []
+    for st in (s1, s2):
+        with torch.cuda.stream(st):
+            ys.append([fn.flashnorm_linear_fp8(x, Q, s, 1e-6, out_dtype=torch.float32) for _ in range(20)])
+    torch.cuda.synchronize()
+    ex = O.exact_operand_fp8(bits, 1e-6)
+    for lst in ys:
+        assert O.rel_err(to_host_f64(lst[-1]), ex) <= F32_TOL
+        for y in lst[1:]:
+            assert torch.equal(y.view(torch.int32), lst[0].view(torch.int32))
+    assert O.rel_err(to_host_f64(ref), ex) <= F32_TOL

@@ -84,6 +84,25 @@ def test_postnorm_split_writes_stay_in_bounds(M, d, N, hd):
     assert O.rel_err(to_host_f64(y), ex) <= 5e-3
 
 
+@pytest.mark.parametrize("M,d,N", [(5, 1008, 200), (3, 4096, 12288), (16, 208, 136)])
+def test_fp8_workspace_writes_stay_in_bounds(M, d, N):
+    """FP8 decode with its K split over a workspace: the partials stay inside the size the query reports,
+    the counters are zero again afterwards, and y is written exactly."""
+    need = fn.flashnorm_fp8_workspace_bytes(M, d, N)
+    assert need > 1024
+    bits = I.Workload("t", "linear_fp8", M, d, N, 1e-6, seed=M + d).draw()
+    Q, s = fn.flashnorm_fold_weights_fp8(to_dev(bits["w"]), to_dev(bits["g"]))
+    flat_ws, wsp, n_ws = _guarded((need // 4,), torch.float32)
+    wsp[:256].view(torch.int32).zero_()  # the counters start at zero
+    flat, y, n = _guarded((M, N), torch.bfloat16)
+    for _ in range(3):
+        fn.flashnorm_linear_fp8(to_dev(bits["x"]), Q, s, 1e-6, out=y, path="decode", workspace=wsp.view(torch.uint8))
+    torch.cuda.synchronize()
+    assert _intact(flat_ws, n_ws) and _intact(flat, n)
+    assert int(wsp[:256].view(torch.int32).count_nonzero().item()) == 0
+    assert O.rel_err(to_host_f64(y), O.exact_operand_fp8(bits, 1e-6)) <= 5e-3
+
+
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_layernorm_decode_writes_stay_in_bounds(out_dtype):
     """LayerNorm at decode size (the tensor-core decode kernel, ragged N, K split over a cluster)."""
