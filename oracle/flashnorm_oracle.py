@@ -30,6 +30,10 @@ function below states the plainest reading of that prose:
 * RoPE on the normalised query/key heads (the abstract names RoPE-based
   attention; the paper builds on RoFormer): pairs (2i, 2i+1) of a head rotated
   by pos * base^(-2i/head_dim), RoFormer's own pairing.
+* Quantized W* (the abstract: folded checkpoints stay compatible with quantized
+  models): weight-only FP8 E4M3 with one scale per output channel, and NVFP4
+  (E2M1 elements, an E4M3 scale per 16 k, a per-channel fp32 scale), both
+  quantized after the fold, the channel scale applied with the deferred 1/rms.
 
 Everything is computed in float64 from inputs given as bf16 bit patterns; the
 only library primitive is numpy's float64 matrix product. No blocking, fusion
@@ -312,6 +316,130 @@ def deferred_fp8(x, codes, scales, eps):
 
 
 # ---------------------------------------------------------------------------
+# NVFP4 (4-bit) W*, the second quantized format. Reading: weight-only, the
+# NVFP4 element and micro-block encoding (E2M1 elements, one E4M3 scale per 16
+# consecutive elements along the contraction dimension k), and, in place of the
+# format's per-tensor fp32 scale, one fp32 scale per output channel, so that it
+# multiplies the output together with the deferred 1/rms as the fp8 channel
+# scale does. Quantized after the fold:
+#   W*[n, k] = g[k] W[k, n] (exact in fp32),
+#   s2[n] = max_k |W*[n, k]| / (448 * 6) (fp32; 1 if the channel is all zero),
+#   sb[n, b] = E4M3_rne(max_{k in block b} |W*[n, k]| / (6 * s2[n])) (the
+#              product 6 * s2[n] rounded to fp32, then the fp32 division),
+#   Q[n, k] = E2M1_rne(W*[n, k] / (dec(sb[n, b]) * s2[n])) (the product rounded
+#             to fp32, then the fp32 division; 0 where dec(sb) is 0),
+#   y[m, n] = (sum_k x[m, k] dec(Q[n, k]) dec(sb[n, k // 16])) * s2[n] / rms(x_m).
+# E2M1: 1 sign bit, 2 exponent bits with bias 1, 1 mantissa bit: magnitudes
+# 0, 0.5, 1, 1.5, 2, 3, 4, 6 (0.5 is the one subnormal); no infinity, no NaN.
+# The library stores the codes packed (see pack_nvfp4); the oracle keeps them
+# one per array element.
+# ---------------------------------------------------------------------------
+
+E2M1_MAX = 6.0
+
+
+def f64_to_e2m1(v) -> np.ndarray:
+    """Round to E2M1 with round-to-nearest, ties to even, saturating at +-6; return the 4-bit codes (uint8).
+
+    Written from the format: a magnitude in [2^e, 2^(e+1)) with e >= 0 is a multiple of 2^(e-1) (2
+    significant bits); below 1 the quantum is 0.5. np.rint rounds halfway cases to the even integer.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    a = np.minimum(np.abs(v), E2M1_MAX)
+    _, e = np.frexp(a)                       # a in [2^(e-1), 2^e)
+    q = np.ldexp(1.0, np.maximum(e - 1, 0) - 1)
+    r = np.minimum(np.rint(a / q) * q, E2M1_MAX)
+    _, er = np.frexp(r)
+    ex = er - 1                              # r in [2^ex, 2^(ex+1))
+    normal = r >= 1.0
+    mant = np.where(normal, np.rint((np.ldexp(r, -np.where(normal, ex, 0)) - 1.0) * 2.0), 0)
+    code_n = ((np.where(normal, ex, 0) + 1) << 1) + mant.astype(np.int64)
+    code_s = np.rint(r / 0.5).astype(np.int64)          # 0 or 0.5
+    code = np.where(normal, code_n, code_s).astype(np.int64)
+    code = code | np.where(np.signbit(v), 0x8, 0)
+    return code.astype(np.uint8)
+
+
+def e2m1_to_f64(codes) -> np.ndarray:
+    """Decode E2M1 codes (the low 4 bits) exactly."""
+    c = np.asarray(codes, dtype=np.int64) & 0xF
+    s = np.where(c & 0x8, -1.0, 1.0)
+    e = (c >> 1) & 0x3
+    m = c & 0x1
+    val = np.where(e == 0, m * 0.5, (1.0 + m / 2.0) * np.ldexp(1.0, e - 1))
+    return s * val
+
+
+NVFP4_BLOCK = 16
+
+
+def fold_nvfp4(w_bits, g_bits):
+    """(codes uint8 [N, d] one E2M1 code each, block scales uint8 [N, ceil(d/16)] E4M3, s2 float32 [N]): the
+    fold, then NVFP4 quantization with a per-channel second-level scale, every decision in fp32."""
+    W = (np.asarray(w_bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+    g = (np.asarray(g_bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+    Ws = (g[:, None] * W).T.astype(np.float32)            # [N, d], exact products
+    N, d = Ws.shape
+    nb = -(-d // NVFP4_BLOCK)
+    amax = np.max(np.abs(Ws), axis=1)
+    s2 = np.where(amax > 0, amax / np.float32(E4M3_MAX * E2M1_MAX), np.float32(1.0)).astype(np.float32)
+    pad = np.zeros((N, nb * NVFP4_BLOCK), dtype=np.float32)
+    pad[:, :d] = Ws
+    blocks = pad.reshape(N, nb, NVFP4_BLOCK)
+    bmax = np.max(np.abs(blocks), axis=2)                   # [N, nb]
+    six_s2 = (np.float32(E2M1_MAX) * s2).astype(np.float32)
+    bscale = f64_to_e4m3((bmax / six_s2[:, None]).astype(np.float32).astype(np.float64))
+    dsb = e4m3_to_f64(bscale).astype(np.float32)            # exact in fp32
+    den = (dsb * s2[:, None]).astype(np.float32)             # [N, nb], one fp32 rounding
+    safe = np.where(den > 0, den, np.float32(1.0)).astype(np.float32)
+    t = (blocks / safe[:, :, None]).astype(np.float32)       # IEEE fp32 division
+    t = np.where(den[:, :, None] > 0, t, np.float32(0.0))
+    codes = f64_to_e2m1(t.astype(np.float64)).reshape(N, nb * NVFP4_BLOCK)[:, :d]
+    return codes, bscale, s2
+
+
+def dequant_nvfp4(codes, bscales, s2) -> np.ndarray:
+    """W*q [N, d] in fp64: dec(Q) * dec(sb) * s2."""
+    codes = np.asarray(codes)
+    d = codes.shape[1]
+    sb = e4m3_to_f64(bscales)[:, np.arange(d) // NVFP4_BLOCK]
+    return e2m1_to_f64(codes) * sb * np.asarray(s2, dtype=np.float64)[:, None]
+
+
+def deferred_nvfp4(x, codes, bscales, s2, eps):
+    """y = (x . (dec(Q) dec(sb))^T) * s2 * 1/sqrt(mean(x^2) + eps), in fp64.
+
+    Source: "FlashNorm: Fast Normalization for Transformers", Abstract, folded weights staying
+    compatible with quantized models; the NVFP4 scheme is the reading stated at fold_nvfp4.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    return (x @ dequant_nvfp4(codes, bscales, s2).T) * inv_rms(x, eps)[:, None]
+
+
+NVFP4_GROUP = 256          # k per packed group
+NVFP4_GROUP_BYTES = 144    # 128 bytes of codes + 16 block scales
+
+
+def pack_nvfp4(codes, bscales) -> np.ndarray:
+    """The library's storage of NVFP4 W*: per output channel, groups of 256 k of 144 bytes each. Byte j < 128
+    of group G holds the codes of k = 256 G + 2 j (low nibble) and 256 G + 2 j + 1 (high nibble); byte 128 + b
+    holds the E4M3 scale of block b (k = 256 G + 16 b .. + 15). A last partial group is padded with zero codes
+    and zero scales. Returns uint8 [N, ceil(d/256) * 144]."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    bscales = np.asarray(bscales, dtype=np.uint8)
+    N, d = codes.shape
+    G = -(-d // NVFP4_GROUP)
+    c = np.zeros((N, G * NVFP4_GROUP), dtype=np.uint8)
+    c[:, :d] = codes & 0xF
+    s = np.zeros((N, G * NVFP4_GROUP // NVFP4_BLOCK), dtype=np.uint8)
+    s[:, :bscales.shape[1]] = bscales
+    c = c.reshape(N, G, NVFP4_GROUP // 2, 2)
+    packed = np.concatenate([(c[..., 0] | (c[..., 1] << 4)).astype(np.uint8),
+                             s.reshape(N, G, NVFP4_GROUP // NVFP4_BLOCK)], axis=2)
+    return packed.reshape(N, G * NVFP4_GROUP_BYTES)
+
+
+# ---------------------------------------------------------------------------
 # LayerNorm -> linear. The abstract says the same techniques extend to
 # LayerNorm; the pages give no formula. Reading: the standard LayerNorm over the
 # d features of a row, biased variance, eps inside the root, gain gamma and bias
@@ -514,6 +642,19 @@ def exact_operand_fp8(bits: dict, eps: float, rows=None) -> np.ndarray:
         x = x[rows]
     codes, scales = fold_fp8(bits["w"], bits["g"])
     return deferred_fp8(x, codes, scales, eps)
+
+
+def exact_operand_nvfp4(bits: dict, eps: float, rows=None) -> np.ndarray:
+    """The NVFP4 path on its own operands: the oracle's fold_nvfp4 codes and scales (the library's fold
+    matches them bit for bit), then y = (x . Wq^T) * s2 * 1/rms in fp64.
+
+    Source: as deferred_nvfp4.
+    """
+    x = bf16_to_f64(bits["x"])
+    if rows is not None:
+        x = x[rows]
+    codes, bscales, s2 = fold_nvfp4(bits["w"], bits["g"])
+    return deferred_nvfp4(x, codes, bscales, s2, eps)
 
 
 def reference_layernorm(bits: dict, eps: float, rows=None) -> np.ndarray:

@@ -361,6 +361,91 @@ def check_fp8(O):
     return fails
 
 
+E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]  # the format's eight magnitudes, codes 0..7
+
+
+def check_nvfp4(O):
+    """NVFP4 weight quantization: the E2M1 table, hand-worked roundings (ties to even, saturation), brute
+    force over the grid, a hand-worked fold of one channel, the invariants of the fold on random weights,
+    the packed layout byte by byte, and the deferred output against the unquantized definition."""
+    fails = []
+    # decode: the format's table, sign in bit 3
+    want = np.array(E2M1_TABLE + [-v for v in E2M1_TABLE])
+    got = O.e2m1_to_f64(np.arange(16))
+    if not (np.array_equal(got, want) and np.all(np.signbit(got[8:]))):
+        fails.append("e2m1 decode table")
+    # encode, worked by hand: halfway cases go to the even mantissa, magnitudes above 6 saturate
+    for val, code in ((0.25, 0), (0.3, 1), (0.75, 2), (1.25, 2), (1.75, 4), (2.5, 4), (2.9, 5), (3.5, 6),
+                      (5.0, 6), (5.1, 7), (7.0, 7), (1e9, 7), (-0.25, 8), (-1.75, 12), (-6.0, 15), (0.0, 0)):
+        if int(O.f64_to_e2m1(np.array([val]))[0]) != code:
+            fails.append(f"e2m1 code of {val}")
+    # brute force: the nearest grid value, ties to the even code
+    rng = np.random.default_rng(47)
+    v = np.concatenate([rng.uniform(-7.5, 7.5, 3000), np.arange(-30, 31) * 0.25])
+    grid = np.array(E2M1_TABLE)
+    for x in v:
+        a = min(abs(x), 6.0)
+        dist = np.abs(grid - a)
+        best = np.flatnonzero(dist == dist.min())
+        mag = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
+        expect = mag | (8 if np.signbit(x) else 0)
+        if int(O.f64_to_e2m1(np.array([x]))[0]) != expect:
+            fails.append(f"e2m1 brute force at {x}")
+            break
+    # a fold worked by hand: one channel, g = 1, d = 32. Block 0 holds grid values times 2^-3 (channel
+    # maximum 0.75), block 1 grid values times 2^-4 (block maximum 0.09375).
+    #   s2 = 0.75 / 2688; block 0: 0.75 / (6 s2) = 448 -> scale 448 (E4M3 0x7E), step 448 s2 = 1/8;
+    #   block 1: 0.09375 / (6 s2) = 56 -> scale 56 = 1.75 * 2^5 (E4M3 0x66), step 56 s2 = 2^-6.
+    b0 = [6, 3, -1.5, 0.5, 4, -6, 0, 1, 2, -0.5, 1.5, -3, 0, 4, -2, 1]
+    b1 = [1, 0.5, -1, 1.5, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, -0.5]
+    col = np.array([t * 2.0 ** -3 for t in b0] + [t * 2.0 ** -4 for t in b1])
+    codes, bsc, s2 = O.fold_nvfp4(O.f64_to_bf16(col[:, None]), O.f64_to_bf16(np.ones(32)))
+    want0 = [7, 5, 11, 1, 6, 15, 0, 2, 4, 9, 3, 13, 0, 6, 12, 2]
+    want1 = [6, 4, 14, 7, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 12]   # b1 * 2^-4 / 2^-6 = 4 * b1
+    if list(codes[0]) != want0 + want1:
+        fails.append("nvfp4 fold: codes of the hand-worked channel")
+    if list(bsc[0]) != [0x7E, 0x66]:
+        fails.append("nvfp4 fold: block scales of the hand-worked channel")
+    if s2[0] != np.float32(0.75) / np.float32(2688.0):
+        fails.append("nvfp4 fold: channel scale")
+    if np.max(np.abs(O.dequant_nvfp4(codes, bsc, s2)[0] - col)) > 1e-7 * 0.75:
+        fails.append("nvfp4 fold: grid values not reproduced")
+    # invariants on random weights: each nonzero block's largest code is +-6, the block holding the channel
+    # maximum has scale 448, and every weight is within half a quantum of its block's grid
+    d, N = 80, 24
+    wb = O.f64_to_bf16(rng.standard_normal((d, N)) / np.sqrt(d) * np.exp(rng.uniform(-3, 3, (1, N))))
+    gb = O.f64_to_bf16(rng.uniform(0.5, 1.5, d))
+    codes, bsc, s2 = O.fold_nvfp4(wb, gb)
+    Ws = O.fold(O.bf16_to_f64(wb), O.bf16_to_f64(gb)).T           # [N, d]
+    dec = O.e2m1_to_f64(codes)
+    if np.any(np.max(np.abs(dec.reshape(N, d // 16, 16)), axis=2) != 6.0):
+        fails.append("nvfp4 fold: a block maximum not at 6")
+    if np.any(np.max(O.e4m3_to_f64(bsc), axis=1) != 448.0):
+        fails.append("nvfp4 fold: channel maximum block not at scale 448")
+    step = O.e4m3_to_f64(bsc)[:, np.arange(d) // 16] * s2[:, None].astype(np.float64)
+    t = Ws / step
+    half_q = np.where(np.abs(t) < 2, 0.25, np.where(np.abs(t) < 4, 0.5, 1.0))
+    if np.any(np.abs(t - dec) > half_q * (1 + 1e-6)):
+        fails.append("nvfp4 fold: weight off by more than half a quantum")
+    # packed layout, by hand: codes 0..15 repeated along k, scales 0x40, 0x41 for the two blocks of d = 32
+    c = np.tile(np.arange(16, dtype=np.uint8), (2, 2))
+    packed = O.pack_nvfp4(c, np.array([[0x40, 0x41], [0x40, 0x41]], dtype=np.uint8))
+    row = [(2 * j) % 16 | (((2 * j + 1) % 16) << 4) for j in range(16)] + [0] * 112 + [0x40, 0x41] + [0] * 14
+    if packed.shape != (2, 144) or list(packed[1]) != row:
+        fails.append("nvfp4 packed layout")
+    # the deferred output against the definition: within the bound the half quanta give, not exact
+    x = O.bf16_to_f64(O.f64_to_bf16(rng.standard_normal((5, d)) * np.exp(rng.uniform(-2, 2, (5, 1)))))
+    eps = 1e-6
+    y4 = O.deferred_nvfp4(x, codes, bsc, s2, eps)
+    ydef = O.norm_then_project(x, O.bf16_to_f64(gb), O.bf16_to_f64(wb), eps)
+    bound = O.inv_rms(x, eps)[:, None] * (np.abs(x) @ (half_q * step).T)
+    if np.any(np.abs(y4 - ydef) > bound * (1 + 1e-9) + 1e-15):
+        fails.append("nvfp4 deferred output outside the quantization bound")
+    if not (1e-3 < O.rel_err(y4, ydef) < 0.3):
+        fails.append("nvfp4 deferred output: error not of the size E2M1 gives")
+    return fails
+
+
 def check_rel_err(O):
     """The parity metric max|y - y_ref| / max|y_ref| on hand-worked cases, chosen so that a sign, a
     missing absolute value, the wrong denominator or swapped arguments each change the result."""
@@ -381,7 +466,7 @@ def check_rel_err(O):
 
 ALL_CHECKS = [check_golden, check_torch_rmsnorm, check_torch_silu, check_torch_bf16,
               check_closed_forms, check_invariants, check_brute_force, check_rope, check_layernorm, check_fp8,
-              check_rel_err]
+              check_nvfp4, check_rel_err]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
@@ -444,6 +529,10 @@ def test_reference_output_wrappers():
     codes, scales = O.fold_fp8(bits["w"], bits["g"])
     assert np.allclose(O.exact_operand_fp8(bits, 1e-6, rows=[0, 2]), O.deferred_fp8(x[[0, 2]], codes, scales, 1e-6),
                        rtol=1e-15)
+    # NVFP4: likewise, with the block scales and the channel scale
+    codes, bsc, s2 = O.fold_nvfp4(bits["w"], bits["g"])
+    assert np.allclose(O.exact_operand_nvfp4(bits, 1e-6, rows=[0, 2]),
+                       O.deferred_nvfp4(x[[0, 2]], codes, bsc, s2, 1e-6), rtol=1e-15)
 
 
 # ---------------------------------------------------------------------------
@@ -615,6 +704,55 @@ def _mut_fp8_deferred_scale_by_row(x, codes, scales, eps):
     return (x @ O.e4m3_to_f64(codes).T) * O.inv_rms(x, eps)[:, None] * s[: x.shape[0], None]
 
 
+def _mut_e2m1_ties_away(v):
+    v = np.asarray(v, dtype=np.float64)
+    a = np.minimum(np.abs(v), 6.0)
+    _, e = np.frexp(a)
+    q = np.ldexp(1.0, np.maximum(e - 1, 0) - 1)
+    return _ORIG_F64_TO_E2M1(np.where(np.signbit(v), -1.0, 1.0) * np.floor(a / q + 0.5) * q)
+
+
+def _mut_e2m1_bias0(codes):
+    return _ORIG_E2M1_TO_F64(codes) * np.where((np.asarray(codes, dtype=np.int64) >> 1) & 3, 2.0, 1.0)
+
+
+def _mut_nvfp4_block32(w_bits, g_bits):
+    saved = O.NVFP4_BLOCK
+    O.NVFP4_BLOCK = 32
+    try:
+        codes, bsc, s2 = _ORIG_FOLD_NVFP4(w_bits, g_bits)
+    finally:
+        O.NVFP4_BLOCK = saved
+    return codes, np.repeat(bsc, 2, axis=1)[:, : -(-codes.shape[1] // 16)], s2
+
+
+def _mut_nvfp4_scale_without_6(w_bits, g_bits):
+    saved = O.E2M1_MAX
+    O.E2M1_MAX = 1.0  # the block maximum mapped to 1 instead of 6 (codes then saturate)
+    try:
+        return _ORIG_FOLD_NVFP4(w_bits, g_bits)
+    finally:
+        O.E2M1_MAX = saved
+
+
+def _mut_nvfp4_no_s2(codes, bscales, s2):
+    d = np.asarray(codes).shape[1]
+    return O.e2m1_to_f64(codes) * O.e4m3_to_f64(bscales)[:, np.arange(d) // 16]
+
+
+def _mut_nvfp4_pack_nibbles_swapped(codes, bscales):
+    c = np.asarray(codes, dtype=np.uint8)
+    swapped = c.copy()
+    swapped[:, 0::2], swapped[:, 1::2] = c[:, 1::2], c[:, 0::2]
+    return _ORIG_PACK_NVFP4(swapped, bscales)
+
+
+_ORIG_F64_TO_E2M1 = O.f64_to_e2m1
+_ORIG_E2M1_TO_F64 = O.e2m1_to_f64
+_ORIG_FOLD_NVFP4 = O.fold_nvfp4
+_ORIG_PACK_NVFP4 = O.pack_nvfp4
+
+
 def _mut_rel_err_signed(y, y_ref):
     y, y_ref = np.asarray(y, dtype=np.float64), np.asarray(y_ref, dtype=np.float64)
     return float(np.max(y - y_ref) / np.max(np.abs(y_ref)))
@@ -657,6 +795,12 @@ MUTANTS = {
     "fp8 one scale for the whole matrix": ("fold_fp8", _mut_fp8_scale_rows),
     "fp8 channel scale dropped": ("deferred_fp8", _mut_fp8_deferred_no_scale),
     "fp8 scale indexed by token": ("deferred_fp8", _mut_fp8_deferred_scale_by_row),
+    "e2m1 ties away from zero": ("f64_to_e2m1", _mut_e2m1_ties_away),
+    "e2m1 exponent bias 0": ("e2m1_to_f64", _mut_e2m1_bias0),
+    "nvfp4 blocks of 32": ("fold_nvfp4", _mut_nvfp4_block32),
+    "nvfp4 block maximum mapped to 1": ("fold_nvfp4", _mut_nvfp4_scale_without_6),
+    "nvfp4 channel scale dropped": ("dequant_nvfp4", _mut_nvfp4_no_s2),
+    "nvfp4 nibbles swapped": ("pack_nvfp4", _mut_nvfp4_pack_nibbles_swapped),
     "rel_err without the absolute value": ("rel_err", _mut_rel_err_signed),
     "rel_err relative to the result": ("rel_err", _mut_rel_err_denominator_of_y),
     "rel_err relative to max(y_ref)": ("rel_err", _mut_rel_err_max_not_abs),
