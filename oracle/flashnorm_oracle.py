@@ -421,20 +421,24 @@ NVFP4_GROUP_BYTES = 144    # 128 bytes of codes + 16 block scales
 
 
 def pack_nvfp4(codes, bscales) -> np.ndarray:
-    """The library's storage of NVFP4 W*: per output channel, groups of 256 k of 144 bytes each. Byte j < 128
-    of group G holds the codes of k = 256 G + 2 j (low nibble) and 256 G + 2 j + 1 (high nibble); byte 128 + b
-    holds the E4M3 scale of block b (k = 256 G + 16 b .. + 15). A last partial group is padded with zero codes
-    and zero scales. Returns uint8 [N, ceil(d/256) * 144]."""
+    """The library's storage of NVFP4 W*: per output channel, groups of 256 k of 144 bytes each. Bytes
+    0..127 of group G are 32 little-endian 32-bit words; word j holds the codes of k = 256 G + 8 j + 2 i
+    in bits 4 i .. 4 i + 3 and of k = 256 G + 8 j + 2 i + 1 in bits 16 + 4 i .. 16 + 4 i + 3 (i = 0..3):
+    the even k in the low half, the odd k in the high half. Byte 128 + b holds the E4M3 scale of block b
+    (k = 256 G + 16 b .. + 15). A last partial group is padded with zero codes and zero scales. Returns
+    uint8 [N, ceil(d/256) * 144]."""
     codes = np.asarray(codes, dtype=np.uint8)
     bscales = np.asarray(bscales, dtype=np.uint8)
     N, d = codes.shape
     G = -(-d // NVFP4_GROUP)
-    c = np.zeros((N, G * NVFP4_GROUP), dtype=np.uint8)
+    c = np.zeros((N, G * NVFP4_GROUP), dtype=np.uint32)
     c[:, :d] = codes & 0xF
+    c = c.reshape(N, G, NVFP4_GROUP // 8, 4, 2)             # [n, group, word, i, even/odd]
+    shifts = (4 * np.arange(4, dtype=np.uint32))[:, None] + np.array([0, 16], dtype=np.uint32)[None, :]
+    words = np.bitwise_or.reduce(c << shifts, axis=(3, 4)).astype(np.uint32)   # [n, group, 32]
     s = np.zeros((N, G * NVFP4_GROUP // NVFP4_BLOCK), dtype=np.uint8)
     s[:, :bscales.shape[1]] = bscales
-    c = c.reshape(N, G, NVFP4_GROUP // 2, 2)
-    packed = np.concatenate([(c[..., 0] | (c[..., 1] << 4)).astype(np.uint8),
+    packed = np.concatenate([words.astype("<u4").view(np.uint8).reshape(N, G, 128),
                              s.reshape(N, G, NVFP4_GROUP // NVFP4_BLOCK)], axis=2)
     return packed.reshape(N, G * NVFP4_GROUP_BYTES)
 

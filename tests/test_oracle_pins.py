@@ -427,10 +427,13 @@ def check_nvfp4(O):
     half_q = np.where(np.abs(t) < 2, 0.25, np.where(np.abs(t) < 4, 0.5, 1.0))
     if np.any(np.abs(t - dec) > half_q * (1 + 1e-6)):
         fails.append("nvfp4 fold: weight off by more than half a quantum")
-    # packed layout, by hand: codes 0..15 repeated along k, scales 0x40, 0x41 for the two blocks of d = 32
+    # packed layout, by hand: codes 0..15 repeated along k, scales 0x40, 0x41 for the two blocks of d = 32.
+    # Word 0 (k = 0..7) holds even codes 0, 2, 4, 6 in its low half (0x6420) and odd codes 1, 3, 5, 7 in its
+    # high half (0x7531): 0x75316420, little endian; word 1 (k = 8..15): 0xFDB9ECA8.
     c = np.tile(np.arange(16, dtype=np.uint8), (2, 2))
     packed = O.pack_nvfp4(c, np.array([[0x40, 0x41], [0x40, 0x41]], dtype=np.uint8))
-    row = [(2 * j) % 16 | (((2 * j + 1) % 16) << 4) for j in range(16)] + [0] * 112 + [0x40, 0x41] + [0] * 14
+    w0, w1 = [0x20, 0x64, 0x31, 0x75], [0xA8, 0xEC, 0xB9, 0xFD]
+    row = (w0 + w1) * 2 + [0] * 112 + [0x40, 0x41] + [0] * 14
     if packed.shape != (2, 144) or list(packed[1]) != row:
         fails.append("nvfp4 packed layout")
     # the deferred output against the definition: within the bound the half quanta give, not exact
