@@ -81,6 +81,9 @@ BENCH_WORKLOADS = {
     "llama7b_qkv_fp8_tc_m1": ["llama7b_qkv_fp8_m1"],
     # the FP8 tensor-core decode without a workspace: its K split stays inside thread-block clusters
     "llama7b_qkv_fp8_cluster_m4": ["llama7b_qkv_fp8_m4"],
+    "llama7b_qkv_nvfp4_m1": ["llama7b_qkv_nvfp4_m1"],
+    "llama7b_qkv_nvfp4_m4": ["llama7b_qkv_nvfp4_m4"],
+    "llama7b_qkv_nvfp4_m16": ["llama7b_qkv_nvfp4_m16"],
     # the same decode projection on the CUDA-core GEMV instead of the tensor-core decode kernel
     "llama7b_qkv_gemv_m16": ["llama7b_qkv_m16"],
     "llama7b_qkv_gemv_m1": ["llama7b_qkv_m1"],
@@ -169,8 +172,13 @@ def _is_decode(wls) -> bool:
 
 
 def _weight_bytes(w) -> int:
-    """Bytes of the folded weight a decode step streams: bf16 W*, or FP8 codes plus fp32 channel scales."""
-    return w.d * w.w_cols + 4 * w.w_cols if w.kind == "linear_fp8" else 2 * w.d * w.w_cols
+    """Bytes of the folded weight a decode step streams: bf16 W*; FP8 codes plus fp32 channel scales; NVFP4
+    codes (half a byte), E4M3 block scales (one per 16) and fp32 channel scales."""
+    if w.kind == "linear_fp8":
+        return w.d * w.w_cols + 4 * w.w_cols
+    if w.kind == "linear_nvfp4":
+        return w.w_cols * (w.d // 2 + w.d // 16 + 4)
+    return 2 * w.d * w.w_cols
 
 
 def _metric(wls):
@@ -279,6 +287,9 @@ class Projection:
         elif wl.kind == "linear_fp8":  # FP8 codes; the channel scales are copied with them
             ws0, s0 = fn.flashnorm_fold_weights_fp8(W, self.g)
             self.fp8_scales = [s0] + [s0.clone() for _ in range(copies - 1)]
+        elif wl.kind == "linear_nvfp4":  # NVFP4 codes and block scales; the channel scales are copied with them
+            ws0, s0 = fn.flashnorm_fold_weights_nvfp4(W, self.g)
+            self.fp8_scales = [s0] + [s0.clone() for _ in range(copies - 1)]
         else:
             ws0 = fn.flashnorm_fold_weights(W, self.g, glu=glu)
         self.x = [x0] + [x0.clone() for _ in range(copies - 1)]
@@ -299,8 +310,9 @@ class Projection:
             self.pn_ws = torch.empty(need, dtype=torch.uint8, device="cuda") if need > 0 else None
         # likewise the FP8 decode's K split over independent CTAs (its counters zeroed once, here)
         self.fp8_ws = None
-        if wl.kind == "linear_fp8" and path != "cluster":
-            need = fn.flashnorm_fp8_workspace_bytes(wl.M, wl.d, wl.N)
+        if wl.kind in ("linear_fp8", "linear_nvfp4") and path != "cluster":
+            q = fn.flashnorm_fp8_workspace_bytes if wl.kind == "linear_fp8" else fn.flashnorm_nvfp4_workspace_bytes
+            need = q(wl.M, wl.d, wl.N)
             self.fp8_ws = torch.zeros(need, dtype=torch.uint8, device="cuda") if need > 0 else None
         if wl.kind == "postnorm_rope":  # the (cos, sin) table and the row positions are set up once
             self.rope_cs = fn.flashnorm_rope_table(wl.M, wl.head_dim, wl.rope_base)
@@ -318,6 +330,8 @@ class Projection:
         elif wl.kind == "linear_fp8":
             fn.flashnorm_linear_fp8(x, self.ws[r], self.fp8_scales[r], wl.eps, out=self.y[r],
                                     path="decode" if self.path == "cluster" else self.path, workspace=self.fp8_ws)
+        elif wl.kind == "linear_nvfp4":
+            fn.flashnorm_linear_nvfp4(x, self.ws[r], self.fp8_scales[r], wl.eps, out=self.y[r], workspace=self.fp8_ws)
         elif wl.kind == "layernorm":
             fn.flashnorm_layernorm_linear(x, self.ws[r], self.ln_colsum, self.ln_bias, wl.eps, out=self.y[r])
         elif wl.kind == "postnorm_rope":
@@ -685,11 +699,15 @@ def _oracle_setup(workload: str):
         elif w.kind == "linear_fp8":
             codes, scales = O.fold_fp8(b["w"], b["g"])
             call = lambda r, c, x=x, codes=codes, scales=scales, w=w: O.deferred_fp8(x[r], codes[:c], scales[:c], w.eps)
+        elif w.kind == "linear_nvfp4":
+            codes, bsc, s2 = O.fold_nvfp4(b["w"], b["g"])
+            call = lambda r, c, x=x, codes=codes, bsc=bsc, s2=s2, w=w: O.deferred_nvfp4(x[r], codes[:c], bsc[:c],
+                                                                                       s2[:c], w.eps)
         else:
             raise ValueError(w.kind)
         rows = np.arange(min(w.M, 1024))
         # the oracle decodes every FP8 code it is given on each call: a pass covers at most 1024 channels
-        chans = min(w.N, 1024) if w.kind == "linear_fp8" else w.N
+        chans = min(w.N, 1024) if w.kind in ("linear_fp8", "linear_nvfp4") else w.N
         projs.append({"w": w, "call": call, "rows": rows, "chans": chans})
     _ORACLE_CACHE[workload] = (wls, decode, projs)
     return _ORACLE_CACHE[workload]
@@ -698,7 +716,7 @@ def _oracle_setup(workload: str):
 def _pass_units(p, decode: bool) -> float:
     w = p["w"]
     if decode:  # weight bytes of the sampled channels
-        per = (w.d + 4) if w.kind == "linear_fp8" else 2 * w.d
+        per = {"linear_fp8": w.d + 4, "linear_nvfp4": w.d // 2 + w.d // 16 + 4}.get(w.kind, 2 * w.d)
         return float(p["chans"] * per)
     return 2.0 * len(p["rows"]) * w.d * w.w_cols
 

@@ -93,7 +93,7 @@ class Workload:
     """One synthetic problem: shapes, epsilon and the variant it exercises."""
 
     name: str
-    kind: str  # "linear" | "glu" | "postnorm" | "postnorm_rope" | "layernorm" | "linear_fp8"
+    kind: str  # "linear" | "glu" | "postnorm" | "postnorm_rope" | "layernorm" | "linear_fp8" | "linear_nvfp4"
     M: int
     d: int
     N: int  # linear: output columns; glu: F (W has 2F columns); postnorm: latent width
@@ -122,6 +122,8 @@ class Workload:
             b += 4 * self.M + 4 * self.M * self.head_dim
         if self.kind == "linear_fp8":  # one byte per weight plus a fp32 scale per output channel
             b = 2 * (self.M * self.d + self.M * self.N) + self.d * self.N + 4 * self.N
+        if self.kind == "linear_nvfp4":  # half a byte per weight, a byte per 16 weights, a fp32 scale per channel
+            b = 2 * (self.M * self.d + self.M * self.N) + self.N * (self.d // 2 + self.d // 16 + 4)
         return b
 
     def positions(self) -> np.ndarray:
@@ -165,6 +167,11 @@ WORKLOADS = {
     "llama7b_qkv_fp8_m1": Workload("llama7b_qkv_fp8_m1", "linear_fp8", 1, 4096, 12288, 1e-6, seed=BASE_SEED + 2),
     "llama7b_qkv_fp8_m4": Workload("llama7b_qkv_fp8_m4", "linear_fp8", 4, 4096, 12288, 1e-6, seed=BASE_SEED + 2),
     "llama7b_qkv_fp8_m16": Workload("llama7b_qkv_fp8_m16", "linear_fp8", 16, 4096, 12288, 1e-6, seed=BASE_SEED + 2),
+    # the same with NVFP4 (E2M1 codes, E4M3 scales per 16 k, a fp32 scale per output channel)
+    "llama7b_qkv_nvfp4_m1": Workload("llama7b_qkv_nvfp4_m1", "linear_nvfp4", 1, 4096, 12288, 1e-6, seed=BASE_SEED + 2),
+    "llama7b_qkv_nvfp4_m4": Workload("llama7b_qkv_nvfp4_m4", "linear_nvfp4", 4, 4096, 12288, 1e-6, seed=BASE_SEED + 2),
+    "llama7b_qkv_nvfp4_m16": Workload("llama7b_qkv_nvfp4_m16", "linear_nvfp4", 16, 4096, 12288, 1e-6,
+                                      seed=BASE_SEED + 2),
     # LayerNorm (gain and bias) before the SmolLM2-sized QKV projection, 8192 tokens
     "layernorm_qkv_m8192": Workload("layernorm_qkv_m8192", "layernorm", 8192, 576, 960, 1e-5, seed=BASE_SEED + 7),
     # LayerNorm before the Llama-7B-sized QKV projection at decode, 4 tokens

@@ -272,6 +272,39 @@ FN_API fn_status flashnorm_linear_fp8_ws(const void* x, const void* Q, const voi
  * rejects as invalid (d % 16 != 0, N % 8 != 0, out-of-range sizes).
  */
 FN_API fn_status flashnorm_fp8_workspace_bytes(int64_t M, int64_t d, int64_t N, int64_t* bytes);
+FN_API fn_status flashnorm_fp8_workspace_bytes(int64_t M, int64_t d, int64_t N, int64_t* bytes);
+
+/*
+ * NVFP4 (4-bit) W* (the same Abstract item: folded checkpoints stay compatible with quantized models).
+ * Reading: weight-only; the NVFP4 element and micro-block encoding (E2M1 codes, one E4M3 scale per 16
+ * consecutive k of an output channel) with one fp32 scale per output channel in place of the format's
+ * per-tensor scale, quantized after the fold:
+ *     W*[n][k] = g[k] W[k][n],   s2[n] = max_k |W*[n][k]| / (448 * 6)   (1 for an all-zero channel),
+ *     sb[n][b] = E4M3(max_{k in block b} |W*[n][k]| / (6 s2[n])),
+ *     Q[n][k]  = E2M1(W*[n][k] / (sb[n][k / 16] s2[n]))   (0 where sb is 0),
+ *     y[m][n]  = (sum_k x[m][k] Q[n][k] sb[n][k / 16]) * s2[n] / sqrt(mean_k x[m][k]^2 + eps),
+ * products and divisions in fp32, each rounding to nearest even and saturating (E4M3 at 448, E2M1 at 6).
+ * Storage of Q and sb (caller-owned, N rows of ceil(d / 256) * 144 bytes): per output channel, groups of
+ * 256 k of 144 bytes. Bytes 0..127 of a group are 32 little-endian uint32 words; word j holds the codes of
+ * k = 8 j + 2 i in bits 4 i .. 4 i + 3 and of k = 8 j + 2 i + 1 in bits 16 + 4 i .. 16 + 4 i + 3 (i = 0..3,
+ * k counted within the group). Byte 128 + b is the E4M3 scale of the group's block b (k = 16 b .. + 15).
+ * Past d: zero codes and zero scales.
+ * flashnorm_fold_weights_nvfp4: W bf16 [d, N] row-major, g bf16 [d] -> Q4 as above and s2 fp32 [N].
+ *   d % 16 == 0, N % 8 == 0.
+ * flashnorm_linear_nvfp4: decode (M <= FN_DECODE_MAX_M) on the tensor cores: each code is widened on chip,
+ *   exactly, to the bf16 value Q * sb, x is used as it is, fp32 accumulation. x bf16 [M, d], y [M, N] of
+ *   out_dtype. workspace / workspace_bytes as for flashnorm_linear_fp8_ws (the first 1024 bytes zero before
+ *   first use and left zero by every call; NULL: one CTA per 128-row slab over all of d, slower). Larger M
+ *   returns FN_ERR_UNSUPPORTED.
+ * flashnorm_nvfp4_workspace_bytes: the workspace flashnorm_linear_nvfp4 uses for this shape on the current
+ *   device, 0 where the split does not apply (more 128-row slabs than SMs, M == 0, M > FN_DECODE_MAX_M).
+ */
+FN_API fn_status flashnorm_fold_weights_nvfp4(const void* W, const void* g, void* Q4, void* s2, int64_t d, int64_t N,
+                                              void* stream);
+FN_API fn_status flashnorm_linear_nvfp4(const void* x, const void* Q4, const void* s2, void* y, int64_t M, int64_t d,
+                                        int64_t N, float eps, int out_dtype, void* workspace, int64_t workspace_bytes,
+                                        void* stream);
+FN_API fn_status flashnorm_nvfp4_workspace_bytes(int64_t M, int64_t d, int64_t N, int64_t* bytes);
 
 /*
  * flashnorm_rope_table — fills rope_cs (fp32 [max_pos][head_dim / 2][2], caller-owned device memory,

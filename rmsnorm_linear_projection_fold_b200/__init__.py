@@ -36,6 +36,9 @@ __all__ = [
     "flashnorm_fold_weights_fp8",
     "flashnorm_linear_fp8",
     "flashnorm_fp8_workspace_bytes",
+    "flashnorm_fold_weights_nvfp4",
+    "flashnorm_linear_nvfp4",
+    "flashnorm_nvfp4_workspace_bytes",
     "flashnorm_layernorm_linear",
     "flashnorm_rmsnorm",
     "flashnorm_linear_unfused",
@@ -81,6 +84,9 @@ _SIGNATURES = {
     "flashnorm_linear_fp8_ex": [_P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _INT, _P],
     "flashnorm_linear_fp8_ws": [_P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _INT, _P, _I64, _P],
     "flashnorm_fp8_workspace_bytes": [_I64, _I64, _I64, _P],
+    "flashnorm_fold_weights_nvfp4": [_P, _P, _P, _P, _I64, _I64, _P],
+    "flashnorm_linear_nvfp4": [_P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P, _I64, _P],
+    "flashnorm_nvfp4_workspace_bytes": [_I64, _I64, _I64, _P],
     "flashnorm_layernorm_linear": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
     "flashnorm_rmsnorm": [_P, _P, _P, _I64, _I64, _F, _P],
     "flashnorm_linear_unfused": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _INT, _P],
@@ -441,6 +447,76 @@ def flashnorm_linear_fp8(x: torch.Tensor, Q: torch.Tensor, scales: torch.Tensor,
     _invoke("flashnorm_linear_fp8_ws", x, _ptr(x), _ptr(Q), _ptr(scales), _ptr(y), M, d, N, float(eps),
             _out_code(out_dtype), PATHS[path], _ptr(ws), ws.numel() if ws is not None else 0, _stream_ptr(x),
             report="flashnorm_linear_fp8")
+    return y
+
+
+NVFP4_GROUP, NVFP4_GROUP_BYTES = 256, 144  # k per stored group and its bytes (include/flashnorm.h)
+
+
+def flashnorm_fold_weights_nvfp4(W: torch.Tensor, g: torch.Tensor):
+    """(Q4 uint8 [N, ceil(d/256) * 144], s2 fp32 [N]): the gain fold, then NVFP4 quantization (E2M1 codes,
+    E4M3 scales per 16 k, a fp32 scale per output channel), in the layout include/flashnorm.h states."""
+    _need(W, "W", dim=2)
+    _need(g, "g", dim=1)
+    d, N = W.shape
+    if g.shape[0] != d:
+        raise ValueError("g must have d elements")
+    _same_device(W, g=g)
+    groups = -(-d // NVFP4_GROUP)
+    Q4 = torch.empty(N, groups * NVFP4_GROUP_BYTES, dtype=torch.uint8, device=W.device)
+    s2 = torch.empty(N, dtype=torch.float32, device=W.device)
+    _invoke("flashnorm_fold_weights_nvfp4", W, _ptr(W), _ptr(g), _ptr(Q4), _ptr(s2), d, N, _stream_ptr(W))
+    return Q4, s2
+
+
+_nvfp4_ws_bytes_cache = {}
+
+
+def flashnorm_nvfp4_workspace_bytes(M: int, d: int, N: int, device=None) -> int:
+    """Workspace bytes flashnorm_linear_nvfp4 uses for this shape on `device` (0: no split)."""
+    dev = torch.cuda.current_device() if device is None else torch.device(device).index
+    if dev is None:
+        dev = torch.cuda.current_device()
+    key = (dev, int(M), int(d), int(N))
+    hit = _nvfp4_ws_bytes_cache.get(key)
+    if hit is not None:
+        return hit
+    nbytes = ctypes.c_int64(0)
+    _invoke_on(dev, "flashnorm_nvfp4_workspace_bytes", int(M), int(d), int(N), ctypes.addressof(nbytes))
+    _nvfp4_ws_bytes_cache[key] = int(nbytes.value)
+    return int(nbytes.value)
+
+
+def flashnorm_linear_nvfp4(x: torch.Tensor, Q4: torch.Tensor, s2: torch.Tensor, eps: float,
+                           out_dtype=torch.bfloat16, out=None, workspace="auto") -> torch.Tensor:
+    """Decode (M <= 16) with NVFP4 weights on the tensor cores:
+    y = (x . (Q * sb)^T) * s2 * 1/sqrt(mean(x^2) + eps).
+
+    workspace: as for flashnorm_linear_fp8 ("auto": a zero-initialised scratch kept per device and stream;
+    None: one CTA per 128-row slab over all of d; or a caller-owned uint8 CUDA tensor)."""
+    _need(x, "x", dim=2)
+    _need(Q4, "Q4", torch.uint8, dim=2)
+    _need(s2, "s2", torch.float32, dim=1)
+    M, d = x.shape
+    N = Q4.shape[0]
+    if Q4.shape[1] != -(-d // NVFP4_GROUP) * NVFP4_GROUP_BYTES or s2.shape[0] != N:
+        raise ValueError("Q4 [N, ceil(d/256) * 144] and s2 [N] must match x [M, d]")
+    _same_device(x, Q4=Q4, s2=s2)
+    y = _output(out, (M, N), out_dtype, x)
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError('workspace must be "auto", None or a uint8 CUDA tensor')
+        nbytes = flashnorm_nvfp4_workspace_bytes(M, d, N, x.get_device()) if 0 < M <= 16 else 0
+        ws = _fp8_stream_workspace(x, nbytes) if nbytes > 0 else None
+    elif workspace is None:
+        ws = None
+    else:
+        _need(workspace, "workspace", torch.uint8, dim=1)
+        _same_device(x, workspace=workspace)
+        ws = workspace
+    _invoke("flashnorm_linear_nvfp4", x, _ptr(x), _ptr(Q4), _ptr(s2), _ptr(y), M, d, N, float(eps),
+            _out_code(out_dtype), _ptr(ws), ws.numel() if ws is not None else 0, _stream_ptr(x),
+            report="flashnorm_linear_nvfp4")
     return y
 
 

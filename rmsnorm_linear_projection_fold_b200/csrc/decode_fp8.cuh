@@ -42,6 +42,19 @@ constexpr int kD8Tok = 16;                         // token slots (MMA N)
 constexpr int kD8KStage = 128;                     // k per stage: 128 one-byte codes, one 128-byte row
 constexpr int kD8WStage = kD8Rows * kD8KStage;     // 16 KB of codes
 constexpr int kD8XStage = kD8Tok * kD8KStage * 2;  // 4 KB of x: two 64-k atoms of 16 rows x 128 bytes
+// Formats of the quantized W*. FP8 E4M3: one byte per weight; a pipeline stage is one 128-k unit (a
+// 128-byte row per W* row, 128-byte swizzle). NVFP4: E2M1 codes with E4M3 scales per 16 k, stored in
+// groups of 256 k of 144 bytes per W* row (fp8.cuh); a stage is one group, two 128-k units, loaded
+// without swizzle: rows 144 bytes apart put the eight rows of a quarter warp on distinct banks.
+constexpr int kFmtFp8 = 0, kFmtNvfp4 = 1;
+template <int FMT>
+struct D8Fmt {
+  static constexpr int kUnits = FMT == kFmtNvfp4 ? 2 : 1;         // 128-k units per stage
+  static constexpr int kRowBytes = FMT == kFmtNvfp4 ? 144 : 128;  // bytes of one W* row per stage
+  static constexpr int kWStage = kD8Rows * kRowBytes;
+  static constexpr int kXStage = kUnits * kD8XStage;
+  static constexpr int kKStage = kUnits * kD8KStage;  // k per stage
+};
 constexpr int kD8ABufs = 3;                        // bf16 A tiles in tensor memory, 64 columns each
 constexpr int kD8ACol0 = 64;                       // first A column (the accumulators take columns 0..63)
 // MMA issuers: stage i of a CTA's K range is issued by issuer i % kD8Issuers, into that issuer's own
@@ -76,9 +89,9 @@ struct DecodeFp8Params {
   float* part_ss;      // KSPLIT == 0: [slabs][ksplit][16]
 };
 
-template <int STAGES, int KSPLIT>
+template <int STAGES, int KSPLIT, int FMT = kFmtFp8>
 __host__ __device__ constexpr int decode_fp8_smem_bytes() {
-  return 1024 + STAGES * (kD8WStage + kD8XStage) +
+  return 1024 + STAGES * (D8Fmt<FMT>::kWStage + D8Fmt<FMT>::kXStage) +
          (KSPLIT > 1 ? (KSPLIT - 1) * kD8Rows * kD8Tok * 4 + KSPLIT * kD8Tok * 4 : 0) + 512;
 }
 
@@ -122,16 +135,31 @@ __device__ __forceinline__ uint32_t e4m3_pairs_to_bf16x2(uint32_t v) {
   return r;
 }
 
-template <int STAGES, int KSPLIT, bool OUT_F32>
+// Two E2M1 codes, the even k in bits 0..3 of `v` and the odd k in bits 16..19, to bf16x2 times the block
+// scale, exactly. A code s.ee.m has ee at bits 2..1 and m at bit 0; moved to bits 8..7 and 6 (a bf16's low
+// exponent bits and top mantissa bit), with s at bit 15, the bf16 read from those bits is 2^(ee-127)(1 +
+// m/2) (for ee = 0 the subnormal m 2^-127): 2^-126 times the E2M1 value 2^(ee-1)(1 + m/2) (or m/2). One
+// multiply by 2^126 makes it the E2M1 value, a second by the block scale (an E4M3 value: at most 4
+// significant bits against E2M1's 2) the weight, both exact in bf16.
+__device__ __forceinline__ uint32_t e2m1_pair_to_bf16x2(uint32_t v, uint32_t scale2) {
+  const uint32_t f = ((v & 0x00070007u) << 6) | ((v & 0x00080008u) << 12);
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(f), "r"(0x7E807E80u));  // x 2^126
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(r), "r"(scale2));
+  return r;
+}
+
+template <int STAGES, int KSPLIT, bool OUT_F32, int FMT = kFmtFp8>
 __global__ void __launch_bounds__(kD8Threads, 1)
     k_decode_fp8(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_x,
                  DecodeFp8Params p) {
+  using F = D8Fmt<FMT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
-  uint8_t* sW = smem;                     // [STAGES][128 rows][128 codes], 128-byte swizzle
-  uint8_t* sX = sW + STAGES * kD8WStage;  // [STAGES][2 atoms][16 rows x 128 bytes], 128-byte swizzle
-  float* part_d = reinterpret_cast<float*>(sX + STAGES * kD8XStage);             // [KSPLIT-1][128][16]
+  uint8_t* sW = smem;                       // [STAGES][128 rows][F::kRowBytes]
+  uint8_t* sX = sW + STAGES * F::kWStage;   // [STAGES][2 atoms per unit][16 rows x 128 bytes], 128-byte swizzle
+  float* part_d = reinterpret_cast<float*>(sX + STAGES * F::kXStage);            // [KSPLIT-1][128][16]
   float* part_ss = part_d + (KSPLIT > 1 ? (KSPLIT - 1) * kD8Rows * kD8Tok : 0);  // [KSPLIT][16]
   uint64_t* full = reinterpret_cast<uint64_t*>(part_ss + (KSPLIT > 1 ? KSPLIT * kD8Tok : 0));
   uint64_t* empty = full + STAGES;
@@ -150,14 +178,15 @@ __global__ void __launch_bounds__(kD8Threads, 1)
   const uint32_t rank = KSPLIT == 0 ? blockIdx.x % static_cast<uint32_t>(ks) : (KSPLIT > 1 ? cluster_ctarank() : 0);
   const int slab = static_cast<int>(blockIdx.x) / ks;
   const int n0 = slab * kD8Rows;
-  const int num_units = (p.K + kD8KStage - 1) / kD8KStage;  // stages of 128 over all of K
-  const int u0 = static_cast<int>((static_cast<long long>(rank) * num_units) / ks);
-  const int u1 = static_cast<int>((static_cast<long long>(rank + 1) * num_units) / ks);
+  const int num_stages = (p.K + F::kKStage - 1) / F::kKStage;  // stages over all of K
+  const int g0 = static_cast<int>((static_cast<long long>(rank) * num_stages) / ks);
+  const int g1 = static_cast<int>((static_cast<long long>(rank + 1) * num_stages) / ks);
+  const int u0 = g0 * F::kUnits, u1 = g1 * F::kUnits;  // this range's 128-k units
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 4 + 1);  // the four converter warps and the MMA's commit
+      mbar_init(&empty[s], 4 + F::kUnits);  // the four converter warps and the commit of each unit's MMAs
     }
     for (int b = 0; b < kD8ABufs; ++b) {
       mbar_init(&afull[b], 4);   // the four converter warps
@@ -172,7 +201,7 @@ __global__ void __launch_bounds__(kD8Threads, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_x);
     // the first ring's worth of this CTA's codes into L2 while the previous kernel drains
-    for (int u = u0; u < u1 && u < u0 + STAGES; ++u) tma_prefetch_l2_2d(&tm_q, u * kD8KStage, n0);
+    for (int gi = g0; gi < g1 && gi < g0 + STAGES; ++gi) tma_prefetch_l2_2d(&tm_q, gi * F::kRowBytes, n0);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 256);
@@ -191,15 +220,16 @@ __global__ void __launch_bounds__(kD8Threads, 1)
       int s = 0, issued = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int u = u0; u < u1; ++u) {
+      for (int gi = g0; gi < g1; ++gi) {
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&full[s], kD8WStage + kD8XStage);
-        tma_load_2d(sW + s * kD8WStage, &tm_q, &full[s], u * kD8KStage, n0);
-        tma_load_2d(sX + s * kD8XStage, &tm_x, &full[s], u * kD8KStage, 0);
-        tma_load_2d(sX + s * kD8XStage + 2048, &tm_x, &full[s], u * kD8KStage + 64, 0);
+        mbar_arrive_expect_tx(&full[s], F::kWStage + F::kXStage);
+        tma_load_2d(sW + s * F::kWStage, &tm_q, &full[s], gi * F::kRowBytes, n0);
+#pragma unroll
+        for (int a = 0; a < 2 * F::kUnits; ++a)  // x in 64-k atoms
+          tma_load_2d(sX + s * F::kXStage + a * 2048, &tm_x, &full[s], gi * F::kKStage + 64 * a, 0);
         ++issued;
         if (++s == STAGES) {
           s = 0;
@@ -238,9 +268,10 @@ __global__ void __launch_bounds__(kD8Threads, 1)
       const uint32_t idesc = make_idesc_bf16(kD8Rows, kD8Tok);
       const uint32_t acc0 = tmem_base + static_cast<uint32_t>(iss * kD8AccPer * kD8Tok);
       bool ok = true;
-      for (int i = iss; u0 + i < u1; i += kD8Issuers) {
-        const int s = i % STAGES, b = i % kD8ABufs;
-        const uint32_t ph = static_cast<uint32_t>(i / STAGES) & 1u, bph = static_cast<uint32_t>(i / kD8ABufs) & 1u;
+      for (int i = iss; u0 + i < u1; i += kD8Issuers) {  // unit i of the range: stage i / F::kUnits
+        const int st = i / F::kUnits;
+        const int s = st % STAGES, b = i % kD8ABufs;
+        const uint32_t ph = static_cast<uint32_t>(st / STAGES) & 1u, bph = static_cast<uint32_t>(i / kD8ABufs) & 1u;
         // the x tile of this stage (TMA) and the widened codes in A buffer b (the converters)
         if (!mbar_wait(&full[s], ph, abort_flag) || !mbar_wait(&afull[b], bph, abort_flag)) {
           ok = false;
@@ -248,7 +279,7 @@ __global__ void __launch_bounds__(kD8Threads, 1)
         }
         tc_fence_after_sync();
         const uint32_t a_col = tmem_base + static_cast<uint32_t>(kD8ACol0 + b * 64);
-        const uint32_t x_st = smem_u32(sX + s * kD8XStage);
+        const uint32_t x_st = smem_u32(sX + s * F::kXStage + (i % F::kUnits) * kD8XStage);
 #pragma unroll
         for (int j = 0; j < kD8KStage / 16; ++j)  // 8 MMAs of K = 16: 8 columns of A, 32 bytes of a B row
           tc_mma_bf16_ts(acc0 + static_cast<uint32_t>((j % kD8AccPer) * kD8Tok), a_col + j * 8,
@@ -271,44 +302,74 @@ __global__ void __launch_bounds__(kD8Threads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const int t = static_cast<int>(threadIdx.x) - 64;  // 0..127
     const int tok = t >> 3, sub = t & 7;    // sum of squares: token, and its 16-byte chunk of each atom row
-    int s = 0, b = 0;
-    uint32_t ph = 0, bph = 0;
     bool ok = true;
     float ss = 0.f;
     // this row's dequantization scale, loaded now so that its latency hides under the main loop
     const float sc = n0 + row < p.N ? p.scales[n0 + row] : 0.f;
-    for (int u = u0; u < u1; ++u) {
+    for (int i = 0; u0 + i < u1; ++i) {  // unit i of the range: half `half` of stage i / F::kUnits
+      const int st = i / F::kUnits, half = i % F::kUnits;
+      const int s = st % STAGES, b = i % kD8ABufs;
+      const uint32_t ph = static_cast<uint32_t>(st / STAGES) & 1u, bph = static_cast<uint32_t>(i / kD8ABufs) & 1u;
       if (!mbar_wait(&full[s], ph, abort_flag) || !mbar_wait(&aempty[b], bph ^ 1u, abort_flag)) {
         ok = false;
         break;
       }
-      // this row's 128 codes: eight 16-byte chunks, chunk c at c ^ (row & 7) (TMA's 128-byte swizzle)
-      const uint8_t* line = sW + s * kD8WStage + row * 128;
-      uint32_t h[32];
+      const uint32_t a_st = tmem_base + lane_base + static_cast<uint32_t>(kD8ACol0 + b * 64);
+      if constexpr (FMT == kFmtFp8) {
+        // this row's 128 codes: eight 16-byte chunks, chunk c at c ^ (row & 7) (TMA's 128-byte swizzle)
+        const uint8_t* line = sW + s * F::kWStage + row * 128;
+        uint32_t h[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+        for (int q2 = 0; q2 < 2; ++q2) {
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int c = half * 4 + c4;
-          const uint4 w = *reinterpret_cast<const uint4*>(line + (((c ^ row) & 7) << 4));
-          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int c = q2 * 4 + c4;
+            const uint4 w = *reinterpret_cast<const uint4*>(line + (((c ^ row) & 7) << 4));
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {  // codes k0..k3 of word i: columns (k0, k1) and (k2, k3)
-            h[c4 * 8 + 2 * i] = e4m3_pairs_to_bf16x2(__byte_perm(ws[i], 0u, 0x4140));
-            h[c4 * 8 + 2 * i + 1] = e4m3_pairs_to_bf16x2(__byte_perm(ws[i], 0u, 0x4342));
+            for (int e = 0; e < 4; ++e) {  // codes k0..k3 of word e: columns (k0, k1) and (k2, k3)
+              h[c4 * 8 + 2 * e] = e4m3_pairs_to_bf16x2(__byte_perm(ws[e], 0u, 0x4140));
+              h[c4 * 8 + 2 * e + 1] = e4m3_pairs_to_bf16x2(__byte_perm(ws[e], 0u, 0x4342));
+            }
           }
+          tmem_st32(a_st + static_cast<uint32_t>(q2 * 32), h);
         }
-        tmem_st32(tmem_base + lane_base + static_cast<uint32_t>(kD8ACol0 + b * 64 + half * 32), h);
+      } else {
+        // this row's group of 144 bytes: unit `half` is code words 16 half .. + 15 (blocks 8 half .. + 7,
+        // two words each) and block scales 128 + 8 half .. + 7
+        const uint8_t* line = sW + s * F::kWStage + row * 144;
+        const uint2 scw = *reinterpret_cast<const uint2*>(line + 128 + 8 * half);
+        uint32_t h[32];
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {  // 32 columns: blocks 4 q2 .. 4 q2 + 3
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {  // one 16-byte chunk: two blocks
+            const uint4 w = *reinterpret_cast<const uint4*>(line + (half * 4 + q2 * 2 + c) * 16);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int bb = q2 * 4 + c * 2 + e;  // block of this unit: columns 8 bb .. 8 bb + 7
+              const uint32_t sbyte = ((bb < 4 ? scw.x : scw.y) >> (8 * (bb & 3))) & 0xFFu;
+              const uint32_t sbf = e4m3_pairs_to_bf16x2(sbyte | (sbyte << 16));  // the scale in both halves
+#pragma unroll
+              for (int wi = 0; wi < 2; ++wi)
+#pragma unroll
+                for (int pi = 0; pi < 4; ++pi)  // k = 16 bb + 8 wi + 2 pi and the next: one column
+                  h[(c * 2 + e) * 8 + wi * 4 + pi] = e2m1_pair_to_bf16x2(ws[2 * e + wi] >> (4 * pi), sbf);
+            }
+          }
+          tmem_st32(a_st + static_cast<uint32_t>(q2 * 32), h);
+        }
       }
-      // x^2 of token `tok` over chunk `sub` of both 64-k atoms of this stage (zero past M and past K)
+      // x^2 of token `tok` over chunk `sub` of both 64-k atoms of this unit (zero past M and past K)
 #pragma unroll
       for (int a = 0; a < 2; ++a) {
-        const uint4 w = *reinterpret_cast<const uint4*>(sX + s * kD8XStage + a * 2048 + (tok >> 3) * 1024 +
-                                                        (tok & 7) * 128 + (sub << 4));
+        const uint4 w = *reinterpret_cast<const uint4*>(sX + s * F::kXStage + half * kD8XStage + a * 2048 +
+                                                        (tok >> 3) * 1024 + (tok & 7) * 128 + (sub << 4));
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float lo = bf16lo_to_f32(ws[i]), hi = bf16hi_to_f32(ws[i]);
+        for (int e = 0; e < 4; ++e) {
+          const float lo = bf16lo_to_f32(ws[e]), hi = bf16hi_to_f32(ws[e]);
           ss = fmaf(lo, lo, ss);
           ss = fmaf(hi, hi, ss);
         }
@@ -318,16 +379,8 @@ __global__ void __launch_bounds__(kD8Threads, 1)
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&empty[s]);
+        if (half == F::kUnits - 1) mbar_arrive(&empty[s]);  // the stage's last unit: its codes are read
         mbar_arrive(&afull[b]);
-      }
-      if (++s == STAGES) {
-        s = 0;
-        ph ^= 1u;
-      }
-      if (++b == kD8ABufs) {
-        b = 0;
-        bph ^= 1u;
       }
     }
     // A wait that gave up leaves this thread's sum incomplete: it contributes NaN instead, so every output

@@ -175,6 +175,19 @@ fn_status make_u8_map(CUtensorMap* map, const void* ptr, int64_t k, int64_t rows
   return FN_OK;
 }
 
+// NVFP4 W* [rows][groups x 144 bytes] (fp8.cuh's storage): one 144-byte group of 128 rows per box, no
+// swizzle (the converters' reads of 144-byte rows fall on distinct banks as they are).
+fn_status make_q4_map(CUtensorMap* map, const void* ptr, int64_t row_bytes, int64_t rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(fn::kNvfp4GroupBytes), static_cast<cuuint32_t>(fn::kD8Rows)};
+  CUresult r = encode_cached(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  if (r == CUDA_ERROR_NOT_FOUND) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (r != CUDA_SUCCESS) return fail(FN_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  return FN_OK;
+}
+
 // 3-D fp32 [planes][rows][cols] (the split post-norm's partial products) with a 32-column x 128-row box
 // and 128-byte swizzle, for TMA stores.
 fn_status make_partial_map(CUtensorMap* map, void* ptr, int64_t cols, int64_t rows, int64_t planes) {
@@ -692,11 +705,11 @@ fn_status launch_gemv_fp8_t(const void* x, const void* q, const void* scales, vo
 // FP8 decode on the tensor cores
 // ------------------------------------------------------------------------------------------------
 
-template <int STAGES, int KSPLIT, bool OUT_F32>
+template <int STAGES, int KSPLIT, bool OUT_F32, int FMT = fn::kFmtFp8>
 fn_status launch_decode_fp8_t(const CUtensorMap& tq, const CUtensorMap& tx, const fn::DecodeFp8Params& p, int slabs,
                               int dev, cudaStream_t stream) {
-  auto kern = fn::k_decode_fp8<STAGES, KSPLIT, OUT_F32>;
-  constexpr int smem = fn::decode_fp8_smem_bytes<STAGES, KSPLIT>();
+  auto kern = fn::k_decode_fp8<STAGES, KSPLIT, OUT_F32, FMT>;
+  constexpr int smem = fn::decode_fp8_smem_bytes<STAGES, KSPLIT, FMT>();
   static bool configured[kMaxDevices] = {false};
   if (!configured[dev]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -711,12 +724,13 @@ fn_status launch_decode_fp8_t(const CUtensorMap& tq, const CUtensorMap& tx, cons
   return FN_OK;
 }
 
-// K ranges per slab of the FP8 decode kernel with a workspace: enough independent CTAs for two on every
-// SM (each holds 5 stages: two fit one SM's shared and tensor memory), while there are at most as many
-// slabs as SMs; 1 (no split, no workspace) otherwise.
-int fp8_ws_ksplit(int64_t N, int64_t d, int sms) {
+// K ranges per slab of the quantized decode kernel with a workspace: enough independent CTAs for two on
+// every SM (each holds 4-5 stages: two fit one SM's shared and tensor memory), while there are at most as
+// many slabs as SMs; 1 (no split, no workspace) otherwise. k_stage: k per pipeline stage (128 for FP8,
+// 256 for NVFP4); a range holds whole stages.
+int fp8_ws_ksplit(int64_t N, int64_t d, int sms, int k_stage = fn::kD8KStage) {
   const int64_t slabs = (N + fn::kD8Rows - 1) / fn::kD8Rows;
-  const int64_t units = (d + fn::kD8KStage - 1) / fn::kD8KStage;
+  const int64_t units = (d + k_stage - 1) / k_stage;
   if (slabs > fn::kD8MaxWsSlabs || slabs > sms) return 1;
   int64_t ks = (2 * static_cast<int64_t>(sms)) / slabs;
   ks = std::min<int64_t>(std::min<int64_t>(ks, units), 16);
@@ -780,6 +794,48 @@ fn_status run_decode_fp8(const void* x, const void* q, const void* scales, void*
   if (ksplit == 2) return FN_D8(5, 2);
   return FN_D8(4, 4);
 #undef FN_D8
+}
+
+// NVFP4 W* on the tensor cores: the same kernel with the 4-bit widening and 256-k stages (two units). With
+// a workspace, the K split over independent CTAs (four 26 KB stages each: two CTAs fit one SM); without
+// one, one CTA per slab over all of K (eight stages).
+fn_status run_decode_nvfp4(const void* x, const void* q4, const void* s2, void* y, int64_t M, int64_t d, int64_t N,
+                           float eps, int out_dtype, void* workspace, cudaStream_t stream) {
+  int dev = 0;
+  const int sms = device_sm_count(&dev);
+  if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
+  const int64_t slabs = (N + fn::kD8Rows - 1) / fn::kD8Rows;
+  const int64_t groups = (d + fn::kNvfp4Group - 1) / fn::kNvfp4Group;
+  const int ks = workspace != nullptr ? fp8_ws_ksplit(N, d, sms, fn::kNvfp4Group) : 1;
+  CUtensorMap tq, tx;
+  fn_status st = make_q4_map(&tq, q4, groups * fn::kNvfp4GroupBytes, N);
+  if (st != FN_OK) return st;
+  st = make_operand_map(&tx, x, d, M, fn::kD8Tok);
+  if (st != FN_OK) return st;
+  fn::DecodeFp8Params p;
+  p.y = y;
+  p.scales = static_cast<const float*>(s2);
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(d);
+  p.N = static_cast<int>(N);
+  p.ldy = static_cast<int>(N);
+  p.ksplit = ks;
+  p.eps = eps;
+  p.counters = nullptr;
+  p.part = p.part_ss = nullptr;
+  const int sl = static_cast<int>(slabs);
+  const bool f32 = out_dtype == FN_F32;
+#define FN_D4(ST, KS)                                                                                          \
+  (f32 ? launch_decode_fp8_t<ST, KS, true, fn::kFmtNvfp4>(tq, tx, p, sl, dev, stream)                          \
+       : launch_decode_fp8_t<ST, KS, false, fn::kFmtNvfp4>(tq, tx, p, sl, dev, stream))
+  if (ks >= 2) {
+    p.counters = static_cast<unsigned*>(workspace);
+    p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + fn::kD8WsCounterBytes);
+    p.part_ss = p.part + slabs * ks * fn::kD8Rows * fn::kD8Tok;
+    return FN_D4(4, 0);
+  }
+  return FN_D4(8, 1);
+#undef FN_D4
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -1065,7 +1121,7 @@ fn_status flashnorm_fold_weights_fp8(const void* W, const void* g, void* Q, void
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_kernel(fn::k_fp8_scales, dim3(static_cast<unsigned>((N + 255) / 256)), dim3(256), 0, s, 1,
                                 static_cast<const uint16_t*>(W), static_cast<const uint16_t*>(g),
-                                static_cast<float*>(scales), static_cast<int>(d), static_cast<int>(N));
+                                static_cast<float*>(scales), static_cast<int>(d), static_cast<int>(N), fn::kE4m3Max);
   if (e == cudaSuccess)
     e = launch_kernel(fn::k_fold_fp8, grid, dim3(256), 0, s, 1, static_cast<const uint16_t*>(W),
                       static_cast<const uint16_t*>(g), static_cast<const float*>(scales), static_cast<uint8_t*>(Q),
@@ -1139,6 +1195,75 @@ fn_status flashnorm_linear_fp8_ws(const void* x, const void* Q, const void* scal
     default: return FN_G8(16, 1);
   }
 #undef FN_G8
+}
+
+fn_status flashnorm_fold_weights_nvfp4(const void* W, const void* g, void* Q4, void* s2, int64_t d, int64_t N,
+                                       void* stream) {
+  g_last_error[0] = '\0';
+  if (d < 16 || d > kMaxDim || d % 16 != 0) return fail(FN_ERR_INVALID_ARG, "d = %lld must be a positive multiple of 16", (long long)d);
+  if (N < 8 || N > kMaxDim || N % 8 != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a positive multiple of 8", (long long)N);
+  fn_status st;
+  if ((st = check_ptr(W, "W")) != FN_OK) return st;
+  if ((st = check_ptr(g, "g")) != FN_OK) return st;
+  if ((st = check_ptr(Q4, "Q4")) != FN_OK) return st;
+  if ((st = check_ptr(s2, "s2")) != FN_OK) return st;
+  const int64_t groups = (d + fn::kNvfp4Group - 1) / fn::kNvfp4Group;
+  if (groups > 65535) return fail(FN_ERR_UNSUPPORTED, "d too large for the fold grid");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_kernel(fn::k_fp8_scales, dim3(static_cast<unsigned>((N + 255) / 256)), dim3(256), 0, s, 1,
+                                static_cast<const uint16_t*>(W), static_cast<const uint16_t*>(g),
+                                static_cast<float*>(s2), static_cast<int>(d), static_cast<int>(N), fn::kNvfp4ScaleDiv);
+  if (e == cudaSuccess)
+    e = launch_kernel(fn::k_fold_nvfp4, dim3(static_cast<unsigned>((N + 31) / 32), static_cast<unsigned>(groups)),
+                      dim3(256), 0, s, 1, static_cast<const uint16_t*>(W), static_cast<const uint16_t*>(g),
+                      static_cast<const float*>(s2), static_cast<uint8_t*>(Q4), static_cast<int>(d),
+                      static_cast<int>(N));
+  if (e != cudaSuccess) return cuda_fail(e, "nvfp4 fold launch");
+  return FN_OK;
+}
+
+fn_status flashnorm_nvfp4_workspace_bytes(int64_t M, int64_t d, int64_t N, int64_t* bytes) {
+  g_last_error[0] = '\0';
+  if (bytes == nullptr) return fail(FN_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = 0;
+  if (M < 0 || M > kMaxDim) return fail(FN_ERR_INVALID_ARG, "M = %lld out of range", (long long)M);
+  if (d < 16 || d > kMaxDim || d % 16 != 0) return fail(FN_ERR_INVALID_ARG, "d = %lld must be a positive multiple of 16", (long long)d);
+  if (N < 8 || N > kMaxDim || N % 8 != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a positive multiple of 8", (long long)N);
+  if (M == 0 || M > FN_DECODE_MAX_M) return FN_OK;
+  int dev = 0;
+  const int sms = device_sm_count(&dev);
+  if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
+  *bytes = fp8_ws_bytes(N, fp8_ws_ksplit(N, d, sms, fn::kNvfp4Group));
+  return FN_OK;
+}
+
+fn_status flashnorm_linear_nvfp4(const void* x, const void* Q4, const void* s2, void* y, int64_t M, int64_t d,
+                                 int64_t N, float eps, int out_dtype, void* workspace, int64_t workspace_bytes,
+                                 void* stream) {
+  g_last_error[0] = '\0';
+  fn_status st = check_common(x, Q4, y, M, d, eps, out_dtype);
+  if (st != FN_OK) return st;
+  if (d % 16 != 0) return fail(FN_ERR_INVALID_ARG, "d = %lld must be a multiple of 16", (long long)d);
+  if (N < 8 || N > kMaxDim || N % 8 != 0) return fail(FN_ERR_INVALID_ARG, "N = %lld must be a positive multiple of 8", (long long)N);
+  if (M > FN_DECODE_MAX_M) return fail(FN_ERR_UNSUPPORTED, "the nvfp4 path is decode only: M <= %d", FN_DECODE_MAX_M);
+  if ((st = check_ptr(s2, "s2")) != FN_OK) return st;
+  if (workspace_bytes < 0) return fail(FN_ERR_INVALID_ARG, "workspace_bytes is negative");
+  if (M == 0) return FN_OK;
+  void* ws = nullptr;
+  if (workspace != nullptr) {
+    int dev = 0;
+    const int sms = device_sm_count(&dev);
+    if (sms <= 0) return fail(FN_ERR_CUDA, "cannot query the current device");
+    const int64_t need = fp8_ws_bytes(N, fp8_ws_ksplit(N, d, sms, fn::kNvfp4Group));
+    if (need > 0) {
+      if (workspace_bytes < need)
+        return fail(FN_ERR_INVALID_ARG, "workspace of %lld bytes; this shape needs %lld", (long long)workspace_bytes,
+                    (long long)need);
+      if ((st = check_ptr(workspace, "workspace")) != FN_OK) return st;
+      ws = workspace;
+    }
+  }
+  return run_decode_nvfp4(x, Q4, s2, y, M, d, N, eps, out_dtype, ws, static_cast<cudaStream_t>(stream));
 }
 
 fn_status flashnorm_linear_fp8_ex(const void* x, const void* Q, const void* scales, void* y, int64_t M, int64_t d,

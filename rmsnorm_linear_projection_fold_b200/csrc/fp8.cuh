@@ -10,6 +10,15 @@
 //     y[m, n]  = (sum_k x[m, k] Q[n, k]) * s[n] * 1/sqrt(mean_k x[m, k]^2 + eps)
 // Decode streams Q (one byte per weight: half the bytes of bf16 W*) with x staged in shared memory, as
 // the bf16 GEMV does; each 16-byte load carries 16 weights.
+//
+// The same abstract item, with NVFP4 (4-bit) weights: E2M1 codes, one E4M3 scale per 16 consecutive k of
+// a channel, and a per-channel fp32 scale in place of the format's per-tensor one:
+//     s2[n]    = max_k |W*[n, k]| / (448 * 6)   (1 for an all-zero channel)
+//     sb[n, b] = e4m3_rn_satfinite(max_{k in b} |W*[n, k]| / (6 * s2[n]))
+//     Q[n, k]  = e2m1_rn_satfinite(W*[n, k] / (sb[n, b] * s2[n]))   (0 where sb is 0)
+//     y[m, n]  = (sum_k x[m, k] Q[n, k] sb[n, k / 16]) * s2[n] * 1/sqrt(mean_k x[m, k]^2 + eps)
+// stored per channel in groups of 256 k of 144 bytes: 32 words of codes (word j: k = 8 j .. 8 j + 7 of the
+// group, the even k in bits 0..15, four bits each, the odd k in bits 16..31), then the 16 block scales.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -26,7 +35,7 @@ constexpr float kE4m3Max = 448.0f;
 // s[n] for every output channel: one thread per column n of W [d, N] (row-major), reads coalesced
 // across the threads of a warp.
 __global__ void __launch_bounds__(256) k_fp8_scales(const uint16_t* __restrict__ W, const uint16_t* __restrict__ g,
-                                                    float* __restrict__ scales, int d, int N) {
+                                                    float* __restrict__ scales, int d, int N, float div) {
   grid_dep_wait();
   const int n = blockIdx.x * 256 + threadIdx.x;
   if (n >= N) return;
@@ -36,7 +45,77 @@ __global__ void __launch_bounds__(256) k_fp8_scales(const uint16_t* __restrict__
                     __uint_as_float(static_cast<uint32_t>(W[static_cast<size_t>(k) * N + n]) << 16);
     amax = fmaxf(amax, fabsf(v));
   }
-  scales[n] = amax > 0.0f ? __fdiv_rn(amax, kE4m3Max) : 1.0f;
+  scales[n] = amax > 0.0f ? __fdiv_rn(amax, div) : 1.0f;  // div: 448 (FP8), 448 * 6 (NVFP4)
+}
+
+constexpr float kNvfp4ScaleDiv = 448.0f * 6.0f;
+constexpr int kNvfp4Group = 256;       // k per stored group
+constexpr int kNvfp4GroupBytes = 144;  // 128 bytes of codes + 16 block scales
+
+// E2M1 code of t: round to nearest, ties to even, saturating at +-6. The magnitudes are 0, 0.5, 1, 1.5, 2,
+// 3, 4, 6 (codes 0..7); each comparison below is one midpoint between neighbours, strict where the lower
+// neighbour has the even code (it takes the tie), inclusive where the upper one has. The sign is kept.
+__device__ __forceinline__ uint32_t e2m1_rn_satfinite(float t) {
+  const float a = fabsf(t);
+  const uint32_t m = static_cast<uint32_t>(a > 0.25f) + static_cast<uint32_t>(a >= 0.75f) +
+                     static_cast<uint32_t>(a > 1.25f) + static_cast<uint32_t>(a >= 1.75f) +
+                     static_cast<uint32_t>(a > 2.5f) + static_cast<uint32_t>(a >= 3.5f) + static_cast<uint32_t>(a > 5.0f);
+  return m | ((__float_as_uint(t) >> 28) & 8u);
+}
+
+// One block per (32 channels, one 256-k group): W* of the group through shared memory ([n][k], one thread
+// per k on the way in, loads of 8 channels at a time), then one thread per (channel, 16-k block): the
+// block's E4M3 scale and its 16 E2M1 codes in the stored layout. Blocks past d get zero codes and a zero
+// scale. d % 16 == 0, N % 8 == 0.
+__global__ void __launch_bounds__(256) k_fold_nvfp4(const uint16_t* __restrict__ W, const uint16_t* __restrict__ g,
+                                                    const float* __restrict__ s2, uint8_t* __restrict__ Q4, int d,
+                                                    int N) {
+  __shared__ float tile[32][kNvfp4Group + 1];  // [n][k]: +1 keeps the column writes on distinct banks
+  const int groups = (d + kNvfp4Group - 1) / kNvfp4Group;
+  const int n0 = blockIdx.x * 32, grp = blockIdx.y;
+  grid_dep_wait();
+  {
+    const int kk = threadIdx.x, k = grp * kNvfp4Group + kk;
+    const float gk = k < d ? bf16lo_to_f32(g[k]) : 0.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int n = n0 + 8 * c;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (k < d && n < N) v = *reinterpret_cast<const uint4*>(W + static_cast<size_t>(k) * N + n);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        tile[8 * c + 2 * e][kk] = gk * bf16lo_to_f32(w[e]);  // exact: a bf16 x bf16 product fits fp32
+        tile[8 * c + 2 * e + 1][kk] = gk * bf16hi_to_f32(w[e]);
+      }
+    }
+  }
+  __syncthreads();
+  for (int item = threadIdx.x; item < 32 * 16; item += 256) {
+    const int nn = item >> 4, bb = item & 15, n = n0 + nn;
+    if (n >= N) continue;
+    const float* v = &tile[nn][bb * 16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    const float sc2 = s2[n];
+    const float t = __fdiv_rn(amax, __fmul_rn(6.0f, sc2));
+    const uint32_t sbc = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(t, t), __NV_SATFINITE, __NV_E4M3)) & 0xFFu;
+    const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(sbc), __NV_E4M3);
+    const float den = __fmul_rn(__half2float(__half(hr)), sc2);  // the decoded scale is exact in half
+    uint32_t words[2] = {0u, 0u};
+    if (den > 0.0f) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t q = e2m1_rn_satfinite(__fdiv_rn(v[j], den));
+        const int jj = j & 7;
+        words[j >> 3] |= q << ((jj & 1) * 16 + (jj >> 1) * 4);
+      }
+    }
+    uint8_t* row = Q4 + static_cast<size_t>(n) * groups * kNvfp4GroupBytes + static_cast<size_t>(grp) * kNvfp4GroupBytes;
+    *reinterpret_cast<uint2*>(row + bb * 8) = make_uint2(words[0], words[1]);
+    row[128 + bb] = static_cast<uint8_t>(sbc);
+  }
 }
 
 // Q [N, d] (K-major, one byte per weight) from W [d, N], g and the scales: one 64 x 64 tile per block,

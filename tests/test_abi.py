@@ -283,3 +283,26 @@ def test_prepare_propagates_errors_and_resets():
         with pytest.raises((ValueError, TypeError, fn.FlashNormError)):
             fn.prepare(fn.flashnorm_linear, x, x, 1e-5)
     assert fn._recording is None and fn._recording_keep is None
+
+
+def test_nvfp4_validation(lib):
+    """The NVFP4 entry points reject bad shapes on the host; the size query needs no device for them."""
+    assert lib.flashnorm_fold_weights_nvfp4(P, P, P, P, 24, 64, NULL) == fn.FN_ERR_INVALID_ARG   # d % 16
+    assert lib.flashnorm_fold_weights_nvfp4(P, P, P, P, 64, 60, NULL) == fn.FN_ERR_INVALID_ARG   # N % 8
+    assert lib.flashnorm_fold_weights_nvfp4(P, P, NULL, P, 64, 64, NULL) == fn.FN_ERR_INVALID_ARG  # Q4 NULL
+    lin = lib.flashnorm_linear_nvfp4
+    assert lin(P, P, P, P, 17, 4096, 12288, 1e-6, 0, NULL, 0, NULL) == fn.FN_ERR_UNSUPPORTED     # M > 16
+    assert lin(P, P, P, P, 4, 4104, 12288, 1e-6, 0, NULL, 0, NULL) == fn.FN_ERR_INVALID_ARG      # d % 16
+    assert lin(P, P, P, P, 4, 4096, 12284, 1e-6, 0, NULL, 0, NULL) == fn.FN_ERR_INVALID_ARG      # N % 8
+    assert lin(P, P, NULL, P, 4, 4096, 12288, 1e-6, 0, NULL, 0, NULL) == fn.FN_ERR_INVALID_ARG   # s2 NULL
+    assert lin(P, P, P, P, 4, 4096, 12288, 1e-6, 0, P, -1, NULL) == fn.FN_ERR_INVALID_ARG        # bytes < 0
+    assert lin(P, P, P, P, 0, 4096, 12288, 1e-6, 0, NULL, 0, NULL) == fn.FN_OK                   # empty call
+    nbytes = ctypes.c_int64(-7)
+    out = ctypes.c_void_p(ctypes.addressof(nbytes))
+    assert lib.flashnorm_nvfp4_workspace_bytes(4, 4096, 12288, NULL) == fn.FN_ERR_INVALID_ARG
+    for shape in [(4, 4104, 12288), (4, 4096, 12284), (-1, 4096, 12288)]:
+        assert lib.flashnorm_nvfp4_workspace_bytes(*shape, out) == fn.FN_ERR_INVALID_ARG, shape
+    for shape in [(0, 4096, 12288), (17, 4096, 12288)]:
+        nbytes.value = -7
+        assert lib.flashnorm_nvfp4_workspace_bytes(*shape, out) == fn.FN_OK
+        assert nbytes.value == 0

@@ -103,6 +103,35 @@ def test_fp8_workspace_writes_stay_in_bounds(M, d, N):
     assert O.rel_err(to_host_f64(y), O.exact_operand_fp8(bits, 1e-6)) <= 5e-3
 
 
+@pytest.mark.parametrize("M,d,N,workspace", [(5, 1008, 200, True), (3, 4096, 12288, True), (7, 272, 136, False)])
+def test_nvfp4_writes_stay_in_bounds(M, d, N, workspace):
+    """NVFP4 decode: the partials stay inside the workspace size the query reports (the counters zero again
+    afterwards), the fold writes exactly its two outputs, and y is written exactly."""
+    bits = I.Workload("t", "linear_nvfp4", M, d, N, 1e-6, seed=M + d + 1).draw()
+    rowb = -(-d // 256) * 144
+    flat_q, q4, n_q = _guarded((N * rowb // 2,), torch.bfloat16)   # the codes' bytes, viewed as int16
+    flat_s, s2, n_s = _guarded((N,), torch.float32)
+    Q4, S2 = q4.view(torch.uint8).view(N, rowb), s2
+    W, g = to_dev(bits["w"]), to_dev(bits["g"])
+    assert fn.load_library().flashnorm_fold_weights_nvfp4(W.data_ptr(), g.data_ptr(), Q4.data_ptr(), S2.data_ptr(),
+                                                          d, N, fn._stream_ptr(W)) == fn.FN_OK
+    ws = None
+    if workspace:
+        need = fn.flashnorm_nvfp4_workspace_bytes(M, d, N)
+        assert need > 1024
+        flat_ws, wsp, n_ws = _guarded((need // 4,), torch.float32)
+        wsp[:256].view(torch.int32).zero_()
+        ws = wsp.view(torch.uint8)
+    flat, y, n = _guarded((M, N), torch.bfloat16)
+    for _ in range(3):
+        fn.flashnorm_linear_nvfp4(to_dev(bits["x"]), Q4, S2, 1e-6, out=y, workspace=ws)
+    torch.cuda.synchronize()
+    assert _intact(flat_q, n_q) and _intact(flat_s, n_s) and _intact(flat, n)
+    if workspace:
+        assert _intact(flat_ws, n_ws) and int(wsp[:256].view(torch.int32).count_nonzero().item()) == 0
+    assert O.rel_err(to_host_f64(y), O.exact_operand_nvfp4(bits, 1e-6)) <= 5e-3
+
+
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_layernorm_decode_writes_stay_in_bounds(out_dtype):
     """LayerNorm at decode size (the tensor-core decode kernel, ragged N, K split over a cluster)."""
