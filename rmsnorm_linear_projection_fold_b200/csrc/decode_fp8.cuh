@@ -135,19 +135,20 @@ __device__ __forceinline__ uint32_t e4m3_pairs_to_bf16x2(uint32_t v) {
   return r;
 }
 
-// Two E2M1 codes, the even k in bits 0..3 of `v` and the odd k in bits 16..19, to bf16x2 times the block
-// scale, exactly. A code s.ee.m has ee at bits 2..1 and m at bit 0; moved to bits 8..7 and 6 (a bf16's low
+// Two E2M1 codes, the even k in bits 0..3 of `v` and the odd k in bits 16..19, to bf16x2 weights times
+// 2^-63, exactly. A code s.ee.m has ee at bits 2..1 and m at bit 0; moved to bits 8..7 and 6 (a bf16's low
 // exponent bits and top mantissa bit), with s at bit 15, the bf16 read from those bits is 2^(ee-127)(1 +
 // m/2) (for ee = 0 the subnormal m 2^-127): 2^-126 times the E2M1 value 2^(ee-1)(1 + m/2) (or m/2). One
-// multiply by 2^126 makes it the E2M1 value, a second by the block scale (an E4M3 value: at most 4
-// significant bits against E2M1's 2) the weight, both exact in bf16.
+// multiply by scale2 = the block scale times 2^63 makes it the weight times 2^-63: at most 6 significant
+// bits (E2M1's 2, E4M3's 4) and, for block scales of 2^-9 .. 448, magnitudes of 2^-73 .. 2^-52, normal in
+// bf16, so the product is exact. The epilogue multiplies the accumulator by 2^63 (kNvfp4Unscale).
 __device__ __forceinline__ uint32_t e2m1_pair_to_bf16x2(uint32_t v, uint32_t scale2) {
   const uint32_t f = ((v & 0x00070007u) << 6) | ((v & 0x00080008u) << 12);
   uint32_t r;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(f), "r"(0x7E807E80u));  // x 2^126
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(r), "r"(scale2));
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(f), "r"(scale2));
   return r;
 }
+constexpr float kNvfp4Unscale = 9223372036854775808.0f;  // 2^63
 
 template <int STAGES, int KSPLIT, bool OUT_F32, int FMT = kFmtFp8>
 __global__ void __launch_bounds__(kD8Threads, 1)
@@ -178,10 +179,12 @@ __global__ void __launch_bounds__(kD8Threads, 1)
   const uint32_t rank = KSPLIT == 0 ? blockIdx.x % static_cast<uint32_t>(ks) : (KSPLIT > 1 ? cluster_ctarank() : 0);
   const int slab = static_cast<int>(blockIdx.x) / ks;
   const int n0 = slab * kD8Rows;
-  const int num_stages = (p.K + F::kKStage - 1) / F::kKStage;  // stages over all of K
-  const int g0 = static_cast<int>((static_cast<long long>(rank) * num_stages) / ks);
-  const int g1 = static_cast<int>((static_cast<long long>(rank + 1) * num_stages) / ks);
-  const int u0 = g0 * F::kUnits, u1 = g1 * F::kUnits;  // this range's 128-k units
+  // this range's 128-k units [u0, u1), split evenly over the ranges; it loads the stages [g0, g1) that
+  // hold them (with NVFP4 a range may start or end in the middle of a 256-k stage)
+  const int num_units = (p.K + F::kKStage - 1) / F::kKStage * F::kUnits;
+  const int u0 = static_cast<int>((static_cast<long long>(rank) * num_units) / ks);
+  const int u1 = static_cast<int>((static_cast<long long>(rank + 1) * num_units) / ks);
+  const int g0 = u0 / F::kUnits, g1 = u1 > u0 ? (u1 + F::kUnits - 1) / F::kUnits : g0;  // an empty range loads nothing
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -268,8 +271,8 @@ __global__ void __launch_bounds__(kD8Threads, 1)
       const uint32_t idesc = make_idesc_bf16(kD8Rows, kD8Tok);
       const uint32_t acc0 = tmem_base + static_cast<uint32_t>(iss * kD8AccPer * kD8Tok);
       bool ok = true;
-      for (int i = iss; u0 + i < u1; i += kD8Issuers) {  // unit i of the range: stage i / F::kUnits
-        const int st = i / F::kUnits;
+      for (int i = iss; u0 + i < u1; i += kD8Issuers) {  // unit i of the range
+        const int u = u0 + i, st = u / F::kUnits - g0;   // its stage, counted from the range's first
         const int s = st % STAGES, b = i % kD8ABufs;
         const uint32_t ph = static_cast<uint32_t>(st / STAGES) & 1u, bph = static_cast<uint32_t>(i / kD8ABufs) & 1u;
         // the x tile of this stage (TMA) and the widened codes in A buffer b (the converters)
@@ -279,7 +282,7 @@ __global__ void __launch_bounds__(kD8Threads, 1)
         }
         tc_fence_after_sync();
         const uint32_t a_col = tmem_base + static_cast<uint32_t>(kD8ACol0 + b * 64);
-        const uint32_t x_st = smem_u32(sX + s * F::kXStage + (i % F::kUnits) * kD8XStage);
+        const uint32_t x_st = smem_u32(sX + s * F::kXStage + (u % F::kUnits) * kD8XStage);
 #pragma unroll
         for (int j = 0; j < kD8KStage / 16; ++j)  // 8 MMAs of K = 16: 8 columns of A, 32 bytes of a B row
           tc_mma_bf16_ts(acc0 + static_cast<uint32_t>((j % kD8AccPer) * kD8Tok), a_col + j * 8,
@@ -306,8 +309,8 @@ __global__ void __launch_bounds__(kD8Threads, 1)
     float ss = 0.f;
     // this row's dequantization scale, loaded now so that its latency hides under the main loop
     const float sc = n0 + row < p.N ? p.scales[n0 + row] : 0.f;
-    for (int i = 0; u0 + i < u1; ++i) {  // unit i of the range: half `half` of stage i / F::kUnits
-      const int st = i / F::kUnits, half = i % F::kUnits;
+    for (int i = 0; u0 + i < u1; ++i) {  // unit i of the range: half `half` of its stage
+      const int u = u0 + i, st = u / F::kUnits - g0, half = u % F::kUnits;
       const int s = st % STAGES, b = i % kD8ABufs;
       const uint32_t ph = static_cast<uint32_t>(st / STAGES) & 1u, bph = static_cast<uint32_t>(i / kD8ABufs) & 1u;
       if (!mbar_wait(&full[s], ph, abort_flag) || !mbar_wait(&aempty[b], bph ^ 1u, abort_flag)) {
@@ -350,7 +353,8 @@ __global__ void __launch_bounds__(kD8Threads, 1)
             for (int e = 0; e < 2; ++e) {
               const int bb = q2 * 4 + c * 2 + e;  // block of this unit: columns 8 bb .. 8 bb + 7
               const uint32_t sbyte = ((bb < 4 ? scw.x : scw.y) >> (8 * (bb & 3))) & 0xFFu;
-              const uint32_t sbf = e4m3_pairs_to_bf16x2(sbyte | (sbyte << 16));  // the scale in both halves
+              uint32_t sbf = e4m3_pairs_to_bf16x2(sbyte | (sbyte << 16));  // the scale in both halves
+              asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(sbf) : "r"(sbf), "r"(0x5F005F00u));  // x 2^63, exact
 #pragma unroll
               for (int wi = 0; wi < 2; ++wi)
 #pragma unroll
@@ -379,7 +383,11 @@ __global__ void __launch_bounds__(kD8Threads, 1)
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) {
-        if (half == F::kUnits - 1) mbar_arrive(&empty[s]);  // the stage's last unit: its codes are read
+        // the stage's last unit of this range: its codes are read. A stage of which this range takes one
+        // unit of two gets one MMA commit instead of two; one converter warp arrives in its place.
+        if (half == F::kUnits - 1 || u == u1 - 1) mbar_arrive(&empty[s]);
+        const bool alone = F::kUnits == 2 && ((half == 0 && u == u1 - 1) || (half == 1 && u == u0));
+        if (alone && warp == 2) mbar_arrive(&empty[s]);
         mbar_arrive(&afull[b]);
       }
     }
@@ -412,6 +420,10 @@ __global__ void __launch_bounds__(kD8Threads, 1)
       for (int j = 0; j < kD8Tok; ++j)
         v[j] = ((w0 ? __uint_as_float(r0[j]) : 0.f) + (w1 ? __uint_as_float(r1[j]) : 0.f)) +
                ((w2 ? __uint_as_float(r2[j]) : 0.f) + (w3 ? __uint_as_float(r3[j]) : 0.f));
+      if constexpr (FMT == kFmtNvfp4) {
+#pragma unroll
+        for (int j = 0; j < kD8Tok; ++j) v[j] *= kNvfp4Unscale;  // the A operand held weights x 2^-63: exact
+      }
     } else {
       // an empty K range contributes zero; a wait that gave up contributes NaN
 #pragma unroll
