@@ -21,12 +21,18 @@ def test_metric_units_prefill_and_decode():
     assert bench._is_decode(dec) and bench._units(dec) == 2 * 4096 * 12288
     fp8 = [I.WORKLOADS["llama7b_qkv_fp8_m4"]]
     assert bench._units(fp8) == 4096 * 12288 + 4 * 12288  # one byte per weight plus the channel scales
+    nv4 = [I.WORKLOADS["llama7b_qkv_nvfp4_m4"]]
+    # half a byte per weight, one E4M3 scale per 16 weights, a fp32 scale per channel
+    assert bench._units(nv4) == 12288 * (4096 // 2 + 4096 // 16 + 4)
 
 
 def test_step_bytes_follow_the_weight_format():
     w16, w8 = I.WORKLOADS["llama7b_qkv_m4"], I.WORKLOADS["llama7b_qkv_fp8_m4"]
     assert bench._set_bytes(w16) - bench._set_bytes(w8) == 4096 * 12288 - 4 * 12288
     assert w8.bytes == 2 * (4 * 4096 + 4 * 12288) + 4096 * 12288 + 4 * 12288
+    w4 = I.WORKLOADS["llama7b_qkv_nvfp4_m4"]
+    assert w4.bytes == 2 * (4 * 4096 + 4 * 12288) + 12288 * (2048 + 256 + 4)
+    assert bench._set_bytes(w8) - bench._set_bytes(w4) == 12288 * (4096 - 2048 - 256)
 
 
 def test_reference_sample_shrinks_and_still_runs_the_oracle():
@@ -64,3 +70,16 @@ def test_gpu_count_must_match_the_ranks():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference"],
                        capture_output=True, text=True, env=env, timeout=120)
     assert r.returncode == 2 and "WORLD_SIZE=1" in r.stderr
+
+
+def test_nvfp4_sample_runs_the_oracle():
+    """The NVFP4 decode workload's CPU baseline decodes a bounded channel sample with the oracle."""
+    wl = "llama7b_qkv_nvfp4_m1"
+    bench._ORACLE_CACHE.pop(wl, None)
+    _, decode, projs = bench._oracle_setup(wl)
+    assert decode and projs[0]["chans"] == 1024
+    bench._shrink_sample(wl, 1 / 16)
+    assert projs[0]["chans"] == 64 and bench._pass_units(projs[0], True) == 64 * (2048 + 256 + 4)
+    y = projs[0]["call"](projs[0]["rows"], projs[0]["chans"])
+    assert y.shape == (1, 64) and np.isfinite(y).all()
+    bench._ORACLE_CACHE.pop(wl, None)
