@@ -102,19 +102,20 @@ E2E_PIPELINE_BYTES = 1 << 20
 # hash differently now, traffic is reported as null.
 NCU_TRAFFIC = {
     # workload: (bytes per launch, sha256[:16] of the csrc/*.cu* sources at capture time)
-    "llama7b_ffn_m2048": (854593024, "9df93328d7be0c0a"),
-    "llama7b_qkv_m2048": (502012928, "9df93328d7be0c0a"),
-    "smollm2_ffn_m8192": (13023488, "9df93328d7be0c0a"),
-    "layernorm_qkv_m8192": (10594048, "9df93328d7be0c0a"),
-    "smollm2_qkv_m64": (1216000, "9df93328d7be0c0a"),
-    "gemma_qkvnorm_hd256_m2048": (31505408, "9df93328d7be0c0a"),
-    "gemma_qkvnorm_rope_hd256_m2048": (33614592, "9df93328d7be0c0a"),
-    "llama7b_qkv_m16": (104636160, "9df93328d7be0c0a"),
-    "layernorm_llama7b_qkv_m4": (104762624, "9df93328d7be0c0a"),
-    "llama7b_qkv_gemv_m16": (104215552, "9df93328d7be0c0a"),
-    "llama7b_qkv_fp8_m1": (50429440, "9df93328d7be0c0a"),
-    "llama7b_qkv_fp8_m4": (50467072, "9df93328d7be0c0a"),
-    "mla_latent_cluster_m2048": (26264320, "9df93328d7be0c0a"),
+    "llama7b_ffn_m2048": (849488384, "b61f1891bc6108ab"),
+    "llama7b_qkv_m2048": (505464064, "b61f1891bc6108ab"),
+    "smollm2_ffn_m8192": (13033728, "b61f1891bc6108ab"),
+    "layernorm_qkv_m8192": (10594048, "b61f1891bc6108ab"),
+    "smollm2_qkv_m64": (1216000, "b61f1891bc6108ab"),
+    "gemma_qkvnorm_hd256_m2048": (31520000, "b61f1891bc6108ab"),
+    "gemma_qkvnorm_rope_hd256_m2048": (33616384, "b61f1891bc6108ab"),
+    "llama7b_qkv_m16": (105891072, "b61f1891bc6108ab"),
+    "layernorm_llama7b_qkv_m4": (104253952, "b61f1891bc6108ab"),
+    "llama7b_qkv_gemv_m16": (104263936, "b61f1891bc6108ab"),
+    "llama7b_qkv_fp8_gemv_m1": (50441472, "b61f1891bc6108ab"),
+    "llama7b_qkv_fp8_m4": (50468352, "b61f1891bc6108ab"),
+    "llama7b_qkv_nvfp4_m4": (28435200, "b61f1891bc6108ab"),
+    "mla_latent_cluster_m2048": (26264320, "b61f1891bc6108ab"),
 }
 
 # The dominant-kernel loop and each block of the fused/unfused comparison run at least this many
