@@ -83,3 +83,22 @@ def test_nvfp4_sample_runs_the_oracle():
     y = projs[0]["call"](projs[0]["rows"], projs[0]["chans"])
     assert y.shape == (1, 64) and np.isfinite(y).all()
     bench._ORACLE_CACHE.pop(wl, None)
+
+
+def test_reference_arm_on_a_quantized_workload():
+    """bench.py --impl reference on the NVFP4 decode workload: one JSON line, the oracle on the host cores,
+    in the GPU arm's metric and unit."""
+    import json
+    import subprocess
+
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3", "--workload", "llama7b_qkv_nvfp4_m4"],
+                       capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["config"]["workload"] == "llama7b_qkv_nvfp4_m4"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
