@@ -102,20 +102,20 @@ E2E_PIPELINE_BYTES = 1 << 20
 # hash differently now, traffic is reported as null.
 NCU_TRAFFIC = {
     # workload: (bytes per launch, sha256[:16] of the csrc/*.cu* sources at capture time)
-    "llama7b_ffn_m2048": (849488384, "b61f1891bc6108ab"),
-    "llama7b_qkv_m2048": (505464064, "b61f1891bc6108ab"),
-    "smollm2_ffn_m8192": (13033728, "b61f1891bc6108ab"),
-    "layernorm_qkv_m8192": (10594048, "b61f1891bc6108ab"),
-    "smollm2_qkv_m64": (1216000, "b61f1891bc6108ab"),
-    "gemma_qkvnorm_hd256_m2048": (31520000, "b61f1891bc6108ab"),
-    "gemma_qkvnorm_rope_hd256_m2048": (33616384, "b61f1891bc6108ab"),
-    "llama7b_qkv_m16": (105891072, "b61f1891bc6108ab"),
-    "layernorm_llama7b_qkv_m4": (104253952, "b61f1891bc6108ab"),
-    "llama7b_qkv_gemv_m16": (104263936, "b61f1891bc6108ab"),
-    "llama7b_qkv_fp8_gemv_m1": (50441472, "b61f1891bc6108ab"),
-    "llama7b_qkv_fp8_m4": (50468352, "b61f1891bc6108ab"),
-    "llama7b_qkv_nvfp4_m4": (28435200, "b61f1891bc6108ab"),
-    "mla_latent_cluster_m2048": (26264320, "b61f1891bc6108ab"),
+    "llama7b_ffn_m2048": (810606848, "bd7602d07f59d4e1"),
+    "llama7b_qkv_m2048": (476248832, "bd7602d07f59d4e1"),
+    "smollm2_ffn_m8192": (13025024, "bd7602d07f59d4e1"),
+    "layernorm_qkv_m8192": (10594304, "bd7602d07f59d4e1"),
+    "smollm2_qkv_m64": (1216256, "bd7602d07f59d4e1"),
+    "gemma_qkvnorm_hd256_m2048": (31504640, "bd7602d07f59d4e1"),
+    "gemma_qkvnorm_rope_hd256_m2048": (33604608, "bd7602d07f59d4e1"),
+    "llama7b_qkv_m16": (104403456, "bd7602d07f59d4e1"),
+    "layernorm_llama7b_qkv_m4": (104041728, "bd7602d07f59d4e1"),
+    "llama7b_qkv_gemv_m16": (104177920, "bd7602d07f59d4e1"),
+    "llama7b_qkv_fp8_gemv_m1": (50477568, "bd7602d07f59d4e1"),
+    "llama7b_qkv_fp8_m4": (52099072, "bd7602d07f59d4e1"),
+    "llama7b_qkv_nvfp4_m4": (30008064, "bd7602d07f59d4e1"),
+    "mla_latent_cluster_m2048": (26264576, "bd7602d07f59d4e1"),
 }
 
 # The dominant-kernel loop and each block of the fused/unfused comparison run at least this many

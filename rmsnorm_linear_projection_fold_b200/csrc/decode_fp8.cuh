@@ -442,9 +442,10 @@ __global__ void __launch_bounds__(kD8Threads, 1)
       // to arrive adds them all, range 0 first (the same order whichever range comes last)
       const size_t rec = static_cast<size_t>(slab) * static_cast<size_t>(ks);  // the slab's first record
       float* mine = p.part + ((rec + rank) * kD8Rows + row) * kD8Tok;
+      // only the token slots the call has (groups of four below M): the slots past M are never read
 #pragma unroll
       for (int j = 0; j < kD8Tok; j += 4)
-        __stcg(reinterpret_cast<float4*>(mine + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
+        if (j < p.M) __stcg(reinterpret_cast<float4*>(mine + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
       if (sub == 0) __stcg(p.part_ss + (rec + rank) * kD8Tok + tok, ss);
       named_bar_sync(1, 128);  // the CTA's partials come before its arrival (barrier, then release)
       if (t == 0) {
@@ -468,7 +469,7 @@ __global__ void __launch_bounds__(kD8Threads, 1)
             const float* src = p.part + ((rec + rr) * kD8Rows + row) * kD8Tok;
 #pragma unroll
             for (int j = 0; j < kD8Tok; j += 4) {
-              const float4 f = __ldcg(reinterpret_cast<const float4*>(src + j));
+              const float4 f = j < p.M ? __ldcg(reinterpret_cast<const float4*>(src + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
               q[j] = f.x, q[j + 1] = f.y, q[j + 2] = f.z, q[j + 3] = f.w;
             }
           }
