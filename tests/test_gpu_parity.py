@@ -396,16 +396,20 @@ def test_cuda_graph_replay_matches_eager():
     dc = _wl("linear", 4, 1024, 1024, seed=32).draw()
     gl = _wl("glu", 300, 576, 1536, seed=33).draw()
     f8 = I.Workload("t", "linear_fp8", 5, 1024, 768, 1e-6, seed=34).draw()
+    f4 = I.Workload("t", "linear_nvfp4", 3, 1536, 1024, 1e-6, seed=35).draw()
     W_pn, g2 = _fold(pn, False), to_dev(pn["g2"])
     W_dc, W_gl = _fold(dc, False), _fold(gl, True)
     Q, sc = fn.flashnorm_fold_weights_fp8(to_dev(f8["w"]), to_dev(f8["g"]))
+    Q4, s2 = fn.flashnorm_fold_weights_nvfp4(to_dev(f4["w"]), to_dev(f4["g"]))
     x_pn, x_dc, x_gl, x_f8 = to_dev(pn["x"]), to_dev(dc["x"]), to_dev(gl["x"]), to_dev(f8["x"])
+    x_f4 = to_dev(f4["x"])
 
     def step():
         return (fn.flashnorm_linear_postnorm(x_pn, W_pn, g2, 512, 1e-6, out_dtype=torch.float32),
                 fn.flashnorm_linear(x_dc, W_dc, 1e-5),
                 fn.flashnorm_linear_fp8(x_f8, Q, sc, 1e-6),
-                fn.flashnorm_glu(x_gl, W_gl, 1e-5))
+                fn.flashnorm_glu(x_gl, W_gl, 1e-5),
+                fn.flashnorm_linear_nvfp4(x_f4, Q4, s2, 1e-6, out_dtype=torch.float32))
 
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -417,7 +421,7 @@ def test_cuda_graph_replay_matches_eager():
     with torch.cuda.graph(g):
         outs = step()
     for t in range(3):
-        for x, m, d in ((x_pn, 256, 1024), (x_dc, 4, 1024), (x_gl, 300, 576), (x_f8, 5, 1024)):
+        for x, m, d in ((x_pn, 256, 1024), (x_dc, 4, 1024), (x_gl, 300, 576), (x_f8, 5, 1024), (x_f4, 3, 1536)):
             x.copy_(to_dev(I.activations(m, d, 4000 + 10 * t + d % 7)))
         g.replay()
         torch.cuda.synchronize()
@@ -431,6 +435,9 @@ def test_cuda_graph_replay_matches_eager():
     b = dict(pn, x=I.activations(256, 1024, 4000 + 20 + 1024 % 7))
     ex = O.exact_operand_output("postnorm", b, O.fold_bf16(pn["w"], pn["g"]), 1e-6, eps2=1e-6, head_dim=512)
     assert O.rel_err(to_host_f64(outs[0]), ex) <= F32_TOL
+    # and the replayed NVFP4 output (its workspace counters went through every replay) the oracle's
+    b4 = dict(f4, x=I.activations(3, 1536, 4000 + 20 + 1536 % 7))
+    assert O.rel_err(to_host_f64(outs[4]), O.exact_operand_nvfp4(b4, 1e-6)) <= F32_TOL
     del g
 
 

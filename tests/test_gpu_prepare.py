@@ -23,18 +23,21 @@ def _cases():
     glu = I.Workload("t", "glu", 300, 576, 768, 1e-5, seed=62).draw()
     pn = I.Workload("t", "postnorm", 256, 2048, 1024, 1e-6, head_dim=512, eps2=1e-6, seed=63).draw()
     f8 = I.Workload("t", "linear_fp8", 5, 4096, 12288, 1e-6, seed=64).draw()
+    f4 = I.Workload("t", "linear_nvfp4", 4, 4096, 12288, 1e-6, seed=65).draw()
     W_lin = fn.flashnorm_fold_weights(to_dev(lin["w"]), to_dev(lin["g"]))
     W_glu = fn.flashnorm_fold_weights(to_dev(glu["w"]), to_dev(glu["g"]), glu=True)
     W_pn, g2 = fn.flashnorm_fold_weights(to_dev(pn["w"]), to_dev(pn["g"])), to_dev(pn["g2"])
     Q, sc = fn.flashnorm_fold_weights_fp8(to_dev(f8["w"]), to_dev(f8["g"]))
-    xs = {k: to_dev(b["x"]) for k, b in (("lin", lin), ("glu", glu), ("pn", pn), ("f8", f8))}
+    Q4, s2 = fn.flashnorm_fold_weights_nvfp4(to_dev(f4["w"]), to_dev(f4["g"]))
+    xs = {k: to_dev(b["x"]) for k, b in (("lin", lin), ("glu", glu), ("pn", pn), ("f8", f8), ("f4", f4))}
     calls = {
         "lin": (fn.flashnorm_linear, (xs["lin"], W_lin, 1e-5), {}),
         "glu": (fn.flashnorm_glu, (xs["glu"], W_glu, 1e-5), {}),
         "pn": (fn.flashnorm_linear_postnorm, (xs["pn"], W_pn, g2, 512, 1e-6), {"out_dtype": torch.float32}),
         "f8": (fn.flashnorm_linear_fp8, (xs["f8"], Q, sc, 1e-6), {"out_dtype": torch.float32}),
+        "f4": (fn.flashnorm_linear_nvfp4, (xs["f4"], Q4, s2, 1e-6), {"out_dtype": torch.float32}),
     }
-    return xs, calls, {"pn": pn, "f8": f8}
+    return xs, calls, {"pn": pn, "f8": f8, "f4": f4}
 
 
 def test_prepared_calls_match_direct_calls():
@@ -61,12 +64,15 @@ def test_prepared_call_keeps_its_workspace():
     p_pn = fn.prepare(f, *a, **kw)
     f, a, kw = calls["f8"]
     p_f8 = fn.prepare(f, *a, **kw)
+    f, a, kw = calls["f4"]
+    p_f4 = fn.prepare(f, *a, **kw)
     fn._fp8_ws_cache.clear()
     gc.collect()
     torch.cuda.empty_cache()
     filler = torch.full((64 << 20,), 0x7F, dtype=torch.uint8, device="cuda")  # reuse any freed blocks
     y_pn = p_pn()
     y_f8 = p_f8()
+    y_f4 = p_f4()
     torch.cuda.synchronize()
     del filler
     pn, f8 = bits["pn"], bits["f8"]
@@ -74,3 +80,4 @@ def test_prepared_call_keeps_its_workspace():
     ex_pn = O.exact_operand_output("postnorm", pn, W, 1e-6, eps2=1e-6, head_dim=512)
     assert O.rel_err(to_host_f64(y_pn), ex_pn) <= 1e-5
     assert O.rel_err(to_host_f64(y_f8), O.exact_operand_fp8(f8, 1e-6)) <= 1e-5
+    assert O.rel_err(to_host_f64(y_f4), O.exact_operand_nvfp4(bits["f4"], 1e-6)) <= 1e-5
