@@ -436,7 +436,8 @@ def flashnorm_linear_fp8(x: torch.Tensor, Q: torch.Tensor, scales: torch.Tensor,
     if isinstance(workspace, str):
         if workspace != "auto":
             raise ValueError('workspace must be "auto", None or a uint8 CUDA tensor')
-        nbytes = flashnorm_fp8_workspace_bytes(M, d, N, x.get_device()) if 0 < M <= 16 else 0
+        # the CUDA-core GEMV takes no workspace
+        nbytes = flashnorm_fp8_workspace_bytes(M, d, N, x.get_device()) if 0 < M <= 16 and path != "gemv" else 0
         ws = _fp8_stream_workspace(x, nbytes) if nbytes > 0 else None
     elif workspace is None:
         ws = None
