@@ -18,6 +18,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import threading
 
 import torch
 
@@ -153,15 +154,20 @@ def _invoke(entry: str, lead: torch.Tensor, *args, report: str | None = None) ->
     _invoke_on(lead.get_device(), entry, *args, report=report)
 
 
-# While prepare() records: the library calls made (size queries excepted) and every tensor whose address
-# was taken, which the prepared call keeps alive.
-_recording = None
-_recording_keep = None
+# While prepare() records, on its own thread: the library calls made (size queries excepted) and every
+# tensor whose address was taken, which the prepared call keeps alive. Thread-local, so that calls made by
+# other threads meanwhile run as usual.
+_rec = threading.local()
+
+
+def _recording():
+    return getattr(_rec, "calls", None)
 
 
 def _invoke_on(dev: int, entry: str, *args, report: str | None = None) -> None:
-    if _recording is not None and not entry.endswith("_workspace_bytes"):
-        _recording.append((dev, entry, args, report or entry))
+    calls = _recording()
+    if calls is not None and not entry.endswith("_workspace_bytes"):
+        calls.append((dev, entry, args, report or entry))
         return
     lib = load_library()
     if dev == torch.cuda.current_device():
@@ -187,8 +193,9 @@ def _ptr(t):
     """A tensor's device address for a void* argument (None passes NULL)."""
     if t is None:
         return None
-    if _recording_keep is not None:
-        _recording_keep.append(t)
+    keep = getattr(_rec, "keep", None)
+    if keep is not None:
+        keep.append(t)
     return t.data_ptr()
 
 
@@ -220,15 +227,14 @@ def prepare(func, *args, **kwargs) -> PreparedCall:
     on the same buffers (a serving step, a benchmark). What is fixed at this point: the device addresses
     (rewrite the inputs in place, and read the outputs from .result), the stream (the one current now),
     and any scratch the call chose (a workspace="auto" buffer is allocated here and kept)."""
-    global _recording, _recording_keep
-    if _recording is not None:
+    if _recording() is not None:
         raise RuntimeError("prepare() does not nest")
     rec, keep = [], []
-    _recording, _recording_keep = rec, keep
+    _rec.calls, _rec.keep = rec, keep
     try:
         result = func(*args, **kwargs)
     finally:
-        _recording, _recording_keep = None, None
+        _rec.calls, _rec.keep = None, None
     if len(rec) != 1:
         raise ValueError(f"prepare() takes a call that makes one library call; this one made {len(rec)}")
     dev, entry, cargs, report = rec[0]

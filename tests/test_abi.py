@@ -282,7 +282,22 @@ def test_prepare_propagates_errors_and_resets():
     for _ in range(2):
         with pytest.raises((ValueError, TypeError, fn.FlashNormError)):
             fn.prepare(fn.flashnorm_linear, x, x, 1e-5)
-    assert fn._recording is None and fn._recording_keep is None
+    assert fn._recording() is None and getattr(fn._rec, "keep", None) is None
+
+
+def test_prepare_recording_is_per_thread():
+    """While one thread records a call for prepare(), library calls of other threads are not captured."""
+    import threading
+
+    seen = {}
+    fn._rec.calls, fn._rec.keep = [], []
+    try:
+        t = threading.Thread(target=lambda: seen.setdefault("other", fn._recording()))
+        t.start()
+        t.join()
+        assert seen["other"] is None and fn._recording() == []
+    finally:
+        fn._rec.calls, fn._rec.keep = None, None
 
 
 def test_nvfp4_validation(lib):
