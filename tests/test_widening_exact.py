@@ -49,3 +49,24 @@ def test_e2m1_widening_times_block_scale_is_exact():
             prod = _bf16(bits) * scale63        # exact in fp64: at most 6 significant bits
             assert _bf16_exact(prod), (c, s)    # so the bf16 multiply returns it unrounded
             assert prod == want * float(scales[s]) * 2.0 ** -63
+
+
+def _e2m1_by_midpoints(t: np.ndarray) -> np.ndarray:
+    """The fold kernel's E2M1 rounding (fp8.cuh, e2m1_rn_satfinite): the count of midpoints a magnitude passes,
+    strict where the lower neighbour has the even code, inclusive where the upper one has, and the sign bit."""
+    a = np.abs(t)
+    m = ((a > 0.25).astype(np.uint8) + (a >= 0.75) + (a > 1.25) + (a >= 1.75) + (a > 2.5) + (a >= 3.5) + (a > 5.0))
+    return (m | np.where(np.signbit(t), 8, 0)).astype(np.uint8)
+
+
+def test_e2m1_rounding_by_midpoints_matches_the_oracle():
+    """Every midpoint between neighbouring E2M1 magnitudes, its float32 neighbours on both sides, both signs, and
+    random values: the comparison form and the oracle's round-to-nearest-even agree code for code."""
+    from oracle import flashnorm_oracle as O
+
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], dtype=np.float32)
+    around = np.concatenate([mids, np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(10)),
+                             np.array(E2M1_TABLE, dtype=np.float32), np.array([6.5, 100.0, 3e38], dtype=np.float32)])
+    rng = np.random.default_rng(3)
+    vals = np.concatenate([around, -around, rng.uniform(-8, 8, 20000).astype(np.float32), np.float32([0.0, -0.0])])
+    assert np.array_equal(_e2m1_by_midpoints(vals), O.f64_to_e2m1(vals.astype(np.float64)))
